@@ -1,0 +1,31 @@
+"""The seeded generator is deterministic and per-sequence streams are independent."""
+import numpy as np
+
+from compressed_sparse_attention_quantize_b200 import synth
+
+
+def test_deterministic_and_shapes():
+    wl = synth.workload(0)
+    a = synth.kv_latent(wl, 0)
+    b = synth.kv_latent(wl, 0)
+    assert a.shape == (1024, 512) and a.dtype == np.float32 and np.array_equal(a, b)
+    oc = synth.outlier_channels(wl.seed)
+    assert len(set(oc.tolist())) == 4
+    assert np.abs(a[:, oc]).mean() > 5 * np.abs(np.delete(a, oc, axis=1)).mean()
+    assert synth.main_query_bf16(wl, 0, 0).shape == (1, 16, 512)
+    assert synth.index_query(wl, 0, 0).shape == (1, 4, 64)
+    w = synth.head_weights(wl, 0, 0)
+    assert w.shape == (1, 4) and (w >= 0).all() and (w < 1).all()
+
+
+def test_workloads():
+    w3 = synth.workload(3)
+    assert w3.B == 4 and all(131072 <= n <= 262144 for n in w3.n_entries)
+    w4 = synth.workload(4)
+    nv = w4.n_visible(0)
+    assert nv[0] == 32768 and nv[-1] == 33792
+    st, ln = synth.swa_window(w4, 0)
+    assert st[0] == 0 and ln[0] == 128 and st[-1] == 4095
+    w1 = synth.workload(1)
+    st, ln = synth.swa_window(w1, 0)
+    assert ln[0] == 128 and w1.modes == ("F", "U", "U", "U", "U", "U")
