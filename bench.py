@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""CSA2 hot-path benchmark: decode queries/s of one CSA2 layer group on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference] [--config C]
+
+One step = one decode token of every sequence of the workload through the whole layer group
+(indexer + top-K of the Full layer, then attention of all six layers), i.e. every hot-path
+step.  Default workload: decode at 128K context, batch 32, 1 Full + 5 Reuse layers.
+
+Printed (rank 0, one JSON line): value = queries/s over all ranks (device time, CUDA events on
+the launch stream, L2 flushed by a 256 MB write between steps, max over ranks); e2e = the same
+metric through csa2_layer_group with host buffers (host->device copies of the step's queries and
+the device->host read of the last layer's output inside the timed region); roofline of the
+dominant kernel; cpu_baseline = the oracle on the host cores over a bounded sample.
+
+With --gpus N > 1 (torchrun) every rank runs its own replica of the workload (independent
+sequences; the decode path has no exchange step), so scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode queries/sec at 128K and 1M ctx; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "queries/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# algorithmic work per call (bytes that must move; flops of the contraction)
+# ------------------------------------------------------------------------------------------
+def attn_work(wl, out_bytes):
+    """Bytes and flops of one csa2_sparse_attn call over the workload."""
+    from compressed_sparse_attention_quantize_b200 import synth
+    byts = 0
+    flops = 0
+    for b in range(wl.B):
+        nvis = wl.n_visible(b)
+        _, swl = synth.swa_window(wl, b)
+        for t in range(wl.T):
+            sel = min(wl.K, int(nvis[t]))
+            keys = sel + int(swl[t])
+            byts += sel * 288 + int(swl[t]) * 516 + wl.H * 512 * (2 + out_bytes) + wl.K * 4 + wl.H * 4
+            flops += wl.H * keys * 512 * 4
+    return byts, flops
+
+
+def index_work(wl):
+    """Bytes of one Full-mode csa2_index_topk call (keys scanned + queries + selection written)."""
+    byts = 0
+    for b in range(wl.B):
+        nvis = wl.n_visible(b)
+        for t in range(wl.T):
+            byts += int(nvis[t]) * 36 + wl.HI * 40 + wl.K * 4
+            if wl.P:
+                byts += wl.P * 4
+    return byts
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        self.f.close()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[3]) or 0.0 for r in rows]
+        pmax = max(power) if power else 0.0
+        loaded = [num(r[1]) for r, p in zip(rows, power) if p >= 0.5 * pmax and num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded or sm) if sm else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": reasons, "samples": len(rows),
+                "power_w_max": pmax}
+
+
+# ------------------------------------------------------------------------------------------
+# reference arm / CPU baseline: the oracle on the host cores
+# ------------------------------------------------------------------------------------------
+def oracle_sample(wl, rows, softmax_scale):
+    """Run the oracle over `rows` query rows (setup outside, returns elapsed seconds of the
+    per-query work: indexer scores, top-K, pool/Reindex, attention of every layer)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tests._parity import OracleSeq
+    seqs = {}
+    for r in rows:
+        b, t = divmod(r, wl.T)
+        if b not in seqs:
+            s = OracleSeq(wl, b)
+            for l in range(len(wl.modes)):
+                s.layer(l)
+            seqs[b] = s
+    t0 = time.perf_counter()
+    for r in rows:
+        b, t = divmod(r, wl.T)
+        sel = seqs[b].indices(t, wl.modes)
+        for l in range(len(wl.modes)):
+            seqs[b].attention(l, t, sel[l][0], softmax_scale)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, softmax_scale, budget_s=15.0):
+    import oracle
+    oracle.build()
+    t1 = oracle_sample(wl, [0], softmax_scale)
+    n = max(1, min(wl.B * wl.T, int(budget_s / max(t1, 1e-3))))
+    rows = list(range(1, 1 + n)) if n + 1 <= wl.B * wl.T else list(range(n))
+    el = oracle_sample(wl, rows, softmax_scale)
+    return {"value": len(rows) / el, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} query rows of '{wl.name}' through all {len(wl.modes)} layers "
+                      f"(indexer over every visible entry, top-K, attention per layer); "
+                      f"oracle-side cache quantisation not timed"}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    scale = 1.0 / math.sqrt(512)
+    # one step = a bounded sample of the workload (a single query row through every layer)
+    for w in range(args.warmup):
+        oracle_sample(wl, [w % (wl.B * wl.T)], scale)
+    tot = 0.0
+    for k in range(args.steps):
+        tot += oracle_sample(wl, [k % (wl.B * wl.T)], scale)
+    value = args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64/f32 (oracle)", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "ctx_tokens": wl.ctx_tokens[0],
+                       "layers": ",".join(wl.modes), "heads": wl.H, "topk": wl.K,
+                       "step": "one query row through every layer (bounded sample)"},
+            "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "value": value,
+                             "unit": UNIT, "sample": "one query row per step through every layer"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+# the CUDA arm
+# ------------------------------------------------------------------------------------------
+def time_steps(torch, step, steps, flush):
+    """Per-step CUDA-event times (ms) with an L2 flush before every step (outside the events)."""
+    st = torch.cuda.current_stream()
+    evs = []
+    for _ in range(steps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        step()
+        e1.record(st)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def breakdown(torch, csa2, runner, steps, flush):
+    """Per-call device times of the decomposed group: csa2_index_topk + csa2_sparse_attn per layer."""
+    wl = runner.wl
+    g = runner.g
+    dev = runner.workspace.device
+    rows = runner.rows
+    idx = torch.empty((rows, wl.K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((rows,), dtype=torch.int32, device=dev)
+    P = wl.P if "I" in runner.modes else 0
+    pool = torch.empty((rows, max(P, 1)), dtype=torch.int32, device=dev)
+    pool_len = torch.empty((rows,), dtype=torch.int32, device=dev)
+    iws_bytes = max(csa2.csa2_index_topk_workspace_size(0, rows, runner.max_n, wl.K, P),
+                    csa2.csa2_index_topk_workspace_size(1, rows, runner.max_n, wl.K, max(P, 1)))
+    iws = torch.empty((iws_bytes,), dtype=torch.uint8, device=dev)
+    aws_bytes = csa2.csa2_sparse_attn_workspace_size(rows, wl.H, wl.K)
+    aws = torch.empty((aws_bytes,), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    times = {"index_topk": [], "reindex_topk": [], "sparse_attn": []}
+    for _ in range(steps):
+        flush()
+        marks = []
+        def ev():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(st)
+            return e
+        for l, m in enumerate(runner.modes):
+            ld = runner.layer_data[l]
+            if m != "U":
+                e0 = ev()
+                if m == "F":
+                    csa2.csa2_index_topk(0, ld["iq_codes"], ld["iq_scales"], ld["iw"], wl.B, wl.T, wl.HI,
+                                         runner.k_codes, 32, runner.k_scales, 4, runner.seq_start,
+                                         runner.n_entries, runner.max_n, runner.q_pos, None, None, 0,
+                                         wl.K, idx, cnt, P, pool if P else None, pool_len if P else None,
+                                         iws, iws_bytes)
+                    marks.append(("index_topk", e0, ev()))
+                else:
+                    csa2.csa2_index_topk(1, ld["iq_codes"], ld["iq_scales"], ld["iw"], wl.B, wl.T, wl.HI,
+                                         runner.k_codes, 32, runner.k_scales, 4, runner.seq_start,
+                                         runner.n_entries, runner.max_n, runner.q_pos, pool, pool_len, P,
+                                         wl.K, idx, cnt, 0, None, None, iws, iws_bytes)
+                    marks.append(("reindex_topk", e0, ev()))
+            e0 = ev()
+            csa2.csa2_sparse_attn(ld["q"], wl.B, wl.T, wl.H, 512, runner.kv, 288, runner.seq_start, idx, cnt,
+                                  wl.K, ld["swa_codes"], ld["swa_scale"], runner.swa_cap, runner.swa_start,
+                                  runner.swa_len, runner.softmax_scale, ld["out"], runner.out_dtype, ld["lse"],
+                                  aws, aws_bytes)
+            marks.append(("sparse_attn", e0, ev()))
+        torch.cuda.synchronize()
+        for name, a, b in marks:
+            times[name].append(a.elapsed_time(b))
+    return {k: v for k, v in times.items() if v}
+
+
+def e2e_measure(torch, csa2, runner, steps, warmup, flush):
+    """The metric through csa2_layer_group with host buffers: per step copy every layer's main
+    query (bf16) and indexer query/weights (fp32) from pinned host memory, quantise the indexer
+    queries on the device, run the group, read the last layer's output back."""
+    from compressed_sparse_attention_quantize_b200 import runtime, synth
+    wl = runner.wl
+    host = []
+    h2d = 0
+    for l, m in enumerate(runner.modes):
+        ld = runner.layer_data[l]
+        hq = ld["q"].cpu().pin_memory()
+        e = {"q": hq}
+        h2d += hq.numel() * 2
+        if m != "U":
+            iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
+            e["iq"] = torch.from_numpy(iq).pin_memory()
+            e["iq_dev"] = torch.empty_like(e["iq"], device=ld["q"].device)
+            e["iw"] = ld["iw"].cpu().pin_memory()
+            h2d += e["iq"].numel() * 4 + e["iw"].numel() * 4
+        host.append(e)
+    out_last = runner.layer_data[-1]["out"]
+    out_host = torch.empty(out_last.shape, dtype=out_last.dtype).pin_memory()
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for l, m in enumerate(runner.modes):
+            ld, e = runner.layer_data[l], host[l]
+            ld["q"].copy_(e["q"], non_blocking=True)
+            if m != "U":
+                e["iq_dev"].copy_(e["iq"], non_blocking=True)
+                ld["iw"].copy_(e["iw"], non_blocking=True)
+                runtime.quantize_fp4_rows(e["iq_dev"], ld["iq_codes"], ld["iq_scales"], 32, 4)
+        runner.run()
+        out_host.copy_(out_last, non_blocking=True)
+
+    for _ in range(warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    ms = time_steps(torch, step, steps, flush)
+    return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": sum(ms) / steps}
+
+
+def run_csa2(args, wl):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    import compressed_sparse_attention_quantize_b200 as csa2
+    from compressed_sparse_attention_quantize_b200 import build as csa2_build, runtime, synth
+    if not os.path.exists(csa2.library_path()):
+        csa2_build.build()
+    if rank > 0:
+        wl.seed = wl.seed + 1000 * rank          # independent sequences per rank
+    hbm_peak, tc_peak, tc_sus, peak_src = _peaks()
+    runner = runtime.GroupRunner(wl, out_dtype=csa2.DTYPE_F32)
+    flush_buf = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1)
+
+    for _ in range(args.warmup):
+        flush()
+        runner.run()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = csa2.csa2_launch_count()
+    with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clk:
+        ms = time_steps(torch, runner.run, args.steps, flush)
+    launches = csa2.csa2_launch_count() - launches0
+    clocks = clk.summary()
+    total_ms = sum(ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    value = wl.B * wl.T * world * args.steps / (total_ms / 1e3)
+
+    # per-call breakdown and roofline of the dominant kernel
+    bd = breakdown(torch, csa2, runner, max(3, min(args.steps, 10)), flush)
+    ab, af = attn_work(wl, 4)
+    ib = index_work(wl)
+    kernels = {}
+    if "sparse_attn" in bd:
+        t_ms = statistics.mean(bd["sparse_attn"])
+        kernels["sparse_attn"] = {"launches_per_step": len(runner.modes), "avg_ms": t_ms,
+                                  "share": None, "algorithmic_bytes": ab, "algorithmic_flops": af,
+                                  "achieved_gbs": ab / (t_ms * 1e-3) / 1e9,
+                                  "achieved_tflops": af / (t_ms * 1e-3) / 1e12}
+    if "index_topk" in bd:
+        t_ms = statistics.mean(bd["index_topk"])
+        kernels["index_topk"] = {"launches_per_step": 1, "avg_ms": t_ms, "algorithmic_bytes": ib,
+                                 "achieved_gbs": ib / (t_ms * 1e-3) / 1e9}
+    tot = sum(k["avg_ms"] * k["launches_per_step"] for k in kernels.values())
+    for k in kernels.values():
+        k["share"] = k["avg_ms"] * k["launches_per_step"] / tot if tot else None
+    dom = max(kernels, key=lambda k: kernels[k]["share"] or 0) if kernels else None
+    roof = None
+    if dom == "sparse_attn":
+        k = kernels[dom]
+        roof = {"kernel": "csa2_sparse_attn", "bound": "tensor", "achieved": k["achieved_tflops"],
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": k["achieved_tflops"] / tc_peak,
+                "traffic": None, "peak_source": f"{peak_src} bf16_tflops (fp16 MMA runs at the same rate)",
+                "hbm_achieved_gbs": k["achieved_gbs"], "hbm_frac": k["achieved_gbs"] / hbm_peak}
+    elif dom == "index_topk":
+        k = kernels[dom]
+        roof = {"kernel": "csa2_index_topk", "bound": "hbm", "achieved": k["achieved_gbs"],
+                "peak": hbm_peak, "unit": "GB/s", "frac": k["achieved_gbs"] / hbm_peak,
+                "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
+
+    e2e = e2e_measure(torch, csa2, runner, max(3, min(args.steps, 10)), 2, flush)
+    if world > 1:
+        t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["value"] = wl.B * wl.T * world / (float(t.item()) / 1e3)
+        e2e["ms_per_step"] = float(t.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, runner.softmax_scale)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "fp4(e2m1)+e4m3 storage; f32 compute",
+                "data": "synthetic (seeded; shapes and distributions of the workload)",
+                "config": {"workload": wl.name, "batch_per_gpu": wl.B, "ctx_tokens": wl.ctx_tokens[0],
+                           "entries_per_seq": wl.n_entries[0], "layers": ",".join(wl.modes),
+                           "heads": wl.H, "index_heads": wl.HI, "topk": wl.K, "pool": wl.P,
+                           "swa": 128, "parallelism": f"replicas x{world} (independent sequences)",
+                           "l2": "flushed between steps (256 MB write, outside the events)"},
+                "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": int(launches), "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    del runner
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from compressed_sparse_attention_quantize_b200 import synth
+    wl = synth.workload(args.config)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_csa2(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,312 @@
+// C ABI of the CSA2 library: argument validation, workspace sizing, launch sequencing.
+//
+// Every call validates all arguments before it enqueues anything, launches only on the
+// caller's stream and never synchronises the host (csa2_device_error excepted).
+#include "common.cuh"
+#include "attn.cuh"
+
+namespace csa2 {
+cudaError_t launch_quant_fp4(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
+                             uint8_t *, int64_t, const int64_t *, cudaStream_t);
+cudaError_t launch_quant_fp8_token(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
+                                   uint8_t *, int64_t, const int64_t *, cudaStream_t);
+}  // namespace csa2
+
+#include "index_api.cuh"
+
+#include <atomic>
+
+namespace csa2 {
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace csa2
+
+using namespace csa2;
+
+namespace {
+
+inline bool aligned16(const void *p) { return (((uintptr_t)p) & 15u) == 0; }
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+inline csa2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+constexpr size_t kAlign = 256;
+inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+csa2_status check_index_args(int mode, const uint8_t *q_codes, const uint8_t *q_scales,
+                             const float *w, int B, int T, int H_I, const uint8_t *k_codes,
+                             int64_t k_code_stride, const uint8_t *k_scales, int64_t k_scale_stride,
+                             const int64_t *seq_start, const int32_t *n_entries, int64_t max_n,
+                             const int32_t *pool, const int32_t *pool_len, int P_in, int K,
+                             int32_t *out_idx, int P, int32_t *out_pool) {
+    if (mode != CSA2_MODE_FULL && mode != CSA2_MODE_REINDEX) return CSA2_ERR_INVALID_ARG;
+    if (!q_codes || !q_scales || !w || !k_codes || !k_scales || !seq_start || !n_entries ||
+        !out_idx)
+        return CSA2_ERR_INVALID_ARG;
+    if (B <= 0 || T <= 0 || (int64_t)B * T > (1 << 30)) return CSA2_ERR_SHAPE;
+    if (H_I < 1 || H_I > CSA2_MAX_INDEX_HEADS) return CSA2_ERR_SHAPE;
+    if (K < 1 || K > CSA2_MAX_TOPK) return CSA2_ERR_SHAPE;
+    if (max_n < 0 || max_n > INT32_MAX) return CSA2_ERR_SHAPE;
+    if (k_code_stride < 32 || k_scale_stride < 4) return CSA2_ERR_SHAPE;
+    if (!aligned16(k_codes) || (k_code_stride & 15)) return CSA2_ERR_ALIGN;
+    if (mode == CSA2_MODE_FULL) {
+        if (P < 0 || P > CSA2_MAX_POOL) return CSA2_ERR_SHAPE;
+        if (P > 0 && !out_pool) return CSA2_ERR_INVALID_ARG;
+    } else {
+        if (!pool || !pool_len) return CSA2_ERR_INVALID_ARG;
+        if (P != 0) return CSA2_ERR_INVALID_ARG;
+        if (P_in < 1 || P_in > CSA2_MAX_POOL) return CSA2_ERR_SHAPE;
+    }
+    return CSA2_OK;
+}
+
+csa2_status check_attn_args(const uint16_t *q, int B, int T, int H, int D, const uint8_t *kv,
+                            int64_t kv_row_stride, const int64_t *seq_start, const int32_t *idx,
+                            int K, const uint8_t *swa_codes, const float *swa_scale, int swa_cap,
+                            const int32_t *swa_len, void *out, int out_dtype) {
+    if (!q || !kv || !seq_start || !idx || !swa_len || !out) return CSA2_ERR_INVALID_ARG;
+    if (out_dtype != CSA2_DTYPE_F32 && out_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
+    if (D != CSA2_LATENT_DIM) return CSA2_ERR_UNSUPPORTED;
+    if (B <= 0 || T <= 0 || (int64_t)B * T > (1 << 30)) return CSA2_ERR_SHAPE;
+    if (H < 16 || H > CSA2_MAX_HEADS || (H % 16)) return CSA2_ERR_SHAPE;
+    if (K < 1 || K > CSA2_MAX_TOPK) return CSA2_ERR_SHAPE;
+    if (swa_cap < 0) return CSA2_ERR_SHAPE;
+    if (swa_cap > 0 && (!swa_codes || !swa_scale)) return CSA2_ERR_INVALID_ARG;
+    if (kv_row_stride < kKvRowBytes) return CSA2_ERR_SHAPE;
+    if (!aligned16(kv) || (kv_row_stride & 15)) return CSA2_ERR_ALIGN;
+    if (swa_codes && !aligned16(swa_codes)) return CSA2_ERR_ALIGN;
+    if (!aligned16(q)) return CSA2_ERR_ALIGN;
+    return CSA2_OK;
+}
+
+size_t attn_ws(int rows, int H, int K) { return round_up(attn_workspace_bytes(rows, H, K)); }
+
+size_t index_ws(int mode, int rows, int64_t max_n, int K, int P) {
+    const int64_t n = mode == CSA2_MODE_REINDEX ? (int64_t)P : max_n;
+    return round_up(index_topk_workspace_bytes(rows, n, K));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *csa2_status_string(csa2_status s) {
+    switch (s) {
+        case CSA2_OK: return "CSA2_OK";
+        case CSA2_ERR_INVALID_ARG: return "CSA2_ERR_INVALID_ARG: a required pointer is NULL or an enum is unknown";
+        case CSA2_ERR_SHAPE: return "CSA2_ERR_SHAPE: a size is out of range";
+        case CSA2_ERR_ALIGN: return "CSA2_ERR_ALIGN: a pointer or stride is not 16-byte aligned";
+        case CSA2_ERR_UNSUPPORTED: return "CSA2_ERR_UNSUPPORTED: valid but not implemented";
+        case CSA2_ERR_CUDA: return "CSA2_ERR_CUDA: the CUDA runtime refused a launch";
+        case CSA2_ERR_TIMEOUT: return "CSA2_ERR_TIMEOUT: a bounded device wait expired";
+        case CSA2_ERR_WORKSPACE: return "CSA2_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "CSA2: unknown status";
+}
+
+int csa2_version(void) { return 1; }
+
+uint64_t csa2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
+                             int64_t x_stride, uint8_t *codes, int64_t code_stride, void *scales,
+                             int64_t scale_stride, const int64_t *dst_rows, void *stream) {
+    if (fmt != CSA2_FMT_FP4_E2M1_E4M3S16 && fmt != CSA2_FMT_FP8_E4M3_TOKEN) return CSA2_ERR_INVALID_ARG;
+    if (x_dtype != CSA2_DTYPE_F32 && x_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
+    if (rows < 0 || dim <= 0 || (dim % 16) || dim > 65536 || x_stride < dim) return CSA2_ERR_SHAPE;
+    if (rows == 0) return CSA2_OK;
+    if (!x || !codes || !scales) return CSA2_ERR_INVALID_ARG;
+    if (fmt == CSA2_FMT_FP4_E2M1_E4M3S16) {
+        if (code_stride < dim / 2 || scale_stride < dim / 16) return CSA2_ERR_SHAPE;
+        return cuda_status(launch_quant_fp4(x, x_dtype, rows, dim, x_stride, codes, code_stride,
+                                            (uint8_t *)scales, scale_stride, dst_rows,
+                                            as_stream(stream)));
+    }
+    if (code_stride < dim || scale_stride < 4) return CSA2_ERR_SHAPE;
+    if ((((uintptr_t)scales) & 3u) || (scale_stride & 3)) return CSA2_ERR_ALIGN;
+    return cuda_status(launch_quant_fp8_token(x, x_dtype, rows, dim, x_stride, codes, code_stride,
+                                              (uint8_t *)scales, scale_stride, dst_rows,
+                                              as_stream(stream)));
+}
+
+csa2_status csa2_index_topk_workspace_size(int mode, int rows, int64_t max_n, int K, int P,
+                                           size_t *bytes) {
+    if (!bytes) return CSA2_ERR_INVALID_ARG;
+    if (rows <= 0 || max_n < 0 || K < 1 || P < 0) return CSA2_ERR_SHAPE;
+    *bytes = index_ws(mode, rows, max_n, K, P);
+    return CSA2_OK;
+}
+
+csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uint8_t *q_scales,
+                            const float *w, int B, int T, int H_I, const uint8_t *k_codes,
+                            int64_t k_code_stride, const uint8_t *k_scales, int64_t k_scale_stride,
+                            const int64_t *seq_start, const int32_t *n_entries, int64_t max_n,
+                            const int32_t *q_pos, const int32_t *pool, const int32_t *pool_len,
+                            int P_in, int K, int32_t *out_idx, int32_t *out_cnt, int P,
+                            int32_t *out_pool, int32_t *out_pool_len, void *workspace,
+                            size_t ws_bytes, void *stream) {
+    csa2_status s = check_index_args(mode, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_stride,
+                                     k_scales, k_scale_stride, seq_start, n_entries, max_n, pool,
+                                     pool_len, P_in, K, out_idx, P, out_pool);
+    if (s != CSA2_OK) return s;
+    const int rows = B * T;
+    const size_t need = index_ws(mode, rows, max_n, K, mode == CSA2_MODE_REINDEX ? P_in : P);
+    if (!workspace || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    IndexLaunch L;
+    L.mode = mode; L.q_codes = q_codes; L.q_scales = q_scales; L.w = w;
+    L.B = B; L.T = T; L.H = H_I;
+    L.k_codes = k_codes; L.k_code_stride = k_code_stride;
+    L.k_scales = k_scales; L.k_scale_stride = k_scale_stride;
+    L.seq_start = seq_start; L.n_entries = n_entries; L.max_n = max_n; L.q_pos = q_pos;
+    L.pool = pool; L.pool_len = pool_len; L.P_in = P_in;
+    L.K = K; L.out_idx = out_idx; L.out_cnt = out_cnt;
+    L.P = P; L.out_pool = out_pool; L.out_pool_len = out_pool_len;
+    L.workspace = workspace; L.ws_bytes = ws_bytes;
+    return cuda_status(launch_index_topk(L, as_stream(stream)));
+}
+
+csa2_status csa2_sparse_attn_workspace_size(int rows, int H, int K, size_t *bytes) {
+    if (!bytes) return CSA2_ERR_INVALID_ARG;
+    if (rows <= 0 || H <= 0 || K <= 0) return CSA2_ERR_SHAPE;
+    *bytes = attn_ws(rows, H, K);
+    return CSA2_OK;
+}
+
+csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D, const uint8_t *kv,
+                             int64_t kv_row_stride, const int64_t *seq_start, const int32_t *idx,
+                             const int32_t *cnt, int K, const uint8_t *swa_codes,
+                             const float *swa_scale, int swa_cap, const int32_t *swa_start,
+                             const int32_t *swa_len, float softmax_scale, void *out,
+                             int out_dtype, float *lse, void *workspace, size_t ws_bytes,
+                             void *stream) {
+    csa2_status s = check_attn_args(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, K, swa_codes,
+                                    swa_scale, swa_cap, swa_len, out, out_dtype);
+    if (s != CSA2_OK) return s;
+    const int rows = B * T;
+    if (!workspace || ws_bytes < attn_ws(rows, H, K)) return CSA2_ERR_WORKSPACE;
+    AttnArgs a;
+    a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
+    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start;
+    a.idx = idx; a.cnt = cnt;
+    a.swa_codes = swa_codes; a.swa_scale = swa_scale; a.swa_cap = swa_cap;
+    a.swa_start = swa_start; a.swa_len = swa_len;
+    a.softmax_scale = softmax_scale; a.out = out; a.out_dtype = out_dtype; a.lse = lse;
+    a.partials = reinterpret_cast<float *>(workspace);
+    a.splits = 1;
+    return cuda_status(launch_attn(a, as_stream(stream)));
+}
+
+// ------------------------------------------------------------------------------------------
+// layer group
+// ------------------------------------------------------------------------------------------
+static csa2_status group_layout(const csa2_group_desc *g, const csa2_layer_desc *layers, int n,
+                                size_t *idx_off, size_t *pool_off, size_t *idx_ws_off,
+                                size_t *attn_off, size_t *total) {
+    if (!g || !layers || n <= 0) return CSA2_ERR_INVALID_ARG;
+    bool need_pool = false, seen_full = false;
+    for (int l = 0; l < n; ++l) {
+        const int m = layers[l].mode;
+        if (m == CSA2_MODE_FULL) seen_full = true;
+        else if (m == CSA2_MODE_REINDEX || m == CSA2_MODE_REUSE) {
+            if (!seen_full) return CSA2_ERR_INVALID_ARG;
+            if (m == CSA2_MODE_REINDEX) need_pool = true;
+        } else return CSA2_ERR_INVALID_ARG;
+    }
+    if (need_pool && g->P <= 0) return CSA2_ERR_INVALID_ARG;
+    if (g->B <= 0 || g->T <= 0) return CSA2_ERR_SHAPE;
+    const int rows = g->B * g->T;
+    size_t off = 0;
+    *idx_off = off; off += round_up((size_t)rows * g->K * 4 + (size_t)rows * 4);
+    *pool_off = off;
+    if (need_pool) off += round_up((size_t)rows * g->P * 4 + (size_t)rows * 4);
+    *idx_ws_off = off;
+    size_t iw = index_ws(CSA2_MODE_FULL, rows, g->max_n, g->K, need_pool ? g->P : 0);
+    if (need_pool) {
+        size_t iw2 = index_ws(CSA2_MODE_REINDEX, rows, g->max_n, g->K, g->P);
+        if (iw2 > iw) iw = iw2;
+    }
+    *attn_off = off + iw;
+    off += iw + attn_ws(rows, g->H, g->K);
+    *total = off;
+    return CSA2_OK;
+}
+
+csa2_status csa2_layer_group_workspace_size(const csa2_group_desc *g, const csa2_layer_desc *layers,
+                                            int n_layers, size_t *bytes) {
+    if (!bytes) return CSA2_ERR_INVALID_ARG;
+    size_t a, b, c, d;
+    return group_layout(g, layers, n_layers, &a, &b, &c, &d, bytes);
+}
+
+csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *layers, int n_layers,
+                             void *workspace, size_t ws_bytes, void *stream) {
+    size_t idx_off, pool_off, iws_off, attn_off, total;
+    csa2_status s = group_layout(g, layers, n_layers, &idx_off, &pool_off, &iws_off, &attn_off, &total);
+    if (s != CSA2_OK) return s;
+    if (!workspace || ws_bytes < total) return CSA2_ERR_WORKSPACE;
+    const int rows = g->B * g->T;
+    bool need_pool = false;
+    for (int l = 0; l < n_layers; ++l) need_pool |= layers[l].mode == CSA2_MODE_REINDEX;
+    // validate every layer before launching anything
+    for (int l = 0; l < n_layers; ++l) {
+        const csa2_layer_desc &L = layers[l];
+        if (L.mode != CSA2_MODE_REUSE) {
+            s = check_index_args(L.mode, L.iq_codes, L.iq_scales, L.iw, g->B, g->T, g->H_I,
+                                 g->k_codes, g->k_code_stride, g->k_scales, g->k_scale_stride,
+                                 g->seq_start, g->n_entries, g->max_n,
+                                 L.mode == CSA2_MODE_REINDEX ? (const int32_t *)1 : nullptr,
+                                 L.mode == CSA2_MODE_REINDEX ? (const int32_t *)1 : nullptr,
+                                 g->P, g->K, (int32_t *)1,
+                                 L.mode == CSA2_MODE_FULL && need_pool ? g->P : 0, (int32_t *)1);
+            if (s != CSA2_OK) return s;
+        }
+        s = check_attn_args(L.q, g->B, g->T, g->H, g->D, g->kv, g->kv_row_stride, g->seq_start,
+                            (const int32_t *)1, g->K, L.swa_codes, L.swa_scale, g->swa_cap,
+                            g->swa_len, L.out, g->out_dtype);
+        if (s != CSA2_OK) return s;
+    }
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws + idx_off);
+    int32_t *cnt = idx + (size_t)rows * g->K;
+    int32_t *pool = need_pool ? reinterpret_cast<int32_t *>(ws + pool_off) : nullptr;
+    int32_t *pool_len = need_pool ? pool + (size_t)rows * g->P : nullptr;
+    void *iws = ws + iws_off;
+    const size_t iws_bytes = attn_off - iws_off;
+    void *aws = ws + attn_off;
+    const size_t aws_bytes = total - attn_off;
+    cudaStream_t st = as_stream(stream);
+    for (int l = 0; l < n_layers; ++l) {
+        const csa2_layer_desc &L = layers[l];
+        if (L.mode == CSA2_MODE_FULL) {
+            s = csa2_index_topk(CSA2_MODE_FULL, L.iq_codes, L.iq_scales, L.iw, g->B, g->T, g->H_I,
+                                g->k_codes, g->k_code_stride, g->k_scales, g->k_scale_stride,
+                                g->seq_start, g->n_entries, g->max_n, g->q_pos, nullptr, nullptr, 0,
+                                g->K, idx, cnt, need_pool ? g->P : 0, pool, pool_len, iws,
+                                iws_bytes, stream);
+        } else if (L.mode == CSA2_MODE_REINDEX) {
+            s = csa2_index_topk(CSA2_MODE_REINDEX, L.iq_codes, L.iq_scales, L.iw, g->B, g->T,
+                                g->H_I, g->k_codes, g->k_code_stride, g->k_scales,
+                                g->k_scale_stride, g->seq_start, g->n_entries, g->max_n, g->q_pos,
+                                pool, pool_len, g->P, g->K, idx, cnt, 0, nullptr, nullptr, iws,
+                                iws_bytes, stream);
+        }
+        if (s != CSA2_OK) return s;
+        // REUSE: idx/cnt still hold the preceding layer's selection
+        if (L.idx_out) {
+            cudaError_t e = cudaMemcpyAsync(L.idx_out, idx, (size_t)rows * g->K * 4,
+                                            cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return CSA2_ERR_CUDA;
+        }
+        s = csa2_sparse_attn(L.q, g->B, g->T, g->H, g->D, g->kv, g->kv_row_stride, g->seq_start, idx,
+                             cnt, g->K, L.swa_codes, L.swa_scale, g->swa_cap, g->swa_start,
+                             g->swa_len, g->softmax_scale, L.out, g->out_dtype, L.lse, aws,
+                             aws_bytes, stream);
+        if (s != CSA2_OK) return s;
+    }
+    return CSA2_OK;
+}
+
+csa2_status csa2_device_error(void *stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CSA2_ERR_CUDA;
+    return read_and_clear_device_error();
+}
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// Arguments shared by the attention kernels.
+#pragma once
+#include "common.cuh"
+
+namespace csa2 {
+
+struct AttnArgs {
+    const uint16_t *q;          // bf16 [rows][H][512]
+    int rows, T, H, K;
+    const uint8_t *kv;          // main entries, kv_row_stride bytes apart
+    int64_t kv_row_stride;
+    const int64_t *seq_start;
+    const int32_t *idx;         // [rows][K]
+    const int32_t *cnt;         // [rows] or NULL
+    const uint8_t *swa_codes;   // [B][swa_cap][512]
+    const float *swa_scale;     // [B][swa_cap]
+    int swa_cap;
+    const int32_t *swa_start;   // [rows] or NULL
+    const int32_t *swa_len;     // [rows]
+    float softmax_scale;
+    void *out;
+    int out_dtype;
+    float *lse;
+    float *partials;            // workspace
+    int splits;
+};
+
+cudaError_t launch_attn_simt(AttnArgs a, cudaStream_t st);
+size_t simt_workspace_bytes(int rows, int H, int K);
+
+// Dispatch used by the C ABI.
+size_t attn_workspace_bytes(int rows, int H, int K);
+cudaError_t launch_attn(AttnArgs a, cudaStream_t st);
+
+}  // namespace csa2

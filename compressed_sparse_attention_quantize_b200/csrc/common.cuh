@@ -1,0 +1,99 @@
+// Device helpers shared by the CSA2 kernels: number formats, keys, launch checks.
+//
+// Formats ([B] = page "DeepSeek V4.1 Flash 如何靠压缩 KV 缓存实现小模型干翻大模型",
+// section "FP4 量化 + Bounded Replay"): E2M1 codes with one E4M3 scale per 16 channels;
+// the 8-bit sliding window uses E4M3 with a per-token fp32 scale.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+#define CSA2_HD __host__ __device__ __forceinline__
+#define CSA2_D __device__ __forceinline__
+
+namespace csa2 {
+
+constexpr int kLatent = 512;
+constexpr int kKvRowBytes = kLatent / 2 + kLatent / 16;   // 288
+constexpr int kIndexDim = 64;
+
+// ---------------------------------------------------------------------------------------
+// E4M3 ("fn": bias 7, max 448, no inf) and E2M1
+// ---------------------------------------------------------------------------------------
+
+// Decode an E4M3 code to fp32 (exact).
+CSA2_D float e4m3_to_f32(uint32_t code) {
+    uint32_t e = (code >> 3) & 15u, m = code & 7u;
+    float mag;
+    if (e == 0) {
+        mag = (float)m * 0.001953125f;                  // m * 2^-9
+    } else {
+        mag = __uint_as_float(((e + 120u) << 23) | (m << 20));
+    }
+    return (code & 0x80u) ? -mag : mag;
+}
+
+// Round a non-negative fp32 magnitude to an E4M3 magnitude code, nearest-even,
+// saturating finite values above 448 to 448 (code 0x7E).
+CSA2_D uint32_t e4m3_code_mag_rne(float a) {
+    if (!(a < 448.0f)) return 0x7Eu;                     // also catches +inf
+    if (a < 0.015625f) {                                  // below 2^-6: subnormal grid 2^-9
+        return (uint32_t)__float2int_rn(a * 512.0f);      // exact scaling; ties to even
+    }
+    uint32_t bits = __float_as_uint(a);
+    uint32_t e = bits >> 23;                              // biased fp32 exponent
+    uint32_t code = ((e - 120u) << 3) | ((bits >> 20) & 7u);
+    uint32_t rem = bits & 0xFFFFFu;
+    if (rem > 0x80000u || (rem == 0x80000u && (code & 1u))) code += 1u;   // carry ok
+    return code > 0x7Eu ? 0x7Eu : code;
+}
+
+// Round a non-negative fp32 magnitude to an E2M1 magnitude code (0..7), nearest-even,
+// saturating at 6.  Midpoints: 0.25->0, 0.75->1.0, 1.25->1.0, 1.75->2, 2.5->2, 3.5->4, 5->4.
+CSA2_D uint32_t e2m1_code_mag_rne(float a) {
+    return (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+           (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
+           (uint32_t)(a > 5.0f);
+}
+
+// E2M1 magnitude table (codes 0..7).
+CSA2_D float e2m1_mag(uint32_t c) {
+    // 0, .5, 1, 1.5, 2, 3, 4, 6 without a memory table
+    uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    float base = e == 0 ? 0.0f : __uint_as_float((126u + e) << 23);   // 2^(e-1)
+    return e == 0 ? 0.5f * (float)m : base * (1.0f + 0.5f * (float)m);
+}
+
+CSA2_D float e2m1_to_f32(uint32_t c) {
+    float v = e2m1_mag(c & 7u);
+    return (c & 8u) ? -v : v;
+}
+
+// ---------------------------------------------------------------------------------------
+// bf16
+// ---------------------------------------------------------------------------------------
+CSA2_D float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+
+// ---------------------------------------------------------------------------------------
+// Order-preserving key: larger float -> larger unsigned key (for radix selection).
+// ---------------------------------------------------------------------------------------
+CSA2_HD uint32_t float_key(float f) {
+#ifdef __CUDA_ARCH__
+    uint32_t u = __float_as_uint(f);
+#else
+    uint32_t u;
+    memcpy(&u, &f, 4);
+#endif
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+CSA2_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Host-side count of kernel launches (csa2_launch_count); every launcher adds its launches.
+void note_launches(int n);
+
+}  // namespace csa2

@@ -1,0 +1,326 @@
+// Indexer scoring and top-K block selection (Full and Reindex modes).
+//
+// [B] page "DeepSeek V4.1 Flash 如何靠压缩 KV 缓存实现小模型干翻大模型":
+//   section "为什么 KV 缓存成了新瓶颈？" names the DSA-style indexer; section
+//   "CSA2：三层压缩一次吃满" defines Full (own indexer query, full scan) and Reindex
+//   (re-score an earlier layer's candidates with the layer's own query); section
+//   "FP4 量化 + Bounded Replay" makes indexer Q and K FP4.
+// [A] page "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径", section
+//   "压缩吸收注意力（二代）": the first layer picks 2048 blocks and keeps a candidate pool.
+//
+// Score I[r,j] = sum_h w_h * relu(q_h . k_j) in fp32.  Per 16-channel block the partial is
+// exact in any order (all terms are multiples of s_q*s_k/4 and the block needs <= 20
+// significant bits), so it is accumulated with fma; the four blocks and the heads are then
+// added in a fixed left-to-right order with explicitly rounded adds and multiplies.  This
+// reproduces the reference order bit for bit, so the selected sets match exactly.
+//
+// Selection is a 4-pass, 8-bit radix select on order-preserving keys, then one compaction
+// pass in entry order: entries above the threshold key, plus the lowest-indexed entries
+// equal to it, written in ascending index order.
+#include "common.cuh"
+#include "index_api.cuh"
+
+namespace csa2 {
+
+constexpr int kScoreThreads = 256;
+constexpr int kSelectThreads = 1024;
+
+struct ScoreArgs {
+    const uint8_t *q_codes;    // [rows][H][32]
+    const uint8_t *q_scales;   // [rows][H][4]
+    const float *w;            // [rows][H]
+    int H;
+    int T;
+    const uint8_t *k_codes;
+    int64_t k_code_stride;
+    const uint8_t *k_scales;
+    int64_t k_scale_stride;
+    const int64_t *seq_start;
+    const int32_t *n_entries;
+    const int32_t *q_pos;      // nullable
+    const int32_t *pool;       // Reindex: [rows][P_in]
+    const int32_t *pool_len;
+    int P_in;
+    int row0;                  // first query row of this launch
+    float *scores;             // [launch rows][score_stride]
+    int64_t score_stride;
+};
+
+// Number of candidates of row r (visible entries, or pool length).
+CSA2_D int64_t row_candidates(const ScoreArgs &a, int r) {
+    if (a.pool) return a.pool_len[r];
+    const int b = r / a.T;
+    int64_t n = a.n_entries[b];
+    if (a.q_pos) {
+        int64_t v = ((int64_t)a.q_pos[r] + 1) / 4;
+        n = v < n ? v : n;
+        if (n < 0) n = 0;
+    }
+    return n;
+}
+
+__global__ void __launch_bounds__(kScoreThreads)
+index_score_kernel(ScoreArgs a) {
+    const int r = a.row0 + blockIdx.y;
+    const int b = r / a.T;
+    __shared__ float qv[CSA2_MAX_INDEX_HEADS * 64];
+    __shared__ float wv[CSA2_MAX_INDEX_HEADS];
+    for (int i = threadIdx.x; i < a.H * 64; i += blockDim.x) {
+        const int h = i >> 6, c = i & 63;
+        const uint8_t byte = a.q_codes[((int64_t)r * a.H + h) * 32 + (c >> 1)];
+        const uint32_t code = (c & 1) ? (byte >> 4) : (byte & 15u);
+        qv[i] = e2m1_to_f32(code) * e4m3_to_f32(a.q_scales[((int64_t)r * a.H + h) * 4 + (c >> 4)]);
+    }
+    for (int i = threadIdx.x; i < a.H; i += blockDim.x) wv[i] = a.w[(int64_t)r * a.H + i];
+    __syncthreads();
+
+    const int64_t n = row_candidates(a, r);
+    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= n || j >= a.score_stride) return;         // score_stride == max_n bounds the row
+    const int64_t e = a.seq_start[b] + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
+    const uint4 *kc = reinterpret_cast<const uint4 *>(a.k_codes + e * a.k_code_stride);
+    const uint4 c0 = __ldg(kc), c1 = __ldg(kc + 1);
+    const uint8_t *ksp = a.k_scales + e * a.k_scale_stride;
+    float ks[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ks[i] = e4m3_to_f32(__ldg(ksp + i));
+    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    float kv[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+        kv[c] = e2m1_to_f32((words[c >> 3] >> ((c & 7) * 4)) & 15u) * ks[c >> 4];
+
+    float acc = 0.0f;
+    for (int h = 0; h < a.H; ++h) {
+        float p[4];
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+            float s = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) s = fmaf(qv[h * 64 + blk * 16 + i], kv[blk * 16 + i], s);
+            p[blk] = s;                                        // exact
+        }
+        const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
+        const float rl = dot > 0.0f ? dot : 0.0f;
+        acc = __fadd_rn(acc, __fmul_rn(wv[h], rl));
+    }
+    if (acc == 0.0f) acc = 0.0f;                               // -0 -> +0
+    a.scores[(int64_t)blockIdx.y * a.score_stride + j] = acc;
+}
+
+// ---------------------------------------------------------------------------------------
+// Block-wide helpers (blockDim.x == kSelectThreads)
+// ---------------------------------------------------------------------------------------
+// Exclusive prefix of a 0/1 flag over the block in thread order; returns the block total.
+CSA2_D int block_exclusive_count(bool flag, int *warp_sums, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned bal = __ballot_sync(0xffffffffu, flag);
+    const int within = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) warp_sums[warp] = __popc(bal);
+    __syncthreads();
+    if (warp == 0) {
+        int v = warp_sums[lane];
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        warp_sums[lane] = incl - v;                 // exclusive
+        if (lane == 31) warp_sums[32] = incl;       // total
+    }
+    __syncthreads();
+    const int res = warp_sums[warp] + within;
+    total = warp_sums[32];
+    __syncthreads();
+    return res;
+}
+
+// Radix-select the threshold key of the k-th largest key among n; returns (key, how many
+// entries equal to key must be taken).
+__device__ void radix_threshold(const float *scores, int64_t n, int64_t k, uint32_t &thr,
+                                int64_t &need_eq) {
+    __shared__ unsigned int hist[256];
+    __shared__ uint32_t s_prefix, s_mask;
+    __shared__ long long s_remaining;
+    if (threadIdx.x == 0) { s_prefix = 0u; s_mask = 0u; s_remaining = k; }
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        const uint32_t prefix = s_prefix, mask = s_mask;
+        for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+            const uint32_t key = float_key(scores[j]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            // lane owns bins [8*lane, 8*lane+8); suffix sums from the top bin down
+            unsigned int local = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) local += hist[lane * 8 + i];
+            unsigned int suffix = local;               // inclusive sum of lanes >= lane
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                unsigned int t = __shfl_down_sync(0xffffffffu, suffix, o);
+                if (lane + o < 32) suffix += t;
+            }
+            const long long rem = s_remaining;
+            const unsigned int above = suffix - local;  // count in lanes > lane
+            const bool crosses = (long long)above < rem && rem <= (long long)suffix;
+            const unsigned bal = __ballot_sync(0xffffffffu, crosses);
+            const int owner = __ffs(bal) - 1;
+            if (lane == owner) {
+                long long acc = above;
+                int d = lane * 8 + 7;
+                for (; d > lane * 8; --d) {
+                    if (acc + hist[d] >= rem) break;
+                    acc += hist[d];
+                }
+                s_remaining = rem - acc;
+                s_prefix = prefix | ((uint32_t)d << shift);
+                s_mask = mask | (255u << shift);
+            }
+        }
+        __syncthreads();
+    }
+    thr = s_prefix;
+    need_eq = s_remaining;
+    __syncthreads();
+}
+
+// Select the top-k of one row into out[0..k) (ascending index, -1 padded); ids maps
+// candidate positions to entry ids (NULL = identity).
+__device__ void select_row(const float *scores, const int32_t *ids, int64_t n, int k,
+                           int32_t *out, int32_t *out_cnt) {
+    __shared__ int warp_sums[33];
+    const int cnt = (int)(n < k ? n : k);
+    if (n <= k) {
+        for (int64_t j = threadIdx.x; j < n; j += blockDim.x) out[j] = ids ? ids[j] : (int32_t)j;
+    } else {
+        uint32_t thr;
+        int64_t need_eq;
+        radix_threshold(scores, n, k, thr, need_eq);
+        int64_t run_out = 0, run_eq = 0;
+        for (int64_t base = 0; base < n; base += blockDim.x) {
+            const int64_t j = base + threadIdx.x;
+            uint32_t key = 0u;
+            if (j < n) key = float_key(scores[j]);
+            const bool gt = j < n && key > thr;
+            const bool eq = j < n && key == thr;
+            int eq_total;
+            const int eq_rank = block_exclusive_count(eq, warp_sums, eq_total);
+            const bool sel = gt || (eq && run_eq + eq_rank < need_eq);
+            int sel_total;
+            const int pos = block_exclusive_count(sel, warp_sums, sel_total);
+            if (sel) out[run_out + pos] = ids ? ids[j] : (int32_t)j;
+            run_out += sel_total;
+            run_eq += eq_total;
+        }
+    }
+    for (int i = cnt + threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    if (threadIdx.x == 0 && out_cnt) *out_cnt = cnt;
+    __syncthreads();
+}
+
+struct SelectArgs {
+    const float *scores;
+    int64_t score_stride;
+    ScoreArgs sa;              // for row_candidates()
+    int K;
+    int32_t *out_idx;
+    int32_t *out_cnt;
+    int P;
+    int32_t *out_pool;
+    int32_t *out_pool_len;
+};
+
+__global__ void __launch_bounds__(kSelectThreads)
+select_kernel(SelectArgs a) {
+    const int lr = blockIdx.x;
+    const int r = a.sa.row0 + lr;
+    int64_t n = row_candidates(a.sa, r);
+    if (n > a.score_stride) n = a.score_stride;        // never read past the row's scores
+    const float *s = a.scores + (int64_t)lr * a.score_stride;
+    const int32_t *ids = a.sa.pool ? a.sa.pool + (int64_t)r * a.sa.P_in : nullptr;
+    select_row(s, ids, n, a.K, a.out_idx + (int64_t)r * a.K, a.out_cnt ? a.out_cnt + r : nullptr);
+    if (a.P > 0)
+        select_row(s, ids, n, a.P, a.out_pool + (int64_t)r * a.P,
+                   a.out_pool_len ? a.out_pool_len + r : nullptr);
+}
+
+// Rows processed per launch so the score buffer stays bounded.
+static int64_t index_rows_per_chunk(int rows, int64_t max_n) {
+    const int64_t cap = (int64_t)256 << 20;                       // 256 MB of scores
+    int64_t per = cap / ((max_n > 0 ? max_n : 1) * 4);
+    if (per < 1) per = 1;
+    return per < rows ? per : rows;
+}
+
+size_t index_topk_workspace_bytes(int rows, int64_t n, int K) {
+    (void)K;
+    const int64_t chunk = index_rows_per_chunk(rows, n);
+    return (size_t)(chunk * (n > 0 ? n : 1) * 4 + 256);
+}
+
+cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
+    ScoreArgs base;
+    base.q_codes = L.q_codes; base.q_scales = L.q_scales; base.w = L.w;
+    base.H = L.H; base.T = L.T;
+    base.k_codes = L.k_codes; base.k_code_stride = L.k_code_stride;
+    base.k_scales = L.k_scales; base.k_scale_stride = L.k_scale_stride;
+    base.seq_start = L.seq_start; base.n_entries = L.n_entries; base.q_pos = L.q_pos;
+    const bool reindex = L.mode == CSA2_MODE_REINDEX;
+    base.pool = reindex ? L.pool : nullptr;
+    base.pool_len = reindex ? L.pool_len : nullptr;
+    base.P_in = L.P_in;
+    const int rows = L.B * L.T;
+    const int64_t max_n = reindex ? (int64_t)L.P_in : L.max_n;
+    const int64_t chunk = index_rows_per_chunk(rows, max_n);
+    float *scores = reinterpret_cast<float *>(L.workspace);
+    for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+        const int nr = (int)((rows - r0) < chunk ? (rows - r0) : chunk);
+        ScoreArgs sa = base;
+        sa.row0 = (int)r0;
+        sa.scores = scores;
+        sa.score_stride = max_n > 0 ? max_n : 1;
+        if (max_n > 0) {
+            dim3 grid((unsigned)ceil_div(max_n, kScoreThreads), (unsigned)nr);
+            index_score_kernel<<<grid, kScoreThreads, 0, st>>>(sa);
+            note_launches(1);
+        }
+        SelectArgs se;
+        se.scores = scores;
+        se.score_stride = sa.score_stride;
+        se.sa = sa;
+        se.K = L.K;
+        se.out_idx = L.out_idx;
+        se.out_cnt = L.out_cnt;
+        se.P = reindex ? 0 : L.P;
+        se.out_pool = L.out_pool;
+        se.out_pool_len = L.out_pool_len;
+        select_kernel<<<nr, kSelectThreads, 0, st>>>(se);
+        note_launches(1);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------------------
+// device error word
+// ---------------------------------------------------------------------------------------
+__device__ int g_device_error = 0;
+
+csa2_status read_and_clear_device_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return CSA2_ERR_CUDA;
+    }
+    return (csa2_status)v;
+}
+
+}  // namespace csa2

@@ -1,0 +1,6 @@
+// Single translation unit of the CSA2 library (keeps device symbols in one module).
+#include "quant.cu"
+#include "index_topk.cu"
+#include "attn_simt.cu"
+#include "attn_dispatch.cu"
+#include "api.cu"

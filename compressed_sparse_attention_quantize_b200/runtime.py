@@ -1,0 +1,139 @@
+"""Device-side setup of a CSA2 workload and one call of the layer group.
+
+``GroupRunner`` owns the caller-side buffers the C ABI expects (PyTorch allocates them):
+the packed main-KV cache (288-byte rows), the indexer-key cache, and per layer the main
+query, the quantised indexer query and head weights, the 8-bit window and the outputs.
+All quantisation is done on the device with ``csa2_quantize_kv`` (quantise-on-write).
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+from . import (DTYPE_BF16, DTYPE_F32, FMT_FP4, FMT_FP8_TOKEN, MODE_FULL, MODE_REINDEX, MODE_REUSE,
+               GroupDesc, LayerDesc, csa2_layer_group, csa2_layer_group_workspace_size,
+               csa2_quantize_kv)
+from . import synth
+
+KV_ROW = 288
+_MODE = {"F": MODE_FULL, "I": MODE_REINDEX, "U": MODE_REUSE}
+
+
+def quantize_fp4_rows(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                      code_stride: int, scale_stride: int, dst_rows=None, stream=None):
+    """Quantise float32/bf16 rows [rows, dim] into FP4 codes/scales (device buffers)."""
+    rows, dim = x.shape
+    dt = DTYPE_F32 if x.dtype == torch.float32 else DTYPE_BF16
+    csa2_quantize_kv(FMT_FP4, x, dt, rows, dim, x.stride(0), codes, code_stride, scales,
+                     scale_stride, dst_rows, stream)
+
+
+def quantize_fp8_rows(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, dst_rows=None,
+                      stream=None):
+    rows, dim = x.shape
+    dt = DTYPE_F32 if x.dtype == torch.float32 else DTYPE_BF16
+    csa2_quantize_kv(FMT_FP8_TOKEN, x, dt, rows, dim, x.stride(0), codes, codes.stride(0), scales,
+                     4, dst_rows, stream)
+
+
+class GroupRunner:
+    """Holds one workload on the device and runs its layer group through the C ABI."""
+
+    def __init__(self, wl: synth.Workload, device="cuda", out_dtype=DTYPE_F32,
+                 softmax_scale: Optional[float] = None, layers: Optional[int] = None):
+        self.wl = wl
+        self.dev = torch.device(device)
+        self.out_dtype = out_dtype
+        self.softmax_scale = (1.0 / math.sqrt(synth.D_LATENT)) if softmax_scale is None else softmax_scale
+        modes = wl.modes if layers is None else wl.modes[:layers]
+        self.modes = modes
+        B, T, H, HI, K = wl.B, wl.T, wl.H, wl.HI, wl.K
+        self.rows = B * T
+        n = wl.n_entries
+        starts = np.concatenate([[0], np.cumsum(n)[:-1]]).astype(np.int64)
+        total = int(np.sum(n))
+        self.total_entries = total
+        self.max_n = int(max(n))
+        d = self.dev
+        self.seq_start = torch.from_numpy(starts).to(d)
+        self.n_entries = torch.tensor(n, dtype=torch.int32, device=d)
+        self.kv = torch.empty((max(total, 1), KV_ROW), dtype=torch.uint8, device=d)
+        self.k_codes = torch.empty((max(total, 1), 32), dtype=torch.uint8, device=d)
+        self.k_scales = torch.empty((max(total, 1), 4), dtype=torch.uint8, device=d)
+        # caches: quantise-on-write, one sequence at a time (bounds host memory)
+        for b in range(B):
+            s0 = int(starts[b])
+            lat = torch.from_numpy(synth.kv_latent(wl, b)).to(d)
+            quantize_fp4_rows(lat, self.kv[s0:], self.kv[s0:, 256:], KV_ROW, KV_ROW)
+            del lat
+            ik = torch.from_numpy(synth.index_keys(wl, b)).to(d)
+            quantize_fp4_rows(ik, self.k_codes[s0:], self.k_scales[s0:], 32, 4)
+            del ik
+        # query positions (prefill) and window slots
+        if wl.prefill_start is not None:
+            qp = np.concatenate([wl.q_pos(b) for b in range(B)]).astype(np.int32)
+            self.q_pos = torch.from_numpy(qp).to(d)
+        else:
+            self.q_pos = None
+        st, ln = zip(*[synth.swa_window(wl, b) for b in range(B)])
+        self.swa_start = torch.from_numpy(np.concatenate(st).astype(np.int32)).to(d)
+        self.swa_len = torch.from_numpy(np.concatenate(ln).astype(np.int32)).to(d)
+        self.swa_cap = wl.swa_tokens()
+        # per layer
+        self.layer_data = []
+        odt = torch.float32 if out_dtype == DTYPE_F32 else torch.bfloat16
+        for l, m in enumerate(modes):
+            q = np.stack([synth.main_query_bf16(wl, l, b) for b in range(B)]).reshape(self.rows, H, 512)
+            ld = {"q": torch.from_numpy(q.view(np.int16)).to(d)}
+            if m != "U":
+                iq = np.stack([synth.index_query(wl, l, b) for b in range(B)]).reshape(self.rows * HI, 64)
+                iqt = torch.from_numpy(iq).to(d)
+                ld["iq_codes"] = torch.empty((self.rows * HI, 32), dtype=torch.uint8, device=d)
+                ld["iq_scales"] = torch.empty((self.rows * HI, 4), dtype=torch.uint8, device=d)
+                quantize_fp4_rows(iqt, ld["iq_codes"], ld["iq_scales"], 32, 4)
+                w = np.stack([synth.head_weights(wl, l, b) for b in range(B)]).reshape(self.rows, HI)
+                ld["iw"] = torch.from_numpy(np.ascontiguousarray(w)).to(d)
+            sw = np.stack([synth.swa_latent(wl, l, b) for b in range(B)]).reshape(B * self.swa_cap, 512)
+            swt = torch.from_numpy(sw).to(d)
+            ld["swa_codes"] = torch.empty((B * self.swa_cap, 512), dtype=torch.uint8, device=d)
+            ld["swa_scale"] = torch.empty((B * self.swa_cap,), dtype=torch.float32, device=d)
+            quantize_fp8_rows(swt, ld["swa_codes"], ld["swa_scale"])
+            ld["out"] = torch.empty((self.rows, H, 512), dtype=odt, device=d)
+            ld["lse"] = torch.empty((self.rows, H), dtype=torch.float32, device=d)
+            ld["idx"] = torch.empty((self.rows, K), dtype=torch.int32, device=d)
+            self.layer_data.append(ld)
+        self.g = self._group_desc()
+        self.layer_descs = [self._layer_desc(l) for l in range(len(modes))]
+        self.ws_bytes = csa2_layer_group_workspace_size(self.g, self.layer_descs)
+        self.workspace = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=d)
+        torch.cuda.synchronize()
+
+    def _group_desc(self) -> GroupDesc:
+        wl = self.wl
+        g = GroupDesc()
+        g.B, g.T, g.H, g.D, g.H_I, g.K, g.P = wl.B, wl.T, wl.H, 512, wl.HI, wl.K, wl.P
+        g.kv, g.kv_row_stride = self.kv.data_ptr(), KV_ROW
+        g.k_codes, g.k_code_stride = self.k_codes.data_ptr(), 32
+        g.k_scales, g.k_scale_stride = self.k_scales.data_ptr(), 4
+        g.seq_start, g.n_entries, g.max_n = self.seq_start.data_ptr(), self.n_entries.data_ptr(), self.max_n
+        g.q_pos = self.q_pos.data_ptr() if self.q_pos is not None else None
+        g.swa_cap, g.swa_start, g.swa_len = self.swa_cap, self.swa_start.data_ptr(), self.swa_len.data_ptr()
+        g.softmax_scale, g.out_dtype = self.softmax_scale, self.out_dtype
+        return g
+
+    def _layer_desc(self, l: int) -> LayerDesc:
+        ld = self.layer_data[l]
+        L = LayerDesc()
+        L.mode = _MODE[self.modes[l]]
+        L.q = ld["q"].data_ptr()
+        if "iq_codes" in ld:
+            L.iq_codes, L.iq_scales, L.iw = ld["iq_codes"].data_ptr(), ld["iq_scales"].data_ptr(), ld["iw"].data_ptr()
+        L.swa_codes, L.swa_scale = ld["swa_codes"].data_ptr(), ld["swa_scale"].data_ptr()
+        L.out, L.lse, L.idx_out = ld["out"].data_ptr(), ld["lse"].data_ptr(), ld["idx"].data_ptr()
+        return L
+
+    def run(self, stream=None) -> None:
+        csa2_layer_group(self.g, self.layer_descs, self.workspace, self.ws_bytes, stream)

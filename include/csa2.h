@@ -1,0 +1,253 @@
+/*
+ * csa2.h -- C ABI of the CSA2 (Compressed Sparse Attention 2) hot-path library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources for what each call computes (web pages about the DeepSeek V4.1 Flash report):
+ *   [A] "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径"
+ *   [B] "DeepSeek V4.1 Flash 如何靠压缩 KV 缓存实现小模型干翻大模型"
+ *
+ * Conventions shared by every call
+ *  - All array arguments are DEVICE pointers owned by the caller; the library keeps no
+ *    reference after the call returns and allocates nothing (scratch space is the
+ *    caller's `workspace`, sized by the matching *_workspace_size call).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
+ *    call only enqueues work on it: nothing synchronises the host, so results are valid
+ *    once the caller synchronises the stream.  Calls are stateless and thread-safe.
+ *  - Arguments are validated before anything is launched; a call that returns an error
+ *    has enqueued nothing.  Faults that happen on the device surface at the caller's
+ *    next synchronisation, as for any CUDA kernel.
+ *  - Strides are in BYTES for quantised buffers and in ELEMENTS for float/bf16 inputs.
+ *  - bf16 values are passed as their uint16_t bit patterns.
+ *  - Indices are int32.  Entry j of sequence b is row seq_start[b] + j of the packed
+ *    caches.  A query row is r = b * T + t.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa2_status {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,   /* a required pointer is NULL or an enum is unknown      */
+    CSA2_ERR_SHAPE = 2,         /* a size is negative, zero where it must not be, or too big */
+    CSA2_ERR_ALIGN = 3,         /* a pointer or stride breaks the 16-byte rule stated below */
+    CSA2_ERR_UNSUPPORTED = 4,   /* valid but not implemented (e.g. latent width != 512)  */
+    CSA2_ERR_CUDA = 5,          /* the CUDA runtime refused a launch                     */
+    CSA2_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (see csa2_device_error) */
+    CSA2_ERR_WORKSPACE = 7      /* workspace NULL or smaller than the size query returned */
+} csa2_status;
+
+/* quantised formats */
+#define CSA2_FMT_FP4_E2M1_E4M3S16 0   /* E2M1 codes, one E4M3 scale per 16 channels */
+#define CSA2_FMT_FP8_E4M3_TOKEN   1   /* E4M3 codes, one fp32 scale per row (token) */
+/* float element types */
+#define CSA2_DTYPE_F32  0
+#define CSA2_DTYPE_BF16 1
+/* layer modes ([B] section "CSA2：三层压缩一次吃满") */
+#define CSA2_MODE_FULL    0
+#define CSA2_MODE_REINDEX 1
+#define CSA2_MODE_REUSE   2
+
+/* Limits of this build. */
+#define CSA2_LATENT_DIM   512     /* main-KV latent width (attention)            */
+#define CSA2_INDEX_DIM    64      /* indexer key / query width                   */
+#define CSA2_MAX_INDEX_HEADS 16
+#define CSA2_MAX_TOPK     4096
+#define CSA2_MAX_POOL     32768
+#define CSA2_MAX_HEADS    128     /* main query heads; a multiple of 16          */
+#define CSA2_SWA_WINDOW   128     /* at most this many window tokens per query   */
+
+/* Human-readable name of a status code (static string, never NULL). */
+CSA2_API const char *csa2_status_string(csa2_status s);
+
+/* Library ABI version (increments on any signature change). */
+CSA2_API int csa2_version(void);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_quantize_kv -- quantise-on-write of cache rows.
+ *
+ * fmt == CSA2_FMT_FP4_E2M1_E4M3S16 ([B] section "FP4 量化 + Bounded Replay": main KV is
+ *   E2M1 with one E4M3 scale per 16 channels and no second-level scale; the indexer Q
+ *   and K use the same FP4 format):  per block of 16 channels
+ *       s = E4M3_rne_satfinite(amax / 6);  code_i = E2M1_rne_satfinite(x_i / s)
+ *   with each quotient rounded once from its exact value; s == 0 gives all-zero codes;
+ *   a negative value that rounds to zero is stored as -0 (code 8).  Two codes per byte,
+ *   channel 2i in the low nibble.  Row r writes dim/2 bytes at codes + d*code_stride and
+ *   dim/16 E4M3 bytes at scales + d*scale_stride, d = dst_rows ? dst_rows[r] : r.
+ *   dim must be a multiple of 16.
+ * fmt == CSA2_FMT_FP8_E4M3_TOKEN (the 8-bit sliding window, [A] section
+ *   "压缩吸收注意力（二代）"):  per row s = amax / 448 rounded to fp32 and stored as a
+ *   float at scales + d*scale_stride; code_i = E4M3_rne_satfinite(x_i / s) rounded once
+ *   from the exact quotient; s == 0 gives all-zero codes.  dim bytes per row.
+ *
+ * x: rows x dim elements of x_dtype (CSA2_DTYPE_F32 or CSA2_DTYPE_BF16), row r at
+ *    x + r*x_stride elements.  dst_rows: optional int64 [rows] destination rows (a cache
+ *    position, or a ring slot of the window); NULL writes row r to row r.
+ * Errors: INVALID_ARG (NULL x/codes/scales, unknown fmt or dtype), SHAPE (rows < 0,
+ *   dim <= 0 or not a multiple of 16, dim > 65536, x_stride < dim), ALIGN (scales for
+ *   FP8 not 4-byte aligned or scale_stride not a multiple of 4), CUDA.
+ * rows == 0 is a no-op returning CSA2_OK.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
+                             int64_t x_stride, uint8_t *codes, int64_t code_stride,
+                             void *scales, int64_t scale_stride, const int64_t *dst_rows,
+                             void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_index_topk -- indexer scoring + top-K block selection for Full and Reindex layers.
+ *
+ * Score ([B] section "为什么 KV 缓存成了新瓶颈？" names the DSA indexer; [B] section
+ * "FP4 量化 + Bounded Replay" makes its Q and K FP4):  for query row r and entry j
+ *     I[r, j] = sum_h w[r,h] * ReLU(q[r,h] . k[j])
+ * with q, k the dequantised FP4 vectors (64 channels), computed in fp32: each 16-channel
+ * block's partial is exact, blocks are added left to right, heads are accumulated left to
+ * right as acc = acc + w*relu(dot) without fused multiply-add, and 0 is returned as +0.
+ *
+ * Selection ([A] section "压缩吸收注意力（二代）": the first layer picks 2048 blocks and
+ * builds a candidate pool that later layers search):  the entries visible to row r are
+ * ordered by (score descending, entry index ascending); the first min(K, n) are written to
+ * out_idx[r][0..K) in ascending index order, padded with -1, and their number to
+ * out_cnt[r].
+ *   mode == CSA2_MODE_FULL: visible entries are j < n_vis(r), n_vis = n_entries[b] when
+ *     q_pos is NULL (decode) else min(n_entries[b], (q_pos[r] + 1) / 4) (entry j covers
+ *     tokens 4j..4j+3).  When P > 0 the first min(P, n) of the same order (the pool,
+ *     which contains the top-K) go to out_pool[r][0..P) ascending, padded with -1, and
+ *     their number to out_pool_len[r].
+ *   mode == CSA2_MODE_REINDEX: only the entries listed in pool[r][0..pool_len[r]) (row
+ *     stride P_in, ascending) are scored with this layer's own q and w; P must be 0.
+ *
+ * Layouts: q_codes [B*T][H_I][32] u8, q_scales [B*T][H_I][4] u8 (E4M3), w [B*T][H_I] f32;
+ *   key codes of entry row e at k_codes + e*k_code_stride (32 bytes), its 4 E4M3 scales at
+ *   k_scales + e*k_scale_stride; seq_start int64 [B]; n_entries int32 [B]; q_pos int32
+ *   [B*T] or NULL; pool int32 [B*T][P_in]; pool_len int32 [B*T].
+ *   max_n: an upper bound of n_entries[b] over the batch (sizes the launch; the device
+ *   values are not read back).
+ * Limits: 1 <= H_I <= CSA2_MAX_INDEX_HEADS, 1 <= K <= CSA2_MAX_TOPK, 0 <= P <=
+ *   CSA2_MAX_POOL, P_in <= CSA2_MAX_POOL, max_n <= 2^31-1.
+ * Workspace: csa2_index_topk_workspace_size(mode, B*T, max_n, K, P (or P_in), &bytes).
+ * Errors: INVALID_ARG, SHAPE, ALIGN (k_codes or k_code_stride not 16-byte aligned),
+ *   WORKSPACE, CUDA.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_index_topk_workspace_size(int mode, int rows, int64_t max_n, int K, int P,
+                                           size_t *bytes);
+
+CSA2_API csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uint8_t *q_scales,
+                            const float *w, int B, int T, int H_I,
+                            const uint8_t *k_codes, int64_t k_code_stride,
+                            const uint8_t *k_scales, int64_t k_scale_stride,
+                            const int64_t *seq_start, const int32_t *n_entries, int64_t max_n,
+                            const int32_t *q_pos,
+                            const int32_t *pool, const int32_t *pool_len, int P_in,
+                            int K, int32_t *out_idx, int32_t *out_cnt,
+                            int P, int32_t *out_pool, int32_t *out_pool_len,
+                            void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_sparse_attn -- attention of each query row over its selected compressed entries
+ * merged with its own 8-bit sliding window.
+ *
+ * [B] section "CSA2：三层压缩一次吃满": entries carry an MLA-style latent shared by all
+ * heads, so keys = values = the dequantised 512-wide latent; every layer keeps its own
+ * query and its own window.  [B] section "FP4 量化 + Bounded Replay": the window is
+ * truncated to the last 128 tokens.  For row r and head h, with X = {selected entries}
+ * followed by {window tokens}:
+ *     z_x = softmax_scale * (q[r,h] . v_x);   out[r,h] = sum_x softmax(z)_x v_x
+ * one joint softmax over X (the window is merged by the log-sum-exp of the two parts);
+ * lse[r,h] = log(sum_x exp(z_x)) (natural log; -inf and out = 0 when X is empty).
+ *
+ * Layouts: q bf16 [B*T][H][D]; main entry e at kv + e*kv_row_stride holds D/2 bytes of
+ *   E2M1 codes followed by D/16 E4M3 scales (288 bytes for D = 512); entry ids are
+ *   relative to seq_start[b]; idx int32 [B*T][K] (-1 = empty slot, ignored); cnt int32
+ *   [B*T] or NULL (number of leading non-negative ids; NULL = scan all K);
+ *   swa_codes u8 [B][swa_cap][D] (E4M3), swa_scale f32 [B][swa_cap]; row r uses slots
+ *   swa_start[r] .. swa_start[r]+swa_len[r]-1 of its sequence (swa_start NULL = 0);
+ *   out [B*T][H][D] of out_dtype (CSA2_DTYPE_F32 or CSA2_DTYPE_BF16); lse f32 [B*T][H]
+ *   or NULL.
+ * Limits: D == 512; H a multiple of 16, 16 <= H <= CSA2_MAX_HEADS; 1 <= K <=
+ *   CSA2_MAX_TOPK; swa_len <= CSA2_SWA_WINDOW; kv and kv_row_stride 16-byte aligned.
+ * Workspace: csa2_sparse_attn_workspace_size(B*T, H, K, &bytes).
+ * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED (D != 512), WORKSPACE, CUDA.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_sparse_attn_workspace_size(int rows, int H, int K, size_t *bytes);
+
+CSA2_API csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D,
+                             const uint8_t *kv, int64_t kv_row_stride, const int64_t *seq_start,
+                             const int32_t *idx, const int32_t *cnt, int K,
+                             const uint8_t *swa_codes, const float *swa_scale, int swa_cap,
+                             const int32_t *swa_start, const int32_t *swa_len,
+                             float softmax_scale, void *out, int out_dtype, float *lse,
+                             void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_layer_group -- one group of CSA2 layers in order ([B] section
+ * "CSA2：三层压缩一次吃满"; [A] section "压缩吸收注意力（二代）": in a group of six only
+ * the first is Full and the rest Reuse).
+ *   FULL    : csa2_index_topk(FULL) with the layer's own indexer query; when any later
+ *             layer is REINDEX the Full layer also emits the pool of size P.
+ *   REINDEX : re-scores the pool of the group's most recent Full layer with the layer's
+ *             own indexer query and takes top-K from it.
+ *   REUSE   : takes the preceding layer's selection as is (no indexer work).
+ * Every layer then runs csa2_sparse_attn with its own main query and its own window over
+ * the shared main KV.  Layers run in order on `stream`.
+ * Rejected (INVALID_ARG): a REUSE or REINDEX layer before any FULL layer; REINDEX with
+ * P == 0.
+ * ---------------------------------------------------------------------------------- */
+typedef struct csa2_group_desc {
+    int B, T, H, D, H_I, K, P;
+    const uint8_t *kv;           int64_t kv_row_stride;     /* main KV (shared)        */
+    const uint8_t *k_codes;      int64_t k_code_stride;     /* indexer keys (shared)   */
+    const uint8_t *k_scales;     int64_t k_scale_stride;
+    const int64_t *seq_start;    const int32_t *n_entries;  int64_t max_n;
+    const int32_t *q_pos;        /* NULL = decode (all entries visible)                */
+    int swa_cap;                 const int32_t *swa_start;  const int32_t *swa_len;
+    float softmax_scale;         int out_dtype;
+} csa2_group_desc;
+
+typedef struct csa2_layer_desc {
+    int mode;                    /* CSA2_MODE_*                                        */
+    const uint16_t *q;           /* main query, bf16 [B*T][H][D]                       */
+    const uint8_t *iq_codes;     /* indexer query [B*T][H_I][32] (FULL / REINDEX)      */
+    const uint8_t *iq_scales;    /* [B*T][H_I][4]                                      */
+    const float *iw;             /* indexer head weights [B*T][H_I]                    */
+    const uint8_t *swa_codes;    /* this layer's window [B][swa_cap][D]                */
+    const float *swa_scale;      /* [B][swa_cap]                                       */
+    void *out;                   /* [B*T][H][D] of out_dtype                           */
+    float *lse;                  /* [B*T][H] or NULL                                   */
+    int32_t *idx_out;            /* optional copy of this layer's selection [B*T][K]   */
+} csa2_layer_desc;
+
+CSA2_API csa2_status csa2_layer_group_workspace_size(const csa2_group_desc *g,
+                                            const csa2_layer_desc *layers, int n_layers,
+                                            size_t *bytes);
+
+CSA2_API csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *layers,
+                             int n_layers, void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_device_error -- reads (and clears) the library's device-side error word for the
+ * current device: 0 when no bounded wait has expired since the last call, otherwise a
+ * csa2_status code.  Synchronises `stream` first.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_device_error(void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_launch_count -- number of kernels this library has launched in this process
+ * (all devices, all streams) since it was loaded.  A diagnostic for benchmarks.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API uint64_t csa2_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

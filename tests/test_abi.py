@@ -1,0 +1,132 @@
+"""The C-ABI library loads, exports every declared symbol, and validates arguments on the host.
+
+No call here reaches the GPU: every case returns from argument validation before any launch.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import compressed_sparse_attention_quantize_b200 as csa2
+from compressed_sparse_attention_quantize_b200 import build as csa2_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa2.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT, WS = range(8)
+
+
+@pytest.fixture(scope="module")
+def L():
+    csa2_build.build()
+    return csa2.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"CSA2_API\s+[\w\s\*]*?\b(csa2_\w+)\s*\(", text)
+
+
+def test_header_declares_the_four_calls():
+    names = set(declared_functions())
+    for n in ("csa2_quantize_kv", "csa2_index_topk", "csa2_sparse_attn", "csa2_layer_group"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", csa2.library_path()], text=True)
+    exported = set(re.findall(r"\bT (csa2_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(L, n)
+
+
+def test_status_strings(L):
+    for s in range(8):
+        assert csa2.csa2_status_string(s).startswith("CSA2")
+    assert csa2.csa2_version() >= 1
+
+
+def test_quantize_validation(L):
+    q = L.csa2_quantize_kv
+    # unknown format / dtype
+    assert q(7, 16, 0, 4, 512, 512, 16, 256, 16, 32, None, None) == INVALID
+    assert q(0, 16, 5, 4, 512, 512, 16, 256, 16, 32, None, None) == INVALID
+    # dim not a multiple of 16, stride smaller than dim
+    assert q(0, 16, 0, 4, 500, 512, 16, 256, 16, 32, None, None) == SHAPE
+    assert q(0, 16, 0, 4, 512, 100, 16, 256, 16, 32, None, None) == SHAPE
+    # rows == 0 is a no-op
+    assert q(0, None, 0, 0, 512, 512, None, 256, None, 32, None, None) == OK
+    # NULL input with rows > 0
+    assert q(0, None, 0, 4, 512, 512, 16, 256, 16, 32, None, None) == INVALID
+    # FP8 scales must be 4-byte aligned
+    assert q(1, 16, 0, 4, 512, 512, 16, 512, 18, 4, None, None) == ALIGN
+
+
+def _attn(L, **kw):
+    a = dict(q=16, B=1, T=1, H=64, D=512, kv=16, kv_row_stride=288, seq_start=16, idx=16, cnt=None,
+             K=64, swa_codes=16, swa_scale=16, swa_cap=128, swa_start=None, swa_len=16,
+             softmax_scale=1.0, out=16, out_dtype=0, lse=None, workspace=16, ws_bytes=1 << 40,
+             stream=None)
+    a.update(kw)
+    return L.csa2_sparse_attn(a["q"], a["B"], a["T"], a["H"], a["D"], a["kv"], a["kv_row_stride"],
+                              a["seq_start"], a["idx"], a["cnt"], a["K"], a["swa_codes"], a["swa_scale"],
+                              a["swa_cap"], a["swa_start"], a["swa_len"], ctypes.c_float(a["softmax_scale"]),
+                              a["out"], a["out_dtype"], a["lse"], a["workspace"], a["ws_bytes"], a["stream"])
+
+
+def test_attn_validation(L):
+    assert _attn(L, D=256) == UNSUP
+    assert _attn(L, H=24) == SHAPE
+    assert _attn(L, K=0) == SHAPE
+    assert _attn(L, K=5000) == SHAPE
+    assert _attn(L, kv=24) == ALIGN
+    assert _attn(L, kv_row_stride=300) == ALIGN
+    assert _attn(L, q=None) == INVALID
+    assert _attn(L, out_dtype=9) == INVALID
+    assert _attn(L, workspace=None) == WS
+    assert _attn(L, ws_bytes=10) == WS
+
+
+def test_workspace_queries():
+    assert csa2.csa2_sparse_attn_workspace_size(32, 64, 2048) > 0
+    assert csa2.csa2_index_topk_workspace_size(0, 32, 32768, 2048, 0) > 0
+    assert csa2.csa2_index_topk_workspace_size(1, 16, 65536, 2048, 16000) > 0
+
+
+def _group(modes, P=0):
+    g = csa2.GroupDesc()
+    g.B, g.T, g.H, g.D, g.H_I, g.K, g.P = 2, 1, 64, 512, 8, 64, P
+    g.kv, g.kv_row_stride = 16, 288
+    g.k_codes, g.k_code_stride, g.k_scales, g.k_scale_stride = 16, 32, 16, 4
+    g.seq_start, g.n_entries, g.max_n = 16, 16, 1000
+    g.swa_cap, g.swa_len = 128, 16
+    g.softmax_scale = 1.0
+    layers = []
+    for m in modes:
+        Ld = csa2.LayerDesc()
+        Ld.mode = m
+        Ld.q, Ld.iq_codes, Ld.iq_scales, Ld.iw, Ld.swa_codes, Ld.swa_scale, Ld.out = (16,) * 7
+        layers.append(Ld)
+    return g, layers
+
+
+def test_layer_group_mode_table_validation(L):
+    F, I, U = csa2.MODE_FULL, csa2.MODE_REINDEX, csa2.MODE_REUSE
+    g, layers = _group([U, F])
+    with pytest.raises(csa2.CSA2Error, match="INVALID_ARG"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    g, layers = _group([F, I])          # Reindex needs a pool
+    with pytest.raises(csa2.CSA2Error, match="INVALID_ARG"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    g, layers = _group([F, I, U], P=300)
+    assert csa2.csa2_layer_group_workspace_size(g, layers) > 0
+    g, layers = _group([F, 7])
+    with pytest.raises(csa2.CSA2Error, match="INVALID_ARG"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    # too-small workspace is refused before anything is launched
+    g, layers = _group([F, U])
+    arr = (csa2.LayerDesc * 2)(*layers)
+    assert L.csa2_layer_group(ctypes.byref(g), arr, 2, 16, 8, None) == WS

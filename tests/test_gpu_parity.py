@@ -1,0 +1,186 @@
+"""CUDA path vs oracle, through the C ABI, on seeded synthetic inputs.
+
+Bit-exact: FP4 codes and scales, FP8 window codes and scales, top-K index sets and pools.
+Attention: relative L2 <= 1e-3 and max-abs <= 2e-3 * RMS(reference) per query row.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import compressed_sparse_attention_quantize_b200 as csa2
+from compressed_sparse_attention_quantize_b200 import runtime, synth
+from tests._parity import OracleSeq, check_attention
+
+pytestmark = pytest.mark.gpu
+
+
+def _special_rows(rng, rows, dim):
+    x = rng.standard_normal((rows, dim)).astype(np.float32)
+    x *= np.exp2(rng.integers(-20, 12, (rows, 1))).astype(np.float32)
+    x[0] = 0.0
+    x[1, :16] = np.float32(-1e-7)
+    x[2, :16] = np.array([6, 5, 3.5, 2.5, 1.75, 1.25, .75, .25, -6, -5, -3.5, -2.5, -1.75, -1.25, -.75, -.25],
+                         np.float32)
+    x[3, 7] = 3e5
+    x[4] = 448.0 * np.sin(np.arange(dim, dtype=np.float32))
+    x[5, ::3] *= 8
+    return x
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_fp4_bitexact(dtype):
+    rng = np.random.default_rng(100)
+    x = _special_rows(rng, 777, 512)
+    xt = torch.from_numpy(x).cuda()
+    if dtype == "bf16":
+        xt = xt.to(torch.bfloat16)
+        x = xt.float().cpu().numpy()
+    codes = torch.zeros((777, 288), dtype=torch.uint8, device="cuda")
+    runtime.quantize_fp4_rows(xt, codes, codes[:, 256:], 288, 288)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.quantize_fp4(x)
+    got = codes.cpu().numpy()
+    assert np.array_equal(got[:, :256], oc)
+    assert np.array_equal(got[:, 256:], os_)
+
+
+def test_quantize_fp4_scatter_rows():
+    rng = np.random.default_rng(101)
+    x = rng.standard_normal((10, 64)).astype(np.float32)
+    dst = torch.tensor([9, 3, 0, 17, 4, 5, 6, 7, 8, 1], dtype=torch.int64, device="cuda")
+    codes = torch.zeros((20, 32), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((20, 4), dtype=torch.uint8, device="cuda")
+    runtime.quantize_fp4_rows(torch.from_numpy(x).cuda(), codes, scales, 32, 4, dst_rows=dst)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.quantize_fp4(x)
+    d = dst.cpu().numpy()
+    assert np.array_equal(codes.cpu().numpy()[d], oc)
+    assert np.array_equal(scales.cpu().numpy()[d], os_)
+    assert not codes.cpu().numpy()[[2, 10, 19]].any()
+
+
+def test_quantize_fp8_token_bitexact():
+    rng = np.random.default_rng(102)
+    x = _special_rows(rng, 300, 512)
+    # rows whose scale is exactly 1 put many values on E4M3 ties
+    x[10] = np.float32(448.0)
+    x[10, 1:100] = np.linspace(200, 250, 99, dtype=np.float32)
+    xt = torch.from_numpy(x).cuda()
+    codes = torch.empty((300, 512), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((300,), dtype=torch.float32, device="cuda")
+    runtime.quantize_fp8_rows(xt, codes, scales)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.quantize_fp8_token(x)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), oc)
+
+
+def _run_group(wl, layers=None, out_dtype=csa2.DTYPE_F32, scale=None):
+    r = runtime.GroupRunner(wl, out_dtype=out_dtype, softmax_scale=scale, layers=layers)
+    r.run()
+    torch.cuda.synchronize()
+    return r
+
+
+def _check_caches(r, wl, seqs):
+    kv = r.kv.cpu().numpy()
+    kc = r.k_codes.cpu().numpy()
+    ks = r.k_scales.cpu().numpy()
+    starts = r.seq_start.cpu().numpy()
+    for b, os_ in seqs.items():
+        s0, n = int(starts[b]), wl.n_entries[b]
+        assert np.array_equal(kv[s0:s0 + n], os_.kv_rows)
+        assert np.array_equal(kc[s0:s0 + n], os_.k_codes)
+        assert np.array_equal(ks[s0:s0 + n], os_.k_scales)
+
+
+def _check_rows(r, wl, rows, check_attn=True):
+    seqs = {}
+    for row in rows:
+        b, t = divmod(row, wl.T)
+        if b not in seqs:
+            seqs[b] = OracleSeq(wl, b)
+        os_ = seqs[b]
+        sel = os_.indices(t, r.modes)
+        for l in range(len(r.modes)):
+            idx, cnt = sel[l]
+            got = r.layer_data[l]["idx"][row].cpu().numpy()
+            assert np.array_equal(got, idx), f"layer {l} row {row}: index set differs"
+            if check_attn:
+                out, lse = os_.attention(l, t, idx, r.softmax_scale)
+                g_out = r.layer_data[l]["out"][row].float().cpu().numpy()
+                check_attention(g_out, out, f"layer {l} row {row}")
+                g_lse = r.layer_data[l]["lse"][row].cpu().numpy()
+                fin = np.isfinite(lse)
+                assert np.array_equal(np.isfinite(g_lse), fin)
+                assert np.all(np.abs(g_lse[fin] - lse[fin]) <= 1e-3)
+    return seqs
+
+
+def test_config0_tiny_full_layer():
+    wl = synth.workload(0)
+    r = _run_group(wl)
+    seqs = _check_rows(r, wl, [0])
+    _check_caches(r, wl, seqs)
+
+
+@pytest.mark.parametrize("scale", [None, 1.0])
+def test_ragged_batch_full_reuse(scale):
+    wl = synth.scaled(synth.workload(1), B=4, n=[1000, 0, 37, 4500], K=64, H=32,
+                      name="ragged_full_reuse")
+    r = _run_group(wl, layers=3, scale=scale)
+    seqs = _check_rows(r, wl, range(4))
+    _check_caches(r, wl, seqs)
+    # Reuse layers select exactly what the Full layer selected
+    for l in (1, 2):
+        assert torch.equal(r.layer_data[l]["idx"], r.layer_data[0]["idx"])
+    # the empty sequence with an empty window gives zeros and lse = -inf
+    assert not r.layer_data[0]["out"][1].any()
+
+
+def test_reindex_group_scaled():
+    wl = synth.scaled(synth.workload(2), B=3, n=[3000, 5000, 700], K=128, P=1000,
+                      name="reindex_scaled")
+    r = _run_group(wl)
+    _check_rows(r, wl, range(3))
+
+
+def test_long_rows_scaled():
+    wl = synth.scaled(synth.workload(3), B=2, n=[70000, 41000], K=512, name="long_scaled")
+    r = _run_group(wl, layers=2)
+    _check_rows(r, wl, range(2))
+
+
+def test_prefill_scaled():
+    wl = synth.scaled(synth.workload(4), n=2000, T=96, K=256, name="prefill_scaled")
+    r = _run_group(wl)
+    _check_rows(r, wl, [0, 1, 2, 3, 47, 95])
+    # causal: no selected entry lies beyond the query's visible range
+    nv = wl.n_visible(0)
+    idx = r.layer_data[0]["idx"].cpu().numpy()
+    for t in range(wl.T):
+        assert idx[t].max() < nv[t]
+
+
+def test_bf16_output():
+    wl = synth.scaled(synth.workload(1), B=2, n=3000, K=128, name="bf16_out")
+    r = _run_group(wl, layers=1, out_dtype=csa2.DTYPE_BF16)
+    for row in range(2):
+        os_ = OracleSeq(wl, row)
+        idx, _ = os_.indices(0, r.modes)[0]
+        out, _ = os_.attention(0, 0, idx, r.softmax_scale)
+        ref = torch.from_numpy(out).float().to(torch.bfloat16).float().numpy()
+        got = r.layer_data[0]["out"][row].float().cpu().numpy()
+        # bf16 rounding of the output itself is ~2^-9 relative; compare to the rounded reference
+        assert np.linalg.norm(got - ref) <= 4e-3 * np.linalg.norm(ref)
+
+
+@pytest.mark.parametrize("cfg,rows", [(1, [0, 17, 31]), (2, [0, 15]), (3, [0, 3]), (4, [0, 1000, 4095])])
+def test_full_size_sampled(cfg, rows):
+    """Full-size workloads in the bench's launch configuration; sampled rows vs the oracle."""
+    wl = synth.workload(cfg)
+    r = _run_group(wl)
+    _check_rows(r, wl, rows)
