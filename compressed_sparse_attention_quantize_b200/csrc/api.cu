@@ -111,8 +111,8 @@ csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, 
                              int64_t scale_stride, const int64_t *dst_rows, void *stream) {
     if (fmt != CSA2_FMT_FP4_E2M1_E4M3S16 && fmt != CSA2_FMT_FP8_E4M3_TOKEN) return CSA2_ERR_INVALID_ARG;
     if (x_dtype != CSA2_DTYPE_F32 && x_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
+    if (rows == 0) return CSA2_OK;                               // no-op, whatever the strides
     if (rows < 0 || dim <= 0 || (dim % 16) || dim > 65536 || x_stride < dim) return CSA2_ERR_SHAPE;
-    if (rows == 0) return CSA2_OK;
     if (!x || !codes || !scales) return CSA2_ERR_INVALID_ARG;
     if (fmt == CSA2_FMT_FP4_E2M1_E4M3S16) {
         if (code_stride < dim / 2 || scale_stride < dim / 16) return CSA2_ERR_SHAPE;

@@ -97,7 +97,7 @@ CSA2_API int csa2_version(void);
  * Errors: INVALID_ARG (NULL x/codes/scales, unknown fmt or dtype), SHAPE (rows < 0,
  *   dim <= 0 or not a multiple of 16, dim > 65536, x_stride < dim), ALIGN (scales for
  *   FP8 not 4-byte aligned or scale_stride not a multiple of 4), CUDA.
- * rows == 0 is a no-op returning CSA2_OK.
+ * rows == 0 is a no-op returning CSA2_OK (checked after fmt and x_dtype, before the rest).
  * ---------------------------------------------------------------------------------- */
 CSA2_API csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
                              int64_t x_stride, uint8_t *codes, int64_t code_stride,

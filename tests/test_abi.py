@@ -59,6 +59,7 @@ def test_quantize_validation(L):
     assert q(0, 16, 0, 4, 512, 100, 16, 256, 16, 32, None, None) == SHAPE
     # rows == 0 is a no-op
     assert q(0, None, 0, 0, 512, 512, None, 256, None, 32, None, None) == OK
+    assert q(0, None, 0, 0, 512, 1, None, 256, None, 32, None, None) == OK   # empty tensor strides
     # NULL input with rows > 0
     assert q(0, None, 0, 4, 512, 512, 16, 256, 16, 32, None, None) == INVALID
     # FP8 scales must be 4-byte aligned
