@@ -23,10 +23,18 @@ struct AttnArgs {
     float *lse;
     float *partials;            // workspace
     int splits;
+    int hgroups;                // head groups of 64 (tensor-core kernel)
+    int keys_per_split;         // keys handled by one split (tensor-core kernel)
 };
+
+// Floats of one tensor-core split partial: running max[64], row sum[64], O[64][512].
+constexpr int kPartialFloats = 2 * 64 + 64 * 512;
 
 cudaError_t launch_attn_simt(AttnArgs a, cudaStream_t st);
 size_t simt_workspace_bytes(int rows, int H, int K);
+
+cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st);
+size_t tc_workspace_bytes(int rows, int H, int K);
 
 // Dispatch used by the C ABI.
 size_t attn_workspace_bytes(int rows, int H, int K);

@@ -1,0 +1,587 @@
+// Sparse attention on the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+//
+// [B] page "DeepSeek V4.1 Flash 如何靠压缩 KV 缓存实现小模型干翻大模型", section
+// "CSA2：三层压缩一次吃满": every layer keeps its own query and window and attends over the
+// selected compressed entries, whose MLA-style latent is shared by the heads (keys = values =
+// the 512-wide latent).  Section "FP4 量化 + Bounded Replay": entries are E2M1 with one E4M3
+// scale per 16 channels; the window is the last 128 tokens, 8-bit.
+//
+// One CTA = (query row, group of 64 heads, split of the row's key list: selected entries
+// followed by window tokens).  Per tile of 128 keys:
+//   S^T[key, head] = V . Q^T   tcgen05.mma kind::f16, M=128 keys, N=64 heads, K=512 channels;
+//                              A = V (K-major), B = Q (K-major), fp32 accumulator in TMEM.
+//   online softmax             4 warps read S^T from TMEM (one key per thread), log2 domain,
+//                              lazy rescale: the running max moves only when a tile's max
+//                              exceeds it by more than 2^8.
+//   O^T[chan, head] += V^T.P^T four MMAs M=128 channels, N=64 heads, K=128 keys; A = the same
+//                              V bytes read as an MN-major operand, B = P^T (MN-major fp16).
+// V is dequantised once per tile into fp16 (E2M1 x E4M3 is exact in fp16); the window's
+// per-token fp32 scale is applied to the logit and folded into P instead.  Q is converted to
+// fp16 with a power-of-two pre-scale so small values keep full precision.
+//
+// Warp roles (9 warps): 0 = TMEM owner + MMA issuer; 1-4 = softmax/epilogue (TMEM
+// subpartitions 1,2,3,0); 5-8 = dequantisers (one key per thread).  Hand-offs use mbarriers
+// per V region (64 channels) so dequantising tile j+1 overlaps the P.V products of tile j.
+// Every wait is bounded: on expiry the CTA records CSA2_ERR_TIMEOUT, drains, frees TMEM and exits.
+#include "attn.cuh"
+#include "tc_ptx.cuh"
+
+namespace csa2 {
+
+namespace tc {
+
+constexpr int kTile = 128;                 // keys per tile (MMA M)
+constexpr int kHeads = 64;                 // heads per CTA (MMA N)
+constexpr int kRegions = 8;                // 64-channel blocks of the 512-wide latent
+constexpr int kQRegion = kHeads * 128;     // 8 KB
+constexpr int kVRegion = kTile * 128;      // 16 KB
+constexpr int kQBytes = kRegions * kQRegion;         // 64 KB
+constexpr int kVBytes = kRegions * kVRegion;         // 128 KB
+constexpr int kPBytes = kTile * kHeads * 2;          // 16 KB
+constexpr int kThreads = 288;
+constexpr int kSoftmaxWarp0 = 1, kDequantWarp0 = 5;
+constexpr int kTmemCols = 512;
+constexpr int kOCol = 256;                 // O^T accumulators at columns 256..511
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct Smem {
+    uint64_t v_full[kRegions];
+    uint64_t v_empty[kRegions];
+    uint64_t s_full, s_empty, p_full, pv_done, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int any_rescale;
+    int q_exp_max;
+    float m_run[kHeads];
+    float alpha[kHeads];
+    float red[4][kHeads];
+    float lsum[4][kHeads];
+};
+
+constexpr int kSmemBytes = kQBytes + kVBytes + kPBytes + (int)sizeof(Smem) + 1024;
+
+// Where key x of row r comes from.
+struct KeySrc {
+    bool valid, swa;
+    const uint8_t *ptr;      // main: 288-byte row; window: 512 E4M3 codes
+    float scale;             // window token scale (1 for main entries, 0 if invalid)
+};
+
+CSA2_D KeySrc key_source(const AttnArgs &a, int r, int b, int x, int x_end, int n_sel) {
+    KeySrc k{false, false, nullptr, 0.0f};
+    if (x >= x_end) return k;
+    if (x < n_sel) {
+        const int32_t e = a.idx[(int64_t)r * a.K + x];
+        if (e < 0) return k;
+        k.valid = true;
+        k.ptr = a.kv + (a.seq_start[b] + e) * a.kv_row_stride;
+        k.scale = 1.0f;
+    } else {
+        const int slot = (a.swa_start ? a.swa_start[r] : 0) + (x - n_sel);
+        const int64_t srow = (int64_t)b * a.swa_cap + slot;
+        k.valid = true;
+        k.swa = true;
+        k.ptr = a.swa_codes + srow * kLatent;
+        k.scale = a.swa_scale[srow];
+    }
+    return k;
+}
+
+// Transpose-reduce 32 values across a warp: afterwards v[0] of lane L holds the max (or sum)
+// over the 32 lanes of element L.  31 shuffles instead of 32 x 5.
+template <bool kSum>
+CSA2_D void warp_transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+    for (int off = 16, n = 16; off >= 1; off >>= 1, n >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float send = upper ? v[i] : v[i + n];
+            const float keep = upper ? v[i + n] : v[i];
+            const float got = __shfl_xor_sync(0xffffffffu, send, off);
+            v[i] = kSum ? keep + got : fmaxf(keep, got);
+        }
+    }
+}
+
+// swizzled 16-byte chunk c of row `row` inside a 128B-swizzled region
+CSA2_D uint32_t sw128_off(int row, int c) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(AttnArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sQ = base;
+    uint8_t *sV = base + kQBytes;
+    uint8_t *sP = sV + kVBytes;
+    Smem &S = *reinterpret_cast<Smem *>(sP + kPBytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x;                       // query row
+    const int hg = blockIdx.y;                      // head group
+    const int split = blockIdx.z;
+    const int b = r / a.T;
+    const int h0 = hg * kHeads;
+
+    const int n_sel = a.cnt ? a.cnt[r] : a.K;
+    const int total = n_sel + a.swa_len[r];
+    const int x_begin = split * a.keys_per_split;
+    const int x_end = min(total, x_begin + a.keys_per_split);
+    const int ntiles = x_end > x_begin ? (x_end - x_begin + kTile - 1) / kTile : 0;
+
+    // ---------------- setup ----------------
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRegions; ++i) {
+            ptx::mbar_init(&S.v_full[i], 128);
+            ptx::mbar_init(&S.v_empty[i], 1);
+        }
+        ptx::mbar_init(&S.s_full, 1);
+        ptx::mbar_init(&S.s_empty, 128);
+        ptx::mbar_init(&S.p_full, 128);
+        ptx::mbar_init(&S.pv_done, 1);
+        ptx::mbar_init(&S.drain, 1);
+        S.abort_flag = 0;
+        S.any_rescale = 0;
+        S.q_exp_max = 0;
+        ptx::fence_async_smem();
+    }
+    if (threadIdx.x < kHeads) S.m_run[threadIdx.x] = -INFINITY;
+    if (threadIdx.x < 4 * kHeads) S.lsum[threadIdx.x / kHeads][threadIdx.x % kHeads] = 0.0f;
+    if (warp == 0) {
+        ptx::tmem_alloc(&S.tmem_base, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    // Q: largest bf16 exponent of this head group -> power-of-two pre-scale for fp16
+    const uint16_t *qrow = a.q + (int64_t)r * a.H * kLatent;
+    const int hcount = min(kHeads, a.H - h0);
+    {
+        int emax = 0;
+        for (int i = threadIdx.x; i < hcount * (kLatent / 8); i += kThreads) {
+            const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
+            const uint4 v = *reinterpret_cast<const uint4 *>(qrow + (int64_t)(h0 + h) * kLatent + c8 * 8);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                emax = max(emax, (int)((w[k] >> 7) & 0xFFu));
+                emax = max(emax, (int)((w[k] >> 23) & 0xFFu));
+            }
+        }
+        emax = __reduce_max_sync(0xffffffffu, emax);
+        __syncthreads();
+        if (lane == 0) atomicMax(&S.q_exp_max, emax);
+    }
+    __syncthreads();
+    // fp16 holds up to 2^15 comfortably: scale so the largest |q| lands in [2^13, 2^14)
+    const int qshift = S.q_exp_max == 0 ? 0 : (13 - (S.q_exp_max - 127));
+    const float qmul = exp2f((float)qshift);
+    for (int i = threadIdx.x; i < kHeads * (kLatent / 8); i += kThreads) {
+        const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
+        uint32_t packed[4] = {0u, 0u, 0u, 0u};
+        if (h < hcount) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(qrow + (int64_t)(h0 + h) * kLatent + c8 * 8);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float lo = __uint_as_float(w[k] << 16) * qmul;
+                const float hi = __uint_as_float(w[k] & 0xFFFF0000u) * qmul;
+                __half2 hh = __floats2half2_rn(lo, hi);
+                packed[k] = *reinterpret_cast<uint32_t *>(&hh);
+            }
+        }
+        const int region = c8 >> 3, chunk = c8 & 7;
+        *reinterpret_cast<uint4 *>(sQ + region * kQRegion + sw128_off(h, chunk)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+    ptx::fence_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort_flag = &S.abort_flag;
+
+    if (warp == 0) {
+        // ================= MMA issuer =================
+        const uint32_t idesc_s = ptx::idesc_f16_f32(128, kHeads, false, false);
+        const uint32_t idesc_pv = ptx::idesc_f16_f32(128, kHeads, true, true);
+        const uint32_t q_addr = ptx::smem_u32(sQ), v_addr = ptx::smem_u32(sV), p_addr = ptx::smem_u32(sP);
+        for (int j = 0; j < ntiles; ++j) {
+            const uint32_t ph = j & 1;
+            if (j > 0) {
+                ptx::mbar_wait(&S.s_empty, ph ^ 1, abort_flag);
+                __syncwarp();
+                if (*abort_flag) break;
+            }
+            bool ok = true;
+            for (int rg = 0; rg < kRegions && ok; ++rg) {
+                ptx::mbar_wait(&S.v_full[rg], ph, abort_flag);
+                __syncwarp();
+                if (*abort_flag) { ok = false; break; }
+                ptx::tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = ptx::sdesc_sw128(v_addr + rg * kVRegion + k * 32, 16, 1024);
+                        const uint64_t bd = ptx::sdesc_sw128(q_addr + rg * kQRegion + k * 32, 16, 1024);
+                        ptx::mma_f16_ss(tmem, ad, bd, idesc_s, (rg | k) != 0);
+                    }
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) ptx::mma_commit(&S.s_full);
+            __syncwarp();
+            ptx::mbar_wait(&S.p_full, ph, abort_flag);
+            __syncwarp();
+            if (*abort_flag) break;
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        const uint64_t ad = ptx::sdesc_sw128(v_addr + 2 * mb * kVRegion + kk * 2048, kVRegion, 1024);
+                        const uint64_t bd = ptx::sdesc_sw128(p_addr + kk * 2048, kPBytes, 1024);
+                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, ad, bd, idesc_pv, (j > 0 || kk > 0));
+                    }
+                    ptx::mma_commit(&S.v_empty[2 * mb]);
+                    ptx::mma_commit(&S.v_empty[2 * mb + 1]);
+                }
+                ptx::mma_commit(&S.pv_done);
+            }
+            __syncwarp();
+        }
+        // every issued MMA must have completed before TMEM is released (also after an abort)
+        if (lane == 0) ptx::mma_commit(&S.drain);
+        __syncwarp();
+        ptx::mbar_wait_drain(&S.drain, 0);
+    } else if (warp >= kDequantWarp0) {
+        // ================= dequantisers: thread t <-> key t of the tile =================
+        const int t = threadIdx.x - kDequantWarp0 * 32;
+        for (int j = 0; j < ntiles; ++j) {
+            const uint32_t ph = j & 1;
+            const KeySrc src = key_source(a, r, b, x_begin + j * kTile + t, x_end, n_sel);
+            uint4 codes[16], scl[2];
+            if (src.valid && !src.swa) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) codes[i] = __ldg(p + i);
+                scl[0] = __ldg(p + 16);
+                scl[1] = __ldg(p + 17);
+            }
+            bool ok = true;
+#pragma unroll
+            for (int rg = 0; rg < kRegions; ++rg) {
+                uint4 out[8];
+                if (!src.valid) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) out[c] = make_uint4(0u, 0u, 0u, 0u);
+                } else if (!src.swa) {
+                    const uint4 sq = rg < 4 ? scl[0] : scl[1];
+                    const uint32_t sw = (rg & 3) == 0 ? sq.x : (rg & 3) == 1 ? sq.y : (rg & 3) == 2 ? sq.z : sq.w;
+                    const uint4 c0 = codes[2 * rg], c1 = codes[2 * rg + 1];
+                    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    const uint32_t s01 = ptx::e4m3x2_to_f16x2((uint16_t)(sw & 0xFFFFu));
+                    const uint32_t s23 = ptx::e4m3x2_to_f16x2((uint16_t)(sw >> 16));
+                    const uint32_t sc[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                                            __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
+#pragma unroll
+                    for (int wi = 0; wi < 8; ++wi) {           // word wi = channels 8wi..8wi+7
+                        uint32_t hv[4];
+                        ptx::e2m1x8_to_f16x8(words[wi], hv);
+                        const uint32_t s = sc[wi >> 1];
+                        out[wi] = make_uint4(ptx::hmul2_u32(hv[0], s), ptx::hmul2_u32(hv[1], s),
+                                             ptx::hmul2_u32(hv[2], s), ptx::hmul2_u32(hv[3], s));
+                    }
+                } else {
+                    const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr + rg * 64);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 v = __ldg(p + i);          // 16 codes = channels 16i..16i+15
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t hv[8];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            hv[2 * k] = ptx::e4m3x2_to_f16x2((uint16_t)(w[k] & 0xFFFFu));
+                            hv[2 * k + 1] = ptx::e4m3x2_to_f16x2((uint16_t)(w[k] >> 16));
+                        }
+                        out[2 * i] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                        out[2 * i + 1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+                    }
+                }
+                if (j > 0) {
+                    if (!ptx::mbar_wait(&S.v_empty[rg], ph ^ 1, abort_flag)) { ok = false; break; }
+                }
+                uint8_t *dst = sV + rg * kVRegion;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + sw128_off(t, c)) = out[c];
+                ptx::fence_async_smem();
+                ptx::mbar_arrive(&S.v_full[rg]);
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ================= softmax / epilogue: thread s <-> TMEM lane s (key s) =================
+        const int sub = warp & 3;
+        const int s = sub * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
+        const float qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-qshift);
+        bool aborted = false;
+        for (int j = 0; j < ntiles; ++j) {
+            const uint32_t ph = j & 1;
+            const KeySrc src = key_source(a, r, b, x_begin + j * kTile + s, x_end, n_sel);
+            ptx::mbar_wait(&S.s_full, ph, abort_flag);
+            ptx::named_barrier(1, 128);
+            if (*abort_flag) { aborted = true; break; }
+            ptx::tc_fence_after();
+            float z[kHeads];
+            {
+                uint32_t u[32];
+                ptx::tmem_ld32(lane_addr + 0, u);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(u[i]);
+                ptx::tmem_ld32(lane_addr + 32, u);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[32 + i] = __uint_as_float(u[i]);
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&S.s_empty);
+            const float zs = qk_scale * src.scale;
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) z[h] = src.valid ? z[h] * zs : -INFINITY;
+            // per-head max over this warp's 32 keys, 32 heads at a time: lane L ends with head L
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = z[half * 32 + i];
+                warp_transpose_reduce<false>(v, lane);
+                S.red[sub][half * 32 + lane] = v[0];
+            }
+            ptx::named_barrier(1, 128);
+            if (s < kHeads) {
+                const float tmax = fmaxf(fmaxf(S.red[0][s], S.red[1][s]), fmaxf(S.red[2][s], S.red[3][s]));
+                const float mo = S.m_run[s];
+                float al = 1.0f;
+                if (tmax > mo + kRescaleThreshold || (mo == -INFINITY && tmax > -INFINITY)) {
+                    S.m_run[s] = tmax;
+                    al = (mo == -INFINITY) ? 0.0f : ptx::ex2(mo - tmax);
+                    if (j > 0 && mo != -INFINITY) S.any_rescale = 1;
+                }
+                S.alpha[s] = al;
+            }
+            ptx::named_barrier(1, 128);
+            const bool rescale = S.any_rescale != 0;
+            // probabilities (log2 domain); P^T line of key s as fp16 (window scale folded in)
+            uint32_t pw[kHeads / 2];
+#pragma unroll
+            for (int h = 0; h < kHeads; h += 2) {
+                const float m0 = S.m_run[h], m1 = S.m_run[h + 1];
+                z[h] = (m0 == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[h] - m0);
+                z[h + 1] = (m1 == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[h + 1] - m1);
+                __half2 hp = __floats2half2_rn(z[h] * src.scale, z[h + 1] * src.scale);
+                pw[h / 2] = *reinterpret_cast<uint32_t *>(&hp);
+            }
+            // this tile's row sums: lane L of warp `sub` owns heads L and 32+L
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = z[half * 32 + i];
+                warp_transpose_reduce<true>(v, lane);
+                const int h = half * 32 + lane;
+                S.lsum[sub][h] = S.lsum[sub][h] * S.alpha[h] + v[0];
+            }
+            if (j > 0) {
+                ptx::mbar_wait(&S.pv_done, ph ^ 1, abort_flag);
+                ptx::named_barrier(1, 128);
+                if (*abort_flag) { aborted = true; break; }
+                ptx::tc_fence_after();
+                if (rescale) {
+                    for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            uint32_t u[32];
+                            const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
+                            ptx::tmem_ld32(addr, u);
+                            ptx::tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                u[i] = __float_as_uint(__uint_as_float(u[i]) * S.alpha[half * 32 + i]);
+                            ptx::tmem_st32(addr, u);
+                        }
+                    }
+                    ptx::tmem_st_wait();
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(sP + sw128_off(s, c)) =
+                    make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            ptx::fence_async_smem();
+            ptx::tc_fence_before();
+            ptx::named_barrier(1, 128);
+            if (s == 0) S.any_rescale = 0;
+            ptx::mbar_arrive(&S.p_full);
+        }
+        // ---------------- epilogue ----------------
+        if (!aborted && ntiles > 0) {
+            ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag);
+            ptx::named_barrier(1, 128);
+            aborted = *abort_flag != 0;
+            ptx::tc_fence_after();
+        }
+        if (!aborted) {
+            const bool single = a.splits == 1;
+            const int64_t part_idx = ((int64_t)r * a.hgroups + hg) * a.splits + split;
+            float *part = a.partials + part_idx * kPartialFloats;
+            if (s < kHeads) {
+                const float l = ntiles > 0 ? S.lsum[0][s] + S.lsum[1][s] + S.lsum[2][s] + S.lsum[3][s] : 0.0f;
+                S.red[0][s] = l;
+                if (!single) {
+                    part[s] = ntiles > 0 ? S.m_run[s] : -INFINITY;
+                    part[kHeads + s] = l;
+                } else if (a.lse && h0 + s < a.H) {
+                    a.lse[(int64_t)r * a.H + h0 + s] =
+                        (l > 0.0f) ? (S.m_run[s] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                }
+            }
+            ptx::named_barrier(1, 128);
+            for (int mb = 0; mb < 4; ++mb) {
+                const int c = mb * 128 + s;             // this thread's channel
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t u[32];
+                    if (ntiles > 0) {
+                        ptx::tmem_ld32(lane_addr + kOCol + mb * kHeads + half * 32, u);
+                        ptx::tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = 0u;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int h = half * 32 + i;
+                        if (h0 + h >= a.H) continue;
+                        const float o = __uint_as_float(u[i]);
+                        if (!single) {
+                            part[2 * kHeads + h * kLatent + c] = o;
+                        } else {
+                            const float l = S.red[0][h];
+                            const float val = l > 0.0f ? o / l : 0.0f;
+                            const int64_t oi = ((int64_t)r * a.H + h0 + h) * kLatent + c;
+                            if (a.out_dtype == CSA2_DTYPE_F32)
+                                reinterpret_cast<float *>(a.out)[oi] = val;
+                            else
+                                reinterpret_cast<__nv_bfloat16 *>(a.out)[oi] = __float2bfloat16_rn(val);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // ---------------- teardown ----------------
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Merge split partials (log2-domain maxima): one CTA of 128 threads per (row, head).
+__global__ void attn_tc_merge_kernel(AttnArgs a) {
+    const int r = blockIdx.x, h = blockIdx.y;
+    const int hg = h / kHeads, hl = h % kHeads;
+    const float *base = a.partials + ((int64_t)r * a.hgroups + hg) * a.splits * kPartialFloats;
+    float M = -INFINITY;
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, base[s * kPartialFloats + hl]);
+    float L = 0.0f;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < a.splits; ++s) {
+        const float *p = base + s * kPartialFloats;
+        const float ls = p[kHeads + hl];
+        if (!(ls > 0.0f)) continue;
+        const float f = exp2f(p[hl] - M);
+        L += ls * f;
+        const float4 o = *reinterpret_cast<const float4 *>(p + 2 * kHeads + hl * kLatent + threadIdx.x * 4);
+        acc[0] += o.x * f; acc[1] += o.y * f; acc[2] += o.z * f; acc[3] += o.w * f;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    const int64_t oi = ((int64_t)r * a.H + h) * kLatent + threadIdx.x * 4;
+    if (a.out_dtype == CSA2_DTYPE_F32) {
+        *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + oi) =
+            make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    } else {
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.out) + oi;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = __float2bfloat16_rn(acc[i] * inv);
+    }
+    if (threadIdx.x == 0 && a.lse)
+        a.lse[(int64_t)r * a.H + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+static int g_num_sms = 0;
+
+static int num_sms() {
+    if (g_num_sms == 0) {
+        int dev = 0, n = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            g_num_sms = n;
+        else
+            g_num_sms = 148;
+    }
+    return g_num_sms;
+}
+
+// Split plan: enough CTAs to fill the SMs once (one CTA per SM), splitting on tile boundaries.
+void tc_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_split) {
+    hgroups = (H + tc::kHeads - 1) / tc::kHeads;
+    const int max_keys = K + CSA2_SWA_WINDOW;
+    const int tiles = (max_keys + tc::kTile - 1) / tc::kTile;
+    const int ctas = rows * hgroups;
+    int s = num_sms() / (ctas > 0 ? ctas : 1);
+    if (s < 1) s = 1;
+    if (s > tiles) s = tiles;
+    const int tiles_per = (tiles + s - 1) / s;
+    splits = (tiles + tiles_per - 1) / tiles_per;
+    keys_per_split = tiles_per * tc::kTile;
+}
+
+size_t tc_workspace_bytes(int rows, int H, int K) {
+    int hg, sp, kps;
+    tc_plan(rows, H, K, hg, sp, kps);
+    if (sp == 1) return 256;
+    return (size_t)rows * hg * sp * kPartialFloats * sizeof(float) + 256;
+}
+
+cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             tc::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    tc_plan(a.rows, a.H, a.K, a.hgroups, a.splits, a.keys_per_split);
+    dim3 grid(a.rows, a.hgroups, a.splits);
+    tc::attn_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a);
+    int n = 1;
+    if (a.splits > 1) {
+        tc::attn_tc_merge_kernel<<<dim3(a.rows, a.H), 128, 0, st>>>(a);
+        ++n;
+    }
+    note_launches(n);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -93,6 +93,9 @@ CSA2_HD uint32_t float_key(float f) {
 
 CSA2_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Device-side error word: a bounded wait that expires stores a csa2_status here.
+__device__ int g_device_error = 0;
+
 // Host-side count of kernel launches (csa2_launch_count); every launcher adds its launches.
 void note_launches(int n);
 

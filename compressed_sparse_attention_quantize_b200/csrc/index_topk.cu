@@ -311,8 +311,6 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
 // ---------------------------------------------------------------------------------------
 // device error word
 // ---------------------------------------------------------------------------------------
-__device__ int g_device_error = 0;
-
 csa2_status read_and_clear_device_error() {
     int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return CSA2_ERR_CUDA;

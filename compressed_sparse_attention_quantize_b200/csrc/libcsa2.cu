@@ -2,5 +2,6 @@
 #include "quant.cu"
 #include "index_topk.cu"
 #include "attn_simt.cu"
+#include "attn_tc.cu"
 #include "attn_dispatch.cu"
 #include "api.cu"
