@@ -107,6 +107,8 @@ def lib():
                                    _sz, _vp]
     L.csa2_device_error.restype = _i32
     L.csa2_device_error.argtypes = [_vp]
+    L.csa2_last_error_string.restype = ctypes.c_char_p
+    L.csa2_last_error_string.argtypes = []
     L.csa2_launch_count.restype = ctypes.c_uint64
     L.csa2_launch_count.argtypes = []
     _lib = L
@@ -137,7 +139,10 @@ def _stream(stream) -> Optional[int]:
 
 def _check(status: int) -> None:
     if status != 0:
-        raise CSA2Error(csa2_status_string(status))
+        msg = csa2_status_string(status)
+        if status == 5:
+            msg += " (" + lib().csa2_last_error_string().decode() + ")"
+        raise CSA2Error(msg)
 
 
 def csa2_status_string(status: int) -> str:

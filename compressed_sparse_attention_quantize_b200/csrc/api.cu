@@ -2,6 +2,8 @@
 //
 // Every call validates all arguments before it enqueues anything, launches only on the
 // caller's stream and never synchronises the host (csa2_device_error excepted).
+#include <cstdio>
+
 #include "common.cuh"
 #include "attn.cuh"
 
@@ -27,7 +29,12 @@ namespace {
 
 inline bool aligned16(const void *p) { return (((uintptr_t)p) & 15u) == 0; }
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
-inline csa2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+thread_local char t_last_error[256] = "";
+inline csa2_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return CSA2_OK;
+    snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return CSA2_ERR_CUDA;
+}
 constexpr size_t kAlign = 256;
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -103,6 +110,8 @@ const char *csa2_status_string(csa2_status s) {
 }
 
 int csa2_version(void) { return 1; }
+
+const char *csa2_last_error_string(void) { return t_last_error; }
 
 uint64_t csa2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -293,7 +302,7 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
         if (L.idx_out) {
             cudaError_t e = cudaMemcpyAsync(L.idx_out, idx, (size_t)rows * g->K * 4,
                                             cudaMemcpyDeviceToDevice, st);
-            if (e != cudaSuccess) return CSA2_ERR_CUDA;
+            if (e != cudaSuccess) return cuda_status(e);
         }
         s = csa2_sparse_attn(L.q, g->B, g->T, g->H, g->D, g->kv, g->kv_row_stride, g->seq_start, idx,
                              cnt, g->K, L.swa_codes, L.swa_scale, g->swa_cap, g->swa_start,

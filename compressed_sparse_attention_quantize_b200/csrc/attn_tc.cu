@@ -112,7 +112,7 @@ CSA2_D uint32_t sw128_off(int row, int c) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
 }
 
-__global__ void __maxnreg__(224)
+__global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -396,19 +396,19 @@ attn_tc_kernel(AttnArgs a) {
             }
             ptx::named_barrier(1, 128);
             const bool rescale = S.any_rescale != 0;
-            // probabilities (log2 domain); P^T line of key s as fp16 (window scale folded in)
-            uint32_t pw[kHeads / 2], plo[kHeads / 2];
+            // P.V of the previous tile completed before this tile's S (the tensor pipe runs in
+            // order), so this wait is immediate; it orders the O^T rescale and the P rewrite.
+            if (j > 0) {
+                ptx::mbar_wait(&S.pv_done, ph ^ 1, abort_flag);
+                ptx::named_barrier(1, 128);
+                if (*abort_flag) { aborted = true; break; }
+                ptx::tc_fence_after();
+            }
+            // probabilities (log2 domain)
 #pragma unroll
-            for (int h = 0; h < kHeads; h += 2) {
-                const float m0 = S.m_run[h], m1 = S.m_run[h + 1];
-                z[h] = (m0 == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[h] - m0);
-                z[h + 1] = (m1 == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[h + 1] - m1);
-                const float q0 = z[h] * src.scale, q1 = z[h + 1] * src.scale;
-                const __half2 hp = __floats2half2_rn(q0, q1);
-                const float2 back = __half22float2(hp);
-                const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
-                pw[h / 2] = *reinterpret_cast<const uint32_t *>(&hp);
-                plo[h / 2] = *reinterpret_cast<const uint32_t *>(&lp);
+            for (int h = 0; h < kHeads; ++h) {
+                const float m = S.m_run[h];
+                z[h] = (m == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[h] - m);
             }
             // this tile's row sums: lane L of warp `sub` owns heads L and 32+L
 #pragma unroll
@@ -420,32 +420,44 @@ attn_tc_kernel(AttnArgs a) {
                 const int h = half * 32 + lane;
                 S.lsum[sub][h] = S.lsum[sub][h] * S.alpha[h] + v[0];
             }
-            if (j > 0) {
-                ptx::mbar_wait(&S.pv_done, ph ^ 1, abort_flag);
-                ptx::named_barrier(1, 128);
-                if (*abort_flag) { aborted = true; break; }
-                ptx::tc_fence_after();
-                if (rescale) {
-                    for (int mb = 0; mb < 4; ++mb) {
+            // P^T line of key s: fp16 high half now (8 heads = one 16-byte chunk at a time);
+            // the low half P - fp16(P) stays in registers until the high half has been used
+            uint32_t plo[kHeads / 2];
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            uint32_t u[32];
-                            const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
-                            ptx::tmem_ld32(addr, u);
-                            ptx::tmem_ld_wait();
+            for (int c = 0; c < 8; ++c) {
+                uint32_t hi4[4];
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                u[i] = __float_as_uint(__uint_as_float(u[i]) * S.alpha[half * 32 + i]);
-                            ptx::tmem_st32(addr, u);
-                        }
-                    }
-                    ptx::tmem_st_wait();
+                for (int k = 0; k < 4; ++k) {
+                    const int h = 8 * c + 2 * k;
+                    const float q0 = z[h] * src.scale, q1 = z[h + 1] * src.scale;
+                    const __half2 hp = __floats2half2_rn(q0, q1);
+                    const float2 back = __half22float2(hp);
+                    const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
+                    hi4[k] = *reinterpret_cast<const uint32_t *>(&hp);
+                    plo[4 * c + k] = *reinterpret_cast<const uint32_t *>(&lp);
                 }
+                *reinterpret_cast<uint4 *>(sP + sw128_off(s, c)) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
             }
+            // O^T rescale for heads whose running max moved (only after the first tile)
+            if (rescale && j > 0) {
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float al[32];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(sP + sw128_off(s, c)) =
-                    make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                    for (int i = 0; i < 32; ++i) al[i] = S.alpha[half * 32 + i];
+#pragma unroll 1
+                    for (int mb = 0; mb < 4; ++mb) {
+                        uint32_t u[32];
+                        const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
+                        ptx::tmem_ld32(addr, u);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * al[i]);
+                        ptx::tmem_st32(addr, u);
+                    }
+                }
+                ptx::tmem_st_wait();
+            }
             ptx::fence_async_smem();
             ptx::tc_fence_before();
             ptx::named_barrier(1, 128);

@@ -242,6 +242,12 @@ CSA2_API csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer
 CSA2_API csa2_status csa2_device_error(void *stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa2_last_error_string -- description of the last CUDA runtime error a call of this
+ * library met on the calling host thread (the reason behind CSA2_ERR_CUDA), or "" if none.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API const char *csa2_last_error_string(void);
+
+/* ------------------------------------------------------------------------------------
  * csa2_launch_count -- number of kernels this library has launched in this process
  * (all devices, all streams) since it was loaded.  A diagnostic for benchmarks.
  * ---------------------------------------------------------------------------------- */
