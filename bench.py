@@ -372,6 +372,16 @@ def run_csa2(args, wl):
         dist.barrier()
     value = wl.B * wl.T * world * args.steps / (total_ms / 1e3)
 
+    if args.quick:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": total_ms / args.steps, "config": {"workload": wl.name},
+                              "gpu_launches": int(launches), "clocks": clocks, "quick": True}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
     # per-call breakdown and roofline of the dominant kernel
     bd = breakdown(torch, csa2, runner, max(3, min(args.steps, 10)), flush)
     ab, af = attn_work(wl, 4)
@@ -441,11 +451,17 @@ def main():
     ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="timed region only (no breakdown, e2e or CPU baseline): for profiler captures")
+    ap.add_argument("--entries", type=int, default=0,
+                    help="override compressed entries per sequence (smaller profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     from compressed_sparse_attention_quantize_b200 import synth
     wl = synth.workload(args.config)
+    if args.entries:
+        wl = synth.scaled(wl, n=args.entries, name=f"{wl.name}_n{args.entries}")
     if args.impl == "reference":
         run_reference(args, wl)
     else:
