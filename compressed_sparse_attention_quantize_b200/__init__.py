@@ -17,7 +17,7 @@ from typing import Optional, Sequence
 __all__ = [
     "CSA2Error", "lib", "library_path",
     "csa2_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
-    "csa2_sparse_attn", "csa2_sparse_attn_workspace_size",
+    "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
     "FMT_FP4", "FMT_FP8_TOKEN", "DTYPE_F32", "DTYPE_BF16", "MODE_FULL", "MODE_REINDEX",
@@ -99,6 +99,9 @@ def lib():
     L.csa2_sparse_attn.restype = _i32
     L.csa2_sparse_attn.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _i32,
                                    _vp, _vp, _i32, _vp, _vp, _f32, _vp, _i32, _vp, _vp, _sz, _vp]
+    L.csa2_sparse_attn_noalloc.restype = _i32
+    L.csa2_sparse_attn_noalloc.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _i32,
+                                           _vp, _vp, _i32, _vp, _vp, _f32, _vp, _i32, _vp, _vp]
     L.csa2_layer_group_workspace_size.restype = _i32
     L.csa2_layer_group_workspace_size.argtypes = [ctypes.POINTER(GroupDesc), ctypes.POINTER(LayerDesc),
                                                   _i32, ctypes.POINTER(_sz)]
@@ -190,6 +193,17 @@ def csa2_sparse_attn(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, cnt, K, s
                                   _ptr(idx), _ptr(cnt), K, _ptr(swa_codes), _ptr(swa_scale), swa_cap,
                                   _ptr(swa_start), _ptr(swa_len), float(softmax_scale), _ptr(out),
                                   out_dtype, _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def csa2_sparse_attn_noalloc(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, cnt, K, swa_codes,
+                             swa_scale, swa_cap, swa_start, swa_len, softmax_scale, out, out_dtype, lse,
+                             stream=None) -> None:
+    """csa2_sparse_attn without a workspace argument, for callers that cannot allocate device
+    memory: the scratch lives in a fixed array inside the library (see include/csa2.h)."""
+    _check(lib().csa2_sparse_attn_noalloc(_ptr(q), B, T, H, D, _ptr(kv), kv_row_stride, _ptr(seq_start),
+                                          _ptr(idx), _ptr(cnt), K, _ptr(swa_codes), _ptr(swa_scale),
+                                          swa_cap, _ptr(swa_start), _ptr(swa_len), float(softmax_scale),
+                                          _ptr(out), out_dtype, _ptr(lse), _stream(stream)))
 
 
 def _layers_array(layers: Sequence[LayerDesc]):

@@ -5,3 +5,4 @@
 #include "attn_tc.cu"
 #include "attn_dispatch.cu"
 #include "api.cu"
+#include "noalloc.cu"

@@ -190,6 +190,32 @@ CSA2_API csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, in
                              void *workspace, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa2_sparse_attn_noalloc -- csa2_sparse_attn for callers that cannot allocate device memory.
+ *
+ * No counterpart in the pages: this is an interface convenience, not part of the method.
+ * Same arguments, layouts, limits and result as csa2_sparse_attn, without `workspace`: the
+ * split partials go to a fixed 20 MiB scratch array inside the library (a static device
+ * array that every device loading the library holds until the process exits).  Callers that
+ * cannot call cudaMalloc -- an allocator that owns the whole device pool, a host process that
+ * forbids device allocations after start-up -- use this call instead.
+ *   - The first call on a device looks up the array's address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the array, and each call fully rewrites what it reads, so nothing needs
+ *     clearing; calls whose kernels overlap on the GPU (other streams or host threads) race.
+ *   - Returns CSA2_ERR_WORKSPACE when the launch needs more scratch than the array holds
+ *     (never on a GPU with <= 159 SMs: the split plan makes at most one partial per SM, each
+ *     131,584 bytes); otherwise the errors of csa2_sparse_attn.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t *q, int B, int T, int H, int D,
+                                              const uint8_t *kv, int64_t kv_row_stride,
+                                              const int64_t *seq_start, const int32_t *idx,
+                                              const int32_t *cnt, int K, const uint8_t *swa_codes,
+                                              const float *swa_scale, int swa_cap,
+                                              const int32_t *swa_start, const int32_t *swa_len,
+                                              float softmax_scale, void *out, int out_dtype,
+                                              float *lse, void *stream);
+
+/* ------------------------------------------------------------------------------------
  * csa2_layer_group -- one group of CSA2 layers in order ([B] section
  * "CSA2：三层压缩一次吃满"; [A] section "压缩吸收注意力（二代）": in a group of six only
  * the first is Full and the rest Reuse).
