@@ -22,9 +22,11 @@
 // per-token fp32 scale is applied to the logit and folded into P instead.  Q is converted to
 // fp16 with a power-of-two pre-scale so small values keep full precision.
 //
-// Warp roles (9 warps): 0 = TMEM owner + MMA issuer; 1-4 = softmax/epilogue (TMEM
-// subpartitions 1,2,3,0); 5-8 = dequantisers (one key per thread).  Hand-offs use mbarriers
-// per V region (64 channels) so dequantising tile j+1 overlaps the P.V products of tile j.
+// Warp roles (9 warps): 0 = TMEM owner + MMA issuer; 1-8 = workers.  Worker warp w owns TMEM
+// sub-partition w%4 (keys 32*(w%4)..+31) and one half: it dequantises channels 256*half..+255
+// of its keys and runs the softmax for heads 32*half..+31.  Hand-offs use mbarriers per V
+// region (64 channels) so dequantising tile j+1 overlaps the P.V products of tile j; the
+// per-head max is only re-reduced when some logit exceeds the running max by 2^8.
 // Every wait is bounded: on expiry the CTA records CSA2_ERR_TIMEOUT, drains, frees TMEM and exits.
 #include "attn.cuh"
 #include "tc_ptx.cuh"
@@ -41,8 +43,8 @@ constexpr int kVRegion = kTile * 128;      // 16 KB
 constexpr int kQBytes = kRegions * kQRegion;         // 64 KB
 constexpr int kVBytes = kRegions * kVRegion;         // 128 KB
 constexpr int kPBytes = kTile * kHeads * 2;          // 16 KB
-constexpr int kThreads = 288;
-constexpr int kSoftmaxWarp0 = 1, kDequantWarp0 = 5;
+constexpr int kThreads = 288;             // warp 0: MMA issuer; warps 1-8: workers
+constexpr int kWorkers = 256;
 constexpr int kTmemCols = 512;
 constexpr int kOCol = 256;                 // O^T accumulators at columns 256..511
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -112,6 +114,79 @@ CSA2_D uint32_t sw128_off(int row, int c) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
 }
 
+// Prefetched half-row of one key: main entries keep 128 code bytes + 16 scale bytes of the
+// four 64-channel regions of this thread's half; window keys are loaded per region.
+struct HalfRow {
+    uint4 codes[8];
+    uint4 scales;
+};
+
+CSA2_D void prefetch_half(const KeySrc &src, int half, HalfRow &hr) {
+    if (src.valid && !src.swa) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hr.codes[i] = __ldg(p + half * 8 + i);
+        hr.scales = __ldg(p + 16 + half);
+    } else {                                     // always assigned: no stale registers live
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hr.codes[i] = make_uint4(0u, 0u, 0u, 0u);
+        hr.scales = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// Dequantise region `rg` (64 channels) of one key into 8 fp16 chunks.
+CSA2_D void dequant_region(const KeySrc &src, const HalfRow &hr, int rl, int rg, uint4 (&out)[8]) {
+    if (!src.valid) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) out[c] = make_uint4(0u, 0u, 0u, 0u);
+    } else if (!src.swa) {
+        // rl = region index within the half: code bytes 32rl.., scale bytes 4rl..
+        const uint32_t sw = rl == 0 ? hr.scales.x : rl == 1 ? hr.scales.y : rl == 2 ? hr.scales.z : hr.scales.w;
+        const uint4 c0 = hr.codes[2 * rl], c1 = hr.codes[2 * rl + 1];
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t s01 = ptx::e4m3x2_to_f16x2((uint16_t)(sw & 0xFFFFu));
+        const uint32_t s23 = ptx::e4m3x2_to_f16x2((uint16_t)(sw >> 16));
+        const uint32_t sc[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                                __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
+#pragma unroll
+        for (int wi = 0; wi < 8; ++wi) {                 // word wi = channels 8wi..8wi+7
+            uint32_t hv[4];
+            ptx::e2m1x8_to_f16x8(words[wi], hv);
+            const uint32_t sv = sc[wi >> 1];
+            out[wi] = make_uint4(ptx::hmul2_u32(hv[0], sv), ptx::hmul2_u32(hv[1], sv),
+                                 ptx::hmul2_u32(hv[2], sv), ptx::hmul2_u32(hv[3], sv));
+        }
+    } else {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr + rg * 64);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(p + i);                  // 16 codes = channels 16i..16i+15
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t hv[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                hv[2 * k] = ptx::e4m3x2_to_f16x2((uint16_t)(w[k] & 0xFFFFu));
+                hv[2 * k + 1] = ptx::e4m3x2_to_f16x2((uint16_t)(w[k] >> 16));
+            }
+            out[2 * i] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            out[2 * i + 1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        }
+    }
+}
+
+CSA2_D bool block_any(bool flag, uint32_t barrier_id, uint32_t threads) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)flag), "r"(barrier_id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -137,14 +212,14 @@ attn_tc_kernel(AttnArgs a) {
     // ---------------- setup ----------------
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRegions; ++i) {
-            ptx::mbar_init(&S.v_full[i], 128);
+            ptx::mbar_init(&S.v_full[i], kWorkers / 2);
             ptx::mbar_init(&S.v_empty[i], 1);
         }
         ptx::mbar_init(&S.s_full, 1);
-        ptx::mbar_init(&S.s_empty, 128);
-        ptx::mbar_init(&S.p_full, 128);
+        ptx::mbar_init(&S.s_empty, kWorkers);
+        ptx::mbar_init(&S.p_full, kWorkers);
         ptx::mbar_init(&S.pv_hi_done, 1);
-        ptx::mbar_init(&S.p_lo_full, 128);
+        ptx::mbar_init(&S.p_lo_full, kWorkers);
         ptx::mbar_init(&S.pv_done, 1);
         ptx::mbar_init(&S.drain, 1);
         S.abort_flag = 0;
@@ -158,46 +233,56 @@ attn_tc_kernel(AttnArgs a) {
         ptx::tmem_alloc(&S.tmem_base, kTmemCols);
         ptx::tmem_relinquish();
     }
-    // Q: largest bf16 exponent of this head group -> power-of-two pre-scale for fp16
+    // Q: every thread loads its chunks once; the largest bf16 exponent of the head group picks a
+    // power-of-two pre-scale so the fp16 copy keeps full precision for small values.
     const uint16_t *qrow = a.q + (int64_t)r * a.H * kLatent;
     const int hcount = min(kHeads, a.H - h0);
+    constexpr int kQChunks = kHeads * (kLatent / 8);                 // 16-byte chunks
+    constexpr int kQPer = (kQChunks + kThreads - 1) / kThreads;
+    uint4 qreg[kQPer];
     {
         int emax = 0;
-        for (int i = threadIdx.x; i < hcount * (kLatent / 8); i += kThreads) {
-            const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
-            const uint4 v = *reinterpret_cast<const uint4 *>(qrow + (int64_t)(h0 + h) * kLatent + c8 * 8);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                emax = max(emax, (int)((w[k] >> 7) & 0xFFu));
-                emax = max(emax, (int)((w[k] >> 23) & 0xFFu));
+        for (int k = 0; k < kQPer; ++k) {
+            const int i = threadIdx.x + k * kThreads;
+            const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
+            qreg[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < kQChunks && h < hcount)
+                qreg[k] = *reinterpret_cast<const uint4 *>(qrow + (int64_t)(h0 + h) * kLatent + c8 * 8);
+        }
+#pragma unroll
+        for (int k = 0; k < kQPer; ++k) {
+            const uint32_t w[4] = {qreg[k].x, qreg[k].y, qreg[k].z, qreg[k].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                emax = max(emax, (int)((w[e] >> 7) & 0xFFu));
+                emax = max(emax, (int)((w[e] >> 23) & 0xFFu));
             }
         }
         emax = __reduce_max_sync(0xffffffffu, emax);
-        __syncthreads();
+        __syncthreads();                                   // barrier init visible
         if (lane == 0) atomicMax(&S.q_exp_max, emax);
     }
     __syncthreads();
-    // fp16 holds up to 2^15 comfortably: scale so the largest |q| lands in [2^13, 2^14)
+    // the largest |q| lands in [2^13, 2^14): far from fp16 overflow, far above its subnormals
     const int qshift = S.q_exp_max == 0 ? 0 : (13 - (S.q_exp_max - 127));
     const float qmul = exp2f((float)qshift);
-    for (int i = threadIdx.x; i < kHeads * (kLatent / 8); i += kThreads) {
-        const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
-        uint32_t packed[4] = {0u, 0u, 0u, 0u};
-        if (h < hcount) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(qrow + (int64_t)(h0 + h) * kLatent + c8 * 8);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float lo = __uint_as_float(w[k] << 16) * qmul;
-                const float hi = __uint_as_float(w[k] & 0xFFFF0000u) * qmul;
-                __half2 hh = __floats2half2_rn(lo, hi);
-                packed[k] = *reinterpret_cast<uint32_t *>(&hh);
+    for (int k = 0; k < kQPer; ++k) {
+        const int i = threadIdx.x + k * kThreads;
+        if (i < kQChunks) {
+            const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
+            const uint32_t w[4] = {qreg[k].x, qreg[k].y, qreg[k].z, qreg[k].w};
+            uint32_t packed[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __half2 hh = __floats2half2_rn(__uint_as_float(w[e] << 16) * qmul,
+                                                     __uint_as_float(w[e] & 0xFFFF0000u) * qmul);
+                packed[e] = *reinterpret_cast<const uint32_t *>(&hh);
             }
+            *reinterpret_cast<uint4 *>(sQ + (c8 >> 3) * kQRegion + sw128_off(h, c8 & 7)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
-        const int region = c8 >> 3, chunk = c8 & 7;
-        *reinterpret_cast<uint4 *>(sQ + region * kQRegion + sw128_off(h, chunk)) =
-            make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
     ptx::fence_async_smem();
     ptx::tc_fence_before();
@@ -219,7 +304,7 @@ attn_tc_kernel(AttnArgs a) {
                 if (*abort_flag) break;
             }
             bool ok = true;
-            for (int rg = 0; rg < kRegions && ok; ++rg) {
+            for (int rg = 0; rg < kRegions; ++rg) {
                 ptx::mbar_wait(&S.v_full[rg], ph, abort_flag);
                 __syncwarp();
                 if (*abort_flag) { ok = false; break; }
@@ -277,199 +362,154 @@ attn_tc_kernel(AttnArgs a) {
         if (lane == 0) ptx::mma_commit(&S.drain);
         __syncwarp();
         ptx::mbar_wait_drain(&S.drain, 0);
-    } else if (warp >= kDequantWarp0) {
-        // ================= dequantisers: thread t <-> key t of the tile =================
-        const int t = threadIdx.x - kDequantWarp0 * 32;
-        for (int j = 0; j < ntiles; ++j) {
+    } else {
+        // ================= workers: key t = sub*32 + lane; half = channel/head half =========
+        const int sub = warp & 3;
+        const int half = (warp - 1) >> 2;
+        const int t = sub * 32 + lane;
+        const int wt = threadIdx.x - 32;                 // 0..255
+        const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
+        const float qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-qshift);
+        bool aborted = false;
+        KeySrc src = key_source(a, r, b, x_begin + t, x_end, n_sel);
+        HalfRow hr;
+        prefetch_half(src, half, hr);
+        for (int j = 0; j < ntiles && !aborted; ++j) {
             const uint32_t ph = j & 1;
-            const KeySrc src = key_source(a, r, b, x_begin + j * kTile + t, x_end, n_sel);
-            uint4 codes[16], scl[2];
-            if (src.valid && !src.swa) {
-                const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
+            // ---- dequantise this thread's half of key t into V (regions 4*half .. 4*half+3)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) codes[i] = __ldg(p + i);
-                scl[0] = __ldg(p + 16);
-                scl[1] = __ldg(p + 17);
-            }
-            bool ok = true;
-#pragma unroll
-            for (int rg = 0; rg < kRegions; ++rg) {
+            for (int rl = 0; rl < 4; ++rl) {
+                const int rg = half * 4 + rl;
                 uint4 out[8];
-                if (!src.valid) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) out[c] = make_uint4(0u, 0u, 0u, 0u);
-                } else if (!src.swa) {
-                    const uint4 sq = rg < 4 ? scl[0] : scl[1];
-                    const uint32_t sw = (rg & 3) == 0 ? sq.x : (rg & 3) == 1 ? sq.y : (rg & 3) == 2 ? sq.z : sq.w;
-                    const uint4 c0 = codes[2 * rg], c1 = codes[2 * rg + 1];
-                    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    const uint32_t s01 = ptx::e4m3x2_to_f16x2((uint16_t)(sw & 0xFFFFu));
-                    const uint32_t s23 = ptx::e4m3x2_to_f16x2((uint16_t)(sw >> 16));
-                    const uint32_t sc[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
-                                            __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
-#pragma unroll
-                    for (int wi = 0; wi < 8; ++wi) {           // word wi = channels 8wi..8wi+7
-                        uint32_t hv[4];
-                        ptx::e2m1x8_to_f16x8(words[wi], hv);
-                        const uint32_t s = sc[wi >> 1];
-                        out[wi] = make_uint4(ptx::hmul2_u32(hv[0], s), ptx::hmul2_u32(hv[1], s),
-                                             ptx::hmul2_u32(hv[2], s), ptx::hmul2_u32(hv[3], s));
-                    }
-                } else {
-                    const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr + rg * 64);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 v = __ldg(p + i);          // 16 codes = channels 16i..16i+15
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                        uint32_t hv[8];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            hv[2 * k] = ptx::e4m3x2_to_f16x2((uint16_t)(w[k] & 0xFFFFu));
-                            hv[2 * k + 1] = ptx::e4m3x2_to_f16x2((uint16_t)(w[k] >> 16));
-                        }
-                        out[2 * i] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                        out[2 * i + 1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-                    }
-                }
-                if (j > 0) {
-                    if (!ptx::mbar_wait(&S.v_empty[rg], ph ^ 1, abort_flag)) { ok = false; break; }
-                }
+                dequant_region(src, hr, rl, rg, out);
+                if (j > 0 && !ptx::mbar_wait(&S.v_empty[rg], ph ^ 1, abort_flag)) { aborted = true; break; }
                 uint8_t *dst = sV + rg * kVRegion;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + sw128_off(t, c)) = out[c];
                 ptx::fence_async_smem();
                 ptx::mbar_arrive(&S.v_full[rg]);
             }
-            if (!ok) break;
-        }
-    } else {
-        // ================= softmax / epilogue: thread s <-> TMEM lane s (key s) =================
-        const int sub = warp & 3;
-        const int s = sub * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
-        const float qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-qshift);
-        bool aborted = false;
-        for (int j = 0; j < ntiles; ++j) {
-            const uint32_t ph = j & 1;
-            const KeySrc src = key_source(a, r, b, x_begin + j * kTile + s, x_end, n_sel);
+            // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             ptx::mbar_wait(&S.s_full, ph, abort_flag);
-            ptx::named_barrier(1, 128);
+            ptx::named_barrier(1, kWorkers);
             if (*abort_flag) { aborted = true; break; }
             ptx::tc_fence_after();
-            float z[kHeads];
+            float z[32];
             {
                 uint32_t u[32];
-                ptx::tmem_ld32(lane_addr + 0, u);
+                ptx::tmem_ld32(lane_addr + half * 32, u);
                 ptx::tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(u[i]);
-                ptx::tmem_ld32(lane_addr + 32, u);
-                ptx::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) z[32 + i] = __uint_as_float(u[i]);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&S.s_empty);
             const float zs = qk_scale * src.scale;
+            bool over = false;
 #pragma unroll
-            for (int h = 0; h < kHeads; ++h) z[h] = src.valid ? z[h] * zs : -INFINITY;
-            // per-head max over this warp's 32 keys, 32 heads at a time: lane L ends with head L
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int i = 0; i < 32; ++i) {
+                z[i] = src.valid ? z[i] * zs : -INFINITY;
+                over |= z[i] > S.m_run[half * 32 + i] + kRescaleThreshold;
+            }
+            // the running max moves only when some logit exceeds it by more than 2^8
+            const bool move = block_any(over, 1, kWorkers);
+            if (move) {
                 float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = z[half * 32 + i];
+                for (int i = 0; i < 32; ++i) v[i] = z[i];
                 warp_transpose_reduce<false>(v, lane);
                 S.red[sub][half * 32 + lane] = v[0];
-            }
-            ptx::named_barrier(1, 128);
-            if (s < kHeads) {
-                const float tmax = fmaxf(fmaxf(S.red[0][s], S.red[1][s]), fmaxf(S.red[2][s], S.red[3][s]));
-                const float mo = S.m_run[s];
-                float al = 1.0f;
-                if (tmax > mo + kRescaleThreshold || (mo == -INFINITY && tmax > -INFINITY)) {
-                    S.m_run[s] = tmax;
-                    al = (mo == -INFINITY) ? 0.0f : ptx::ex2(mo - tmax);
-                    if (j > 0 && mo != -INFINITY) S.any_rescale = 1;
+                ptx::named_barrier(1, kWorkers);
+                if (wt < kHeads) {
+                    const float tmax = fmaxf(fmaxf(S.red[0][wt], S.red[1][wt]), fmaxf(S.red[2][wt], S.red[3][wt]));
+                    const float mo = S.m_run[wt];
+                    float al = 1.0f;
+                    if (tmax > mo + kRescaleThreshold) {
+                        S.m_run[wt] = tmax;
+                        al = (mo == -INFINITY) ? 0.0f : ptx::ex2(mo - tmax);
+                        if (j > 0 && mo != -INFINITY) S.any_rescale = 1;
+                    }
+                    S.alpha[wt] = al;
                 }
-                S.alpha[s] = al;
+                ptx::named_barrier(1, kWorkers);
             }
-            ptx::named_barrier(1, 128);
-            const bool rescale = S.any_rescale != 0;
+            const bool rescale = move && S.any_rescale != 0;
+            // probabilities (log2 domain)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float m = S.m_run[half * 32 + i];
+                z[i] = (m == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[i] - m);
+            }
+            // this tile's row sums: lane L owns head 32*half + L of its 32 keys
+            {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = z[i];
+                warp_transpose_reduce<true>(v, lane);
+                const int h = half * 32 + lane;
+                const float al = move ? S.alpha[h] : 1.0f;
+                S.lsum[sub][h] = S.lsum[sub][h] * al + v[0];
+            }
             // P.V of the previous tile completed before this tile's S (the tensor pipe runs in
-            // order), so this wait is immediate; it orders the O^T rescale and the P rewrite.
+            // order), so this wait is immediate; it orders the P rewrite and the O^T rescale.
             if (j > 0) {
                 ptx::mbar_wait(&S.pv_done, ph ^ 1, abort_flag);
-                ptx::named_barrier(1, 128);
+                ptx::named_barrier(1, kWorkers);
                 if (*abort_flag) { aborted = true; break; }
                 ptx::tc_fence_after();
             }
-            // probabilities (log2 domain)
+            // P^T line of key t, heads of this half: fp16 high half now, low half kept
+            uint32_t plo[16];
 #pragma unroll
-            for (int h = 0; h < kHeads; ++h) {
-                const float m = S.m_run[h];
-                z[h] = (m == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[h] - m);
-            }
-            // this tile's row sums: lane L of warp `sub` owns heads L and 32+L
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = z[half * 32 + i];
-                warp_transpose_reduce<true>(v, lane);
-                const int h = half * 32 + lane;
-                S.lsum[sub][h] = S.lsum[sub][h] * S.alpha[h] + v[0];
-            }
-            // P^T line of key s: fp16 high half now (8 heads = one 16-byte chunk at a time);
-            // the low half P - fp16(P) stays in registers until the high half has been used
-            uint32_t plo[kHeads / 2];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint32_t hi4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int h = 8 * c + 2 * k;
-                    const float q0 = z[h] * src.scale, q1 = z[h + 1] * src.scale;
+                    const int i = 8 * c + 2 * k;
+                    const float q0 = z[i] * src.scale, q1 = z[i + 1] * src.scale;
                     const __half2 hp = __floats2half2_rn(q0, q1);
                     const float2 back = __half22float2(hp);
                     const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
                     hi4[k] = *reinterpret_cast<const uint32_t *>(&hp);
                     plo[4 * c + k] = *reinterpret_cast<const uint32_t *>(&lp);
                 }
-                *reinterpret_cast<uint4 *>(sP + sw128_off(s, c)) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) =
+                    make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
             }
-            // O^T rescale for heads whose running max moved (only after the first tile)
+            // O^T rescale for heads whose running max moved (columns of this half)
             if (rescale && j > 0) {
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float al[32];
+                float al[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) al[i] = S.alpha[half * 32 + i];
+                for (int i = 0; i < 32; ++i) al[i] = S.alpha[half * 32 + i];
 #pragma unroll 1
-                    for (int mb = 0; mb < 4; ++mb) {
-                        uint32_t u[32];
-                        const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
-                        ptx::tmem_ld32(addr, u);
-                        ptx::tmem_ld_wait();
+                for (int mb = 0; mb < 4; ++mb) {
+                    uint32_t u[32];
+                    const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
+                    ptx::tmem_ld32(addr, u);
+                    ptx::tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * al[i]);
-                        ptx::tmem_st32(addr, u);
-                    }
+                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * al[i]);
+                    ptx::tmem_st32(addr, u);
                 }
                 ptx::tmem_st_wait();
             }
             ptx::fence_async_smem();
             ptx::tc_fence_before();
-            ptx::named_barrier(1, 128);
-            if (s == 0) S.any_rescale = 0;
+            ptx::named_barrier(1, kWorkers);
+            if (wt == 0) S.any_rescale = 0;
             ptx::mbar_arrive(&S.p_full);
+            // next tile's rows are fetched while the tensor core runs P.V
+            if (j + 1 < ntiles) {
+                src = key_source(a, r, b, x_begin + (j + 1) * kTile + t, x_end, n_sel);
+                prefetch_half(src, half, hr);
+            }
             // once the high halves have been consumed, the same buffer takes the low halves
             ptx::mbar_wait(&S.pv_hi_done, ph, abort_flag);
-            ptx::named_barrier(1, 128);
+            ptx::named_barrier(1, kWorkers);
             if (*abort_flag) { aborted = true; break; }
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(sP + sw128_off(s, c)) =
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) =
                     make_uint4(plo[4 * c], plo[4 * c + 1], plo[4 * c + 2], plo[4 * c + 3]);
             ptx::fence_async_smem();
             ptx::mbar_arrive(&S.p_lo_full);
@@ -477,54 +517,51 @@ attn_tc_kernel(AttnArgs a) {
         // ---------------- epilogue ----------------
         if (!aborted && ntiles > 0) {
             ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag);
-            ptx::named_barrier(1, 128);
-            aborted = *abort_flag != 0;
-            ptx::tc_fence_after();
         }
+        ptx::named_barrier(1, kWorkers);
+        aborted = aborted || *abort_flag != 0;
+        ptx::tc_fence_after();
         if (!aborted) {
             const bool single = a.splits == 1;
             const int64_t part_idx = ((int64_t)r * a.hgroups + hg) * a.splits + split;
             float *part = a.partials + part_idx * kPartialFloats;
-            if (s < kHeads) {
-                const float l = ntiles > 0 ? S.lsum[0][s] + S.lsum[1][s] + S.lsum[2][s] + S.lsum[3][s] : 0.0f;
-                S.red[0][s] = l;
+            if (wt < kHeads) {
+                const float l = ntiles > 0 ? S.lsum[0][wt] + S.lsum[1][wt] + S.lsum[2][wt] + S.lsum[3][wt] : 0.0f;
+                S.red[0][wt] = l > 0.0f ? 1.0f / l : 0.0f;       // 1/l for the single-split output
                 if (!single) {
-                    part[s] = ntiles > 0 ? S.m_run[s] : -INFINITY;
-                    part[kHeads + s] = l;
-                } else if (a.lse && h0 + s < a.H) {
-                    a.lse[(int64_t)r * a.H + h0 + s] =
-                        (l > 0.0f) ? (S.m_run[s] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                    part[wt] = ntiles > 0 ? S.m_run[wt] : -INFINITY;
+                    part[kHeads + wt] = l;
+                } else if (a.lse && h0 + wt < a.H) {
+                    a.lse[(int64_t)r * a.H + h0 + wt] =
+                        (l > 0.0f) ? (S.m_run[wt] + log2f(l)) * 0.6931471805599453f : -INFINITY;
                 }
             }
-            ptx::named_barrier(1, 128);
+            ptx::named_barrier(1, kWorkers);
+#pragma unroll 1
             for (int mb = 0; mb < 4; ++mb) {
-                const int c = mb * 128 + s;             // this thread's channel
+                const int c = mb * 128 + t;               // this thread's channel
+                uint32_t u[32];
+                if (ntiles > 0) {
+                    ptx::tmem_ld32(lane_addr + kOCol + mb * kHeads + half * 32, u);
+                    ptx::tmem_ld_wait();
+                } else {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t u[32];
-                    if (ntiles > 0) {
-                        ptx::tmem_ld32(lane_addr + kOCol + mb * kHeads + half * 32, u);
-                        ptx::tmem_ld_wait();
+                    for (int i = 0; i < 32; ++i) u[i] = 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int h = half * 32 + i;
+                    if (h0 + h >= a.H) continue;
+                    const float o = __uint_as_float(u[i]);
+                    if (!single) {
+                        part[2 * kHeads + h * kLatent + c] = o;
                     } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) u[i] = 0u;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int h = half * 32 + i;
-                        if (h0 + h >= a.H) continue;
-                        const float o = __uint_as_float(u[i]);
-                        if (!single) {
-                            part[2 * kHeads + h * kLatent + c] = o;
-                        } else {
-                            const float l = S.red[0][h];
-                            const float val = l > 0.0f ? o / l : 0.0f;
-                            const int64_t oi = ((int64_t)r * a.H + h0 + h) * kLatent + c;
-                            if (a.out_dtype == CSA2_DTYPE_F32)
-                                reinterpret_cast<float *>(a.out)[oi] = val;
-                            else
-                                reinterpret_cast<__nv_bfloat16 *>(a.out)[oi] = __float2bfloat16_rn(val);
-                        }
+                        const float val = o * S.red[0][h];
+                        const int64_t oi = ((int64_t)r * a.H + h0 + h) * kLatent + c;
+                        if (a.out_dtype == CSA2_DTYPE_F32)
+                            reinterpret_cast<float *>(a.out)[oi] = val;
+                        else
+                            reinterpret_cast<__nv_bfloat16 *>(a.out)[oi] = __float2bfloat16_rn(val);
                     }
                 }
             }
