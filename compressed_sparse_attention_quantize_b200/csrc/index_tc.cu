@@ -1,0 +1,280 @@
+// Indexer scores on the tensor cores (tcgen05.mma kind::mxf4), exact in fp32.
+//
+// [B] page "DeepSeek V4.1 Flash 如何靠压缩 KV 缓存实现小模型干翻大模型": section "为什么 KV 缓存成了
+// 新瓶颈？" (DSA-style indexer), "CSA2：三层压缩一次吃满" (Full / Reindex), "FP4 量化 + Bounded
+// Replay" (indexer Q and K in FP4).
+//
+// I[r, j] = sum_h w_h * relu(q_h . k_j).  The MMA computes, for 128 keys at a time, the raw E2M1
+// products of every (head, 16-channel block) pair: B holds the query "block-diagonally" --
+// column (h, b) carries head h's codes for block b and zeros elsewhere -- and every block scale
+// fed to the MMA is 1.0, so each output is a sum of 16 exact products (multiples of 1/4, at most
+// 576): exact in fp32.  The epilogue multiplies by the two E4M3 scales (exact) and adds blocks
+// and heads in the fixed order of the reference (explicitly rounded adds and multiplies), so
+// the scores -- and therefore the selected sets -- are bit-identical to it.
+//
+// Operands in shared memory, K-major without swizzle: a 32-byte row of FP4 codes is two 16-byte
+// planes (elements 0-31 and 32-63), rows 16 bytes apart inside a plane.  D: 128 lanes (keys) x
+// N columns (4 per head, N rounded up to 16) fp32 in TMEM.  Each thread keeps the key rows of
+// the next 4 tiles in flight in registers; a CTA uses 128 TMEM columns and 56 KB of shared
+// memory so at most 4 CTAs share an SM and TMEM allocation never waits.
+#include "common.cuh"
+#include "index_api.cuh"
+#include "tc_ptx.cuh"
+
+namespace csa2 {
+namespace itc {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 128;
+constexpr int kMaxN = 4 * CSA2_MAX_INDEX_HEADS;      // 64 columns
+constexpr int kTmemCols = 128;                       // D at 0..63, scale factors at 64..127
+constexpr int kSfCol = 64;
+constexpr int kTilesPerCta = 32;                     // 4096 keys per CTA
+constexpr int kDepth = 4;                            // tiles of key rows in flight per thread
+constexpr int kOccupancySmem = 56 * 1024;            // dynamic smem that caps residency at 4/SM
+
+struct Args {
+    const uint8_t *q_codes, *q_scales;
+    const float *w;
+    int H, T;
+    const uint8_t *k_codes;
+    int64_t k_code_stride;
+    const uint8_t *k_scales;
+    int64_t k_scale_stride;
+    const int64_t *seq_start;
+    const int32_t *n_entries;
+    const int32_t *q_pos;
+    const int32_t *pool;
+    const int32_t *pool_len;
+    int P_in;
+    int row0;
+    float *scores;
+    int64_t score_stride;
+};
+
+struct __align__(16) Smem {
+    uint8_t a[2 * kTile * 16];         // keys: two 16-byte planes
+    uint8_t b[2 * kMaxN * 16];         // block-diagonal query
+    float qs[CSA2_MAX_INDEX_HEADS * 4];// query block scales
+    float w[CSA2_MAX_INDEX_HEADS];
+    uint64_t done, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+CSA2_D int64_t candidates(const Args &a, int r) {
+    if (a.pool) return a.pool_len[r];
+    const int b = r / a.T;
+    int64_t n = a.n_entries[b];
+    if (a.q_pos) {
+        const int64_t v = ((int64_t)a.q_pos[r] + 1) / 4;
+        n = v < n ? v : n;
+        if (n < 0) n = 0;
+    }
+    return n;
+}
+
+// Instruction descriptor, kind::mxf4 (block 32, UE8M0 scales): A, B = E2M1, K-major.
+CSA2_HD constexpr uint32_t idesc_mxf4(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+}
+
+CSA2_D uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;                          // version; layout type 0 = no swizzle
+    return d;
+}
+
+CSA2_D void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                     uint32_t sfb) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, 0, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads)
+index_score_tc_kernel(Args a) {
+    __shared__ Smem S;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int r = a.row0 + blockIdx.y;
+    const int b = r / a.T;
+    const int64_t n = min(candidates(a, r), a.score_stride);
+    const int64_t j0 = (int64_t)blockIdx.x * kTilesPerCta * kTile;
+    if (j0 >= n) return;                                  // uniform per CTA: nothing allocated yet
+    const int ntiles = (int)min((int64_t)kTilesPerCta, (n - j0 + kTile - 1) / kTile);
+    const int H = a.H;
+    const int N = ((4 * H + 15) / 16) * 16;
+
+    // ---- setup: query (block-diagonal B), scales, weights, barriers, TMEM ----
+    for (int i = t; i < (int)(sizeof(S.b) / 16); i += kThreads)
+        reinterpret_cast<uint4 *>(S.b)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (t == 0) {
+        ptx::mbar_init(&S.done, 1);
+        ptx::mbar_init(&S.drain, 1);
+        S.abort_flag = 0;
+        ptx::fence_async_smem();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&S.tmem_base, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    __syncthreads();
+    for (int i = t; i < H * 4; i += kThreads) {
+        const int h = i >> 2, blk = i & 3;
+        const uint8_t *qc = a.q_codes + ((int64_t)r * H + h) * 32;
+        // column n = 4h + blk: block blk's 8 code bytes at byte offset 8*blk of the 32-byte row
+        const int plane = blk >> 1, within = (blk & 1) * 8;
+        uint8_t *dst = S.b + plane * (kMaxN * 16) + i * 16 + within;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dst[k] = qc[8 * blk + k];
+        S.qs[i] = e4m3_to_f32(a.q_scales[((int64_t)r * H + h) * 4 + blk]);
+    }
+    for (int i = t; i < H; i += kThreads) S.w[i] = a.w[(int64_t)r * H + i];
+    ptx::fence_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    // every block scale the MMA sees is 1.0 (UE8M0 0x7F): the true E4M3 scales are applied below
+    {
+        uint32_t ones[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ones[i] = 0x7F7F7F7Fu;
+        ptx::tmem_st32(lane_addr + kSfCol, ones);
+        ptx::tmem_st32(lane_addr + kSfCol + 32, ones);
+        ptx::tmem_st_wait();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+
+    const uint32_t idesc = idesc_mxf4(128, N);
+    const uint32_t b_addr = ptx::smem_u32(S.b);
+    const uint64_t bdesc = sdesc_noswizzle(b_addr, kMaxN * 16, 128);
+    const uint32_t sf = tmem + kSfCol;
+    volatile int *abort_flag = &S.abort_flag;
+    const int64_t sbase = a.seq_start[b];
+
+    // key rows of tile i for this thread
+    auto key_row = [&](int i, uint4 &c0, uint4 &c1, uint32_t &sc, bool &valid) {
+        const int64_t j = j0 + (int64_t)i * kTile + t;
+        valid = j < n;
+        c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
+        sc = 0u;
+        if (valid) {
+            const int64_t e = sbase + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
+            const uint4 *kc = reinterpret_cast<const uint4 *>(a.k_codes + e * a.k_code_stride);
+            c0 = __ldg(kc);
+            c1 = __ldg(kc + 1);
+            const uint8_t *ks = a.k_scales + e * a.k_scale_stride;
+            sc = (uint32_t)__ldg(ks) | ((uint32_t)__ldg(ks + 1) << 8) | ((uint32_t)__ldg(ks + 2) << 16) |
+                 ((uint32_t)__ldg(ks + 3) << 24);
+        }
+    };
+
+    uint4 c0[kDepth], c1[kDepth];
+    uint32_t sc[kDepth];
+    bool valid[kDepth];
+#pragma unroll
+    for (int k = 0; k < kDepth; ++k) key_row(k, c0[k], c1[k], sc[k], valid[k]);
+    const uint64_t adesc = sdesc_noswizzle(ptx::smem_u32(S.a), kTile * 16, 128);
+    bool aborted = false;
+    for (int i0 = 0; i0 < ntiles && !aborted; i0 += kDepth) {
+#pragma unroll
+        for (int k = 0; k < kDepth; ++k) {
+            const int i = i0 + k;
+            if (i >= ntiles) break;
+            // stage tile i: the previous MMA has completed and every thread has read its D
+            *reinterpret_cast<uint4 *>(S.a + t * 16) = c0[k];
+            *reinterpret_cast<uint4 *>(S.a + kTile * 16 + t * 16) = c1[k];
+            ptx::fence_async_smem();
+            ptx::tc_fence_before();
+            __syncthreads();
+            if (t == 0) {
+                ptx::tc_fence_after();
+                mma_mxf4(tmem, adesc, bdesc, idesc, sf, sf);
+                ptx::mma_commit(&S.done);
+            }
+            const uint32_t sc_this = sc[k];
+            const bool valid_this = valid[k];
+            if (i + kDepth < ntiles) key_row(i + kDepth, c0[k], c1[k], sc[k], valid[k]);
+            // epilogue of tile i
+            ptx::mbar_wait(&S.done, i & 1, abort_flag);
+            if (__syncthreads_or(*abort_flag != 0)) { aborted = true; break; }
+            ptx::tc_fence_after();
+            float sk[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
+            float acc = 0.0f;
+            for (int hb = 0; hb * 8 < H; ++hb) {
+                uint32_t u[32];
+                ptx::tmem_ld32(lane_addr + hb * 32, u);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int hh = 0; hh < 8; ++hh) {
+                    const int h = hb * 8 + hh;
+                    if (h < H) {
+                        float p[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[h * 4 + q], sk[q]));
+                        const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
+                        const float rl = dot > 0.0f ? dot : 0.0f;
+                        acc = __fadd_rn(acc, __fmul_rn(S.w[h], rl));
+                    }
+                }
+            }
+            if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
+            if (valid_this) a.scores[(int64_t)blockIdx.y * a.score_stride + j0 + (int64_t)i * kTile + t] = acc;
+        }
+    }
+    if (aborted && t == 0) {           // drain the tensor pipe before TMEM is released
+        ptx::mma_commit(&S.drain);
+        ptx::mbar_wait_drain(&S.drain, 0);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace itc
+
+cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, float *scores,
+                                  int64_t score_stride, cudaStream_t st) {
+    itc::Args a;
+    a.q_codes = L.q_codes; a.q_scales = L.q_scales; a.w = L.w;
+    a.H = L.H; a.T = L.T;
+    a.k_codes = L.k_codes; a.k_code_stride = L.k_code_stride;
+    a.k_scales = L.k_scales; a.k_scale_stride = L.k_scale_stride;
+    a.seq_start = L.seq_start; a.n_entries = L.n_entries; a.q_pos = L.q_pos;
+    const bool reindex = L.mode == CSA2_MODE_REINDEX;
+    a.pool = reindex ? L.pool : nullptr;
+    a.pool_len = reindex ? L.pool_len : nullptr;
+    a.P_in = L.P_in;
+    a.row0 = row0;
+    a.scores = scores;
+    a.score_stride = score_stride;
+    const int64_t per_cta = (int64_t)itc::kTilesPerCta * itc::kTile;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(itc::index_score_tc_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, itc::kOccupancySmem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid((unsigned)ceil_div(score_stride, per_cta), (unsigned)nrows);
+    itc::index_score_tc_kernel<<<grid, itc::kThreads, itc::kOccupancySmem, st>>>(a);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -264,6 +264,9 @@ size_t index_topk_workspace_bytes(int rows, int64_t n, int K) {
     return (size_t)(chunk * (n > 0 ? n : 1) * 4 + 256);
 }
 
+cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, float *scores,
+                                  int64_t score_stride, cudaStream_t st);
+
 cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
     ScoreArgs base;
     base.q_codes = L.q_codes; base.q_scales = L.q_scales; base.w = L.w;
@@ -286,9 +289,8 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
         sa.scores = scores;
         sa.score_stride = max_n > 0 ? max_n : 1;
         if (max_n > 0) {
-            dim3 grid((unsigned)ceil_div(max_n, kScoreThreads), (unsigned)nr);
-            index_score_kernel<<<grid, kScoreThreads, 0, st>>>(sa);
-            note_launches(1);
+            cudaError_t e = launch_index_score_tc(L, (int)r0, nr, scores, sa.score_stride, st);
+            if (e != cudaSuccess) return e;
         }
         SelectArgs se;
         se.scores = scores;

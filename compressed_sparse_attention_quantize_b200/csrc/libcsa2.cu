@@ -1,6 +1,7 @@
 // Single translation unit of the CSA2 library (keeps device symbols in one module).
 #include "quant.cu"
 #include "index_topk.cu"
+#include "index_tc.cu"
 #include "attn_simt.cu"
 #include "attn_tc.cu"
 #include "attn_dispatch.cu"
