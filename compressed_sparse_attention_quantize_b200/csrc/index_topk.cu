@@ -267,6 +267,13 @@ size_t index_topk_workspace_bytes(int rows, int64_t n, int K) {
 cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, float *scores,
                                   int64_t score_stride, cudaStream_t st);
 
+int64_t topk_cluster_max_n();
+cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const int32_t *cand,
+                                int cand_stride, const int32_t *n_entries, const int32_t *q_pos,
+                                const int32_t *pool_len, int T, int row0, int nrows, int K,
+                                int32_t *out_idx, int32_t *out_cnt, int P, int32_t *out_pool,
+                                int32_t *out_pool_len, int64_t max_n, cudaStream_t st);
+
 cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
     ScoreArgs base;
     base.q_codes = L.q_codes; base.q_scales = L.q_scales; base.w = L.w;
@@ -291,6 +298,14 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
         if (max_n > 0) {
             cudaError_t e = launch_index_score_tc(L, (int)r0, nr, scores, sa.score_stride, st);
             if (e != cudaSuccess) return e;
+        }
+        if (max_n <= topk_cluster_max_n()) {
+            cudaError_t e = launch_topk_cluster(scores, sa.score_stride, sa.pool, sa.P_in, sa.n_entries,
+                                                sa.q_pos, sa.pool_len, sa.T, sa.row0, nr, L.K, L.out_idx,
+                                                L.out_cnt, reindex ? 0 : L.P, L.out_pool, L.out_pool_len,
+                                                max_n, st);
+            if (e != cudaSuccess) return e;
+            continue;
         }
         SelectArgs se;
         se.scores = scores;

@@ -1,0 +1,261 @@
+// Top-K (and pool) selection by a cluster of 8 CTAs per query row.
+//
+// [A] page "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径", section
+// "压缩吸收注意力（二代）": the indexer keeps 2048 blocks per query and the first layer's
+// candidate pool; order = score descending, entry index ascending on ties; output ascending.
+//
+// Each CTA of the cluster owns a contiguous chunk of the row's candidates and keeps their
+// order-preserving 32-bit keys in shared memory (read from global once).  Four 8-bit radix
+// passes find the exact threshold key: every CTA builds a 256-bin histogram of its chunk,
+// the cluster barrier publishes them, and every CTA sums the 8 histograms through distributed
+// shared memory (identical totals -> identical decisions, no broadcast needed).  Compaction:
+// each CTA publishes how many of its keys are above / equal to the threshold; the CTA's output
+// offset and its share of the "equal" keys (lowest indices first) follow from the lower-ranked
+// CTAs' counts; inside the CTA a block scan writes the selected ids in ascending order.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace csa2 {
+namespace tkc {
+
+namespace cg = cooperative_groups;
+
+constexpr int kCluster = 8;
+constexpr int kThreads = 1024;
+constexpr int kMaxChunk = 32768;                   // keys per CTA (128 KB of shared memory)
+
+struct Args {
+    const float *scores;        // [rows][score_stride]
+    int64_t score_stride;
+    const int32_t *cand;        // NULL: row r has cand_len(r) candidates 0..n-1
+    int cand_stride;            //  else [rows][cand_stride] entry ids (the Reindex pool)
+    const int32_t *n_entries;   // (NULL cand) visible count per row via the helpers below
+    const int32_t *q_pos;
+    const int32_t *pool_len;    // (cand) candidates per row
+    int T;
+    int row0;
+    int K;
+    int32_t *out_idx;
+    int32_t *out_cnt;
+    int P;
+    int32_t *out_pool;
+    int32_t *out_pool_len;
+};
+
+CSA2_D int64_t row_n(const Args &a, int r) {
+    if (a.cand) return a.pool_len[r];
+    const int b = r / a.T;
+    int64_t n = a.n_entries[b];
+    if (a.q_pos) {
+        const int64_t v = ((int64_t)a.q_pos[r] + 1) / 4;
+        n = v < n ? v : n;
+        if (n < 0) n = 0;
+    }
+    return n;
+}
+
+struct Shared {
+    unsigned int hist[2][256];
+    int counts[2];              // [0] above threshold, [1] equal to it
+    int warp_sums[33];
+    uint32_t prefix, mask;
+    int remaining;
+};
+
+// Block-wide exclusive count of a flag in thread order (kThreads threads).
+CSA2_D int block_excl(bool f, int *ws, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) ws[warp] = __popc(bal);
+    __syncthreads();
+    if (warp == 0) {
+        const int v = ws[lane];
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += x;
+        }
+        ws[lane] = incl - v;
+        if (lane == 31) ws[32] = incl;
+    }
+    __syncthreads();
+    const int res = ws[warp] + __popc(bal & ((1u << lane) - 1u));
+    total = ws[32];
+    __syncthreads();
+    return res;
+}
+
+// One selection of the k largest keys of the row (k < n): writes ids ascending to out[0..k).
+CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *keys, int chunk_len,
+                           int64_t chunk_base, const int32_t *ids, int k, int32_t *out) {
+    const int rank = (int)cl.block_rank();
+    if (threadIdx.x == 0) { S.prefix = 0u; S.mask = 0u; S.remaining = k; }
+    __syncthreads();
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        unsigned int *h = S.hist[pass & 1];
+        for (int i = threadIdx.x; i < 256; i += kThreads) h[i] = 0u;
+        __syncthreads();
+        const uint32_t prefix = S.prefix, mask = S.mask;
+        for (int i = threadIdx.x; i < chunk_len; i += kThreads) {
+            const uint32_t key = keys[i];
+            if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+        }
+        cl.sync();                                  // every CTA's histogram is complete
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            unsigned int bins[8];
+            unsigned int local = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                unsigned int v = 0;
+#pragma unroll
+                for (int c = 0; c < kCluster; ++c) v += cl.map_shared_rank(h, c)[lane * 8 + i];
+                bins[i] = v;
+                local += v;
+            }
+            unsigned int suffix = local;            // sum over lanes >= lane
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned int x = __shfl_down_sync(0xffffffffu, suffix, o);
+                if (lane + o < 32) suffix += x;
+            }
+            const int rem = S.remaining;
+            const unsigned int above = suffix - local;
+            const bool crosses = (int)above < rem && rem <= (int)suffix;
+            const unsigned bal = __ballot_sync(0xffffffffu, crosses);
+            const int owner = __ffs(bal) - 1;
+            if (lane == owner) {
+                int acc = (int)above;
+                int d = 7;
+                for (; d > 0; --d) {
+                    if (acc + (int)bins[d] >= rem) break;
+                    acc += (int)bins[d];
+                }
+                S.remaining = rem - acc;
+                S.prefix = prefix | ((uint32_t)(lane * 8 + d) << shift);
+                S.mask = mask | (255u << shift);
+            }
+        }
+        __syncthreads();
+        // histograms are double-buffered: the next pass writes the other buffer, and the pass
+        // after that is separated from these remote reads by the next pass's cluster barrier
+    }
+    const uint32_t thr = S.prefix;
+    const int need_eq = S.remaining;
+    // counts of this chunk
+    int gt = 0, eq = 0;
+    for (int i = threadIdx.x; i < chunk_len; i += kThreads) {
+        const uint32_t key = keys[i];
+        gt += key > thr;
+        eq += key == thr;
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    if (threadIdx.x == 0) { S.counts[0] = 0; S.counts[1] = 0; }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) { atomicAdd(&S.counts[0], gt); atomicAdd(&S.counts[1], eq); }
+    cl.sync();
+    int out_base = 0, eq_before = 0;
+    for (int c = 0; c < rank; ++c) {
+        const int *rc = cl.map_shared_rank(S.counts, c);
+        const int g = rc[0], e = rc[1];
+        const int take = min(e, max(0, need_eq - eq_before));
+        out_base += g + take;
+        eq_before += e;
+    }
+    // ordered compaction of this chunk
+    int run_out = 0, run_eq = 0;
+    for (int base = 0; base < chunk_len; base += kThreads) {
+        const int i = base + threadIdx.x;
+        uint32_t key = 0u;
+        if (i < chunk_len) key = keys[i];
+        const bool g = i < chunk_len && key > thr;
+        const bool e = i < chunk_len && key == thr;
+        int eq_tot;
+        const int er = block_excl(e, S.warp_sums, eq_tot);
+        const bool sel = g || (e && eq_before + run_eq + er < need_eq);
+        int sel_tot;
+        const int pos = block_excl(sel, S.warp_sums, sel_tot);
+        if (sel) {
+            const int64_t j = chunk_base + i;
+            out[out_base + run_out + pos] = ids ? ids[j] : (int32_t)j;
+        }
+        run_out += sel_tot;
+        run_eq += eq_tot;
+    }
+    cl.sync();                                      // counts may be reused by the next selection
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+topk_cluster_kernel(Args a) {
+    extern __shared__ __align__(16) uint32_t keys[];
+    __shared__ Shared S;
+    cg::cluster_group cl = cg::this_cluster();
+    const int rank = (int)cl.block_rank();
+    const int lr = blockIdx.x / kCluster;
+    const int r = a.row0 + lr;
+    int64_t n = row_n(a, r);
+    if (n > a.score_stride) n = a.score_stride;
+    const int chunk = (int)((n + kCluster - 1) / kCluster);
+    const int64_t cbase = (int64_t)rank * chunk;
+    const int clen = (int)max((int64_t)0, min((int64_t)chunk, n - cbase));
+    const float *s = a.scores + (int64_t)lr * a.score_stride;
+    const int32_t *ids = a.cand ? a.cand + (int64_t)r * a.cand_stride : nullptr;
+    for (int i = threadIdx.x; i < clen; i += kThreads) keys[i] = float_key(s[cbase + i]);
+    __syncthreads();
+    for (int which = 0; which < 2; ++which) {
+        const int k = which == 0 ? a.K : a.P;
+        if (k <= 0) continue;                       // uniform across the cluster
+        int32_t *out = which == 0 ? a.out_idx + (int64_t)r * a.K : a.out_pool + (int64_t)r * a.P;
+        int32_t *cnt = which == 0 ? a.out_cnt : a.out_pool_len;
+        const int c = (int)min((int64_t)k, n);
+        if (n <= k) {
+            for (int i = threadIdx.x; i < clen; i += kThreads) {
+                const int64_t j = cbase + i;
+                out[j] = ids ? ids[j] : (int32_t)j;
+            }
+        } else {
+            select_cluster(cl, S, keys, clen, cbase, ids, k, out);
+        }
+        // padding: rank 0 writes -1 to out[c..k)
+        if (rank == 0) {
+            for (int i = c + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+            if (threadIdx.x == 0 && cnt) cnt[r] = c;
+        }
+    }
+}
+
+}  // namespace tkc
+
+int64_t topk_cluster_max_n() { return (int64_t)tkc::kCluster * tkc::kMaxChunk; }
+
+// Selection for rows [row0, row0+nrows) from scores in global memory (max_n <= topk_cluster_max_n()).
+cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const int32_t *cand,
+                                int cand_stride, const int32_t *n_entries, const int32_t *q_pos,
+                                const int32_t *pool_len, int T, int row0, int nrows, int K,
+                                int32_t *out_idx, int32_t *out_cnt, int P, int32_t *out_pool,
+                                int32_t *out_pool_len, int64_t max_n, cudaStream_t st) {
+    tkc::Args a;
+    a.scores = scores; a.score_stride = score_stride;
+    a.cand = cand; a.cand_stride = cand_stride;
+    a.n_entries = n_entries; a.q_pos = q_pos; a.pool_len = pool_len; a.T = T;
+    a.row0 = row0; a.K = K; a.out_idx = out_idx; a.out_cnt = out_cnt;
+    a.P = P; a.out_pool = out_pool; a.out_pool_len = out_pool_len;
+    const int chunk = (int)((max_n + tkc::kCluster - 1) / tkc::kCluster);
+    const size_t smem = (size_t)(chunk > 0 ? chunk : 1) * sizeof(uint32_t);
+    static size_t attr_smem = 0;
+    if (smem > attr_smem) {
+        cudaError_t e = cudaFuncSetAttribute(tkc::topk_cluster_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_smem = smem;
+    }
+    tkc::topk_cluster_kernel<<<nrows * tkc::kCluster, tkc::kThreads, smem, st>>>(a);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2
