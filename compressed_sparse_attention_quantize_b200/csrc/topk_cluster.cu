@@ -22,7 +22,7 @@ namespace tkc {
 namespace cg = cooperative_groups;
 
 constexpr int kCluster = 8;
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
 constexpr int kMaxChunk = 32768;                   // keys per CTA (128 KB of shared memory)
 
 struct Args {
@@ -57,6 +57,7 @@ CSA2_D int64_t row_n(const Args &a, int r) {
 
 struct Shared {
     unsigned int hist[2][256];
+    unsigned int total[256];
     int counts[2];              // [0] above threshold, [1] equal to it
     int warp_sums[33];
     uint32_t prefix, mask;
@@ -104,17 +105,24 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
             if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
         }
         cl.sync();                                  // every CTA's histogram is complete
+        if (threadIdx.x < 256) {                    // bin t summed over the cluster (8 DSMEM loads)
+            unsigned int v[kCluster];
+#pragma unroll
+            for (int c = 0; c < kCluster; ++c) v[c] = cl.map_shared_rank(h, c)[threadIdx.x];
+            unsigned int sum = 0;
+#pragma unroll
+            for (int c = 0; c < kCluster; ++c) sum += v[c];
+            S.total[threadIdx.x] = sum;
+        }
+        __syncthreads();
         if (threadIdx.x < 32) {
             const int lane = threadIdx.x;
             unsigned int bins[8];
             unsigned int local = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                unsigned int v = 0;
-#pragma unroll
-                for (int c = 0; c < kCluster; ++c) v += cl.map_shared_rank(h, c)[lane * 8 + i];
-                bins[i] = v;
-                local += v;
+                bins[i] = S.total[lane * 8 + i];
+                local += bins[i];
             }
             unsigned int suffix = local;            // sum over lanes >= lane
 #pragma unroll
