@@ -119,7 +119,7 @@ CSA2_D int block_exclusive_count(bool flag, int *warp_sums, int &total) {
     if (lane == 0) warp_sums[warp] = __popc(bal);
     __syncthreads();
     if (warp == 0) {
-        int v = warp_sums[lane];
+        int v = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
         int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -214,7 +214,7 @@ __device__ void select_row(const float *scores, const int32_t *ids, int64_t n, i
             const bool sel = gt || (eq && run_eq + eq_rank < need_eq);
             int sel_total;
             const int pos = block_exclusive_count(sel, warp_sums, sel_total);
-            if (sel) out[run_out + pos] = ids ? ids[j] : (int32_t)j;
+            if (sel && run_out + pos < k) out[run_out + pos] = ids ? ids[j] : (int32_t)j;
             run_out += sel_total;
             run_eq += eq_total;
         }

@@ -64,14 +64,17 @@ struct Shared {
     int remaining;
 };
 
-// Block-wide exclusive count of a flag in thread order (kThreads threads).
+// Block-wide exclusive count of a flag in thread order (kThreads threads, kThreads/32 warps;
+// warp 0 scans one partial per warp and zero for lanes beyond the warp count).
+static_assert(kThreads % 32 == 0 && kThreads <= 1024, "block_excl needs whole warps, at most 32");
+static_assert(kThreads >= 256, "one thread per histogram bin");
 CSA2_D int block_excl(bool f, int *ws, int &total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned bal = __ballot_sync(0xffffffffu, f);
     if (lane == 0) ws[warp] = __popc(bal);
     __syncthreads();
     if (warp == 0) {
-        const int v = ws[lane];
+        const int v = lane < kThreads / 32 ? ws[lane] : 0;
         int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -189,7 +192,8 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
         const int pos = block_excl(sel, S.warp_sums, sel_tot);
         if (sel) {
             const int64_t j = chunk_base + i;
-            out[out_base + run_out + pos] = ids ? ids[j] : (int32_t)j;
+            const int o = out_base + run_out + pos;
+            if (o < k) out[o] = ids ? ids[j] : (int32_t)j;     // never past the row's k slots
         }
         run_out += sel_tot;
         run_eq += eq_tot;
