@@ -28,7 +28,7 @@ constexpr int kTile = 128;
 constexpr int kThreads = 128;
 constexpr int kMaxN = 4 * CSA2_MAX_INDEX_HEADS;      // 64 columns
 constexpr int kTilesPerCta = 8;                      // 1024 keys per CTA
-constexpr int kDepth = 4;                            // tiles of key rows in flight per thread
+constexpr int kDepth = 2;                            // tiles of key rows in flight per thread
 
 struct Args {
     const uint8_t *q_codes, *q_scales;
@@ -51,11 +51,11 @@ struct Args {
 };
 
 struct __align__(16) Smem {
-    uint8_t a[2][2 * kTile * 16];      // keys: two 16-byte planes, double-buffered
+    uint8_t a[2 * kTile * 16];         // keys: two 16-byte planes
     uint8_t b[2 * kMaxN * 16];         // block-diagonal query
     float qs[CSA2_MAX_INDEX_HEADS * 4];// query block scales
     float w[CSA2_MAX_INDEX_HEADS];
-    uint64_t done[2], drain;
+    uint64_t done, drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -95,7 +95,7 @@ CSA2_D void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t i
         : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 8)
 index_score_tc_kernel(Args a) {
     __shared__ Smem S;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -108,14 +108,13 @@ index_score_tc_kernel(Args a) {
     const int H = a.H;
     const int N = ((4 * H + 15) / 16) * 16;
     const uint32_t tmem_cols = a.tmem_cols;
-    const uint32_t sf_col = 2 * N;
+    const uint32_t sf_col = N;
 
     // ---- setup: query (block-diagonal B), scales, weights, barriers, TMEM ----
     for (int i = t; i < (int)(sizeof(S.b) / 16); i += kThreads)
         reinterpret_cast<uint4 *>(S.b)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (t == 0) {
-        ptx::mbar_init(&S.done[0], 1);
-        ptx::mbar_init(&S.done[1], 1);
+        ptx::mbar_init(&S.done, 1);
         ptx::mbar_init(&S.drain, 1);
         S.abort_flag = 0;
         ptx::fence_async_smem();
@@ -183,74 +182,54 @@ index_score_tc_kernel(Args a) {
     bool valid[kDepth];
 #pragma unroll
     for (int k = 0; k < kDepth; ++k) key_row(k, c0[k], c1[k], sc[k], valid[k]);
-    const uint32_t a_addr = ptx::smem_u32(S.a[0]);
+    const uint64_t adesc = sdesc_noswizzle(ptx::smem_u32(S.a), kTile * 16, 128);
     bool aborted = false;
-    uint32_t sc_prev = 0u;
-    bool valid_prev = false;
-    // step i: stage + MMA for tile i (if any), then the epilogue of tile i-1 (if any)
-    for (int i0 = 0; i0 <= ntiles && !aborted; i0 += kDepth) {
+    for (int i0 = 0; i0 < ntiles && !aborted; i0 += kDepth) {
 #pragma unroll
         for (int k = 0; k < kDepth; ++k) {
             const int i = i0 + k;
-            if (i > ntiles) break;
-            const int buf = i & 1;
-            uint32_t sc_this = 0u;
-            bool valid_this = false;
-            if (i < ntiles) {
-                // A[buf] was last read by the MMA of tile i-2, which completed before the
-                // epilogue of tile i-2 (step i-1) read its D
-                *reinterpret_cast<uint4 *>(S.a[buf] + t * 16) = c0[k];
-                *reinterpret_cast<uint4 *>(S.a[buf] + kTile * 16 + t * 16) = c1[k];
-                ptx::fence_async_smem();
-                ptx::tc_fence_before();
-            }
-            __syncthreads();                       // also: every thread is done reading D[buf]
-            if (i < ntiles) {
-                if (t == 0) {
-                    ptx::tc_fence_after();
-                    const uint64_t adesc = sdesc_noswizzle(a_addr + buf * (2 * kTile * 16), kTile * 16, 128);
-                    mma_mxf4(tmem + buf * N, adesc, bdesc, idesc, sf, sf);
-                    ptx::mma_commit(&S.done[buf]);
-                }
-                sc_this = sc[k];
-                valid_this = valid[k];
-                if (i + kDepth < ntiles) key_row(i + kDepth, c0[k], c1[k], sc[k], valid[k]);
-            }
-            if (i > 0) {
-                // epilogue of tile i-1
-                const int pb = (i - 1) & 1;
-                ptx::mbar_wait(&S.done[pb], ((i - 1) >> 1) & 1, abort_flag);
-                if (__syncthreads_or(*abort_flag != 0)) { aborted = true; break; }
+            if (i >= ntiles) break;
+            // stage tile i: the previous MMA has completed and every thread has read its D
+            *reinterpret_cast<uint4 *>(S.a + t * 16) = c0[k];
+            *reinterpret_cast<uint4 *>(S.a + kTile * 16 + t * 16) = c1[k];
+            ptx::fence_async_smem();
+            ptx::tc_fence_before();
+            __syncthreads();
+            if (t == 0) {
                 ptx::tc_fence_after();
-                float sk[4];
+                mma_mxf4(tmem, adesc, bdesc, idesc, sf, sf);
+                ptx::mma_commit(&S.done);
+            }
+            const uint32_t sc_this = sc[k];
+            const bool valid_this = valid[k];
+            if (i + kDepth < ntiles) key_row(i + kDepth, c0[k], c1[k], sc[k], valid[k]);
+            ptx::mbar_wait(&S.done, i & 1, abort_flag);
+            if (__syncthreads_or(*abort_flag != 0)) { aborted = true; break; }
+            ptx::tc_fence_after();
+            float sk[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_prev >> (8 * q)) & 0xFFu);
-                float acc = 0.0f;
-                for (int hb = 0; hb * 8 < H; ++hb) {
-                    uint32_t u[32];
-                    ptx::tmem_ld32(lane_addr + pb * N + hb * 32, u);
-                    ptx::tmem_ld_wait();
+            for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
+            float acc = 0.0f;
+            for (int hb = 0; hb * 8 < H; ++hb) {
+                uint32_t u[32];
+                ptx::tmem_ld32(lane_addr + hb * 32, u);
+                ptx::tmem_ld_wait();
 #pragma unroll
-                    for (int hh = 0; hh < 8; ++hh) {
-                        const int h = hb * 8 + hh;
-                        if (h < H) {
-                            float p[4];
+                for (int hh = 0; hh < 8; ++hh) {
+                    const int h = hb * 8 + hh;
+                    if (h < H) {
+                        float p[4];
 #pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[h * 4 + q], sk[q]));
-                            const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
-                            const float rl = dot > 0.0f ? dot : 0.0f;
-                            acc = __fadd_rn(acc, __fmul_rn(S.w[h], rl));
-                        }
+                        for (int q = 0; q < 4; ++q)
+                            p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[h * 4 + q], sk[q]));
+                        const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
+                        const float rl = dot > 0.0f ? dot : 0.0f;
+                        acc = __fadd_rn(acc, __fmul_rn(S.w[h], rl));
                     }
                 }
-                ptx::tc_fence_before();
-                if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
-                if (valid_prev)
-                    a.scores[(int64_t)blockIdx.y * a.score_stride + j0 + (int64_t)(i - 1) * kTile + t] = acc;
             }
-            sc_prev = sc_this;
-            valid_prev = valid_this;
+            if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
+            if (valid_this) a.scores[(int64_t)blockIdx.y * a.score_stride + j0 + (int64_t)i * kTile + t] = acc;
         }
     }
     if (aborted && t == 0) {           // drain the tensor pipe before TMEM is released
@@ -283,10 +262,10 @@ cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, flo
     a.scores = scores;
     a.score_stride = score_stride;
     const int64_t per_cta = (int64_t)itc::kTilesPerCta * itc::kTile;
-    // TMEM per CTA: two D buffers of N columns + 32 columns of unit scale factors
+    // TMEM per CTA: D (N columns) + 32 columns of unit scale factors
     const int N = ((4 * L.H + 15) / 16) * 16;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * N + 32)) cols <<= 1;
+    while (cols < (uint32_t)(N + 32)) cols <<= 1;
     a.tmem_cols = cols;
     // reserve shared memory so that at most 512/cols CTAs are resident on an SM
     const int per_sm = 512 / (int)cols;

@@ -103,9 +103,15 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
         for (int i = threadIdx.x; i < 256; i += kThreads) h[i] = 0u;
         __syncthreads();
         const uint32_t prefix = S.prefix, mask = S.mask;
-        for (int i = threadIdx.x; i < chunk_len; i += kThreads) {
-            const uint32_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+        // warp-aggregated: lanes with the same bin add once (the top digits of nearby scores
+        // collide heavily, which would serialise plain shared-memory atomics)
+        for (int base = 0; base < chunk_len; base += kThreads) {
+            const int i = base + threadIdx.x;
+            const uint32_t key = i < chunk_len ? keys[i] : 0u;
+            const bool in = i < chunk_len && (key & mask) == prefix;
+            const uint32_t bin = in ? ((key >> shift) & 255u) : 256u;
+            const unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], (unsigned)__popc(peers));
         }
         cl.sync();                                  // every CTA's histogram is complete
         if (threadIdx.x < 256) {                    // bin t summed over the cluster (8 DSMEM loads)
@@ -201,7 +207,7 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
     cl.sync();                                      // counts may be reused by the next selection
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
 topk_cluster_kernel(Args a) {
     extern __shared__ __align__(16) uint32_t keys[];
     __shared__ Shared S;
