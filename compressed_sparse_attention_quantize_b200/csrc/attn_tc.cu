@@ -292,76 +292,69 @@ attn_tc_kernel(AttnArgs a) {
     volatile int *abort_flag = &S.abort_flag;
 
     if (warp == 0) {
-        // ================= MMA issuer =================
-        const uint32_t idesc_s = ptx::idesc_f16_f32(128, kHeads, false, false);
-        const uint32_t idesc_pv = ptx::idesc_f16_f32(128, kHeads, true, true);
-        const uint32_t q_addr = ptx::smem_u32(sQ), v_addr = ptx::smem_u32(sV), p_addr = ptx::smem_u32(sP);
-        for (int j = 0; j < ntiles; ++j) {
-            const uint32_t ph = j & 1;
-            if (j > 0) {
-                ptx::mbar_wait(&S.s_empty, ph ^ 1, abort_flag);
-                __syncwarp();
-                if (*abort_flag) break;
-            }
-            bool ok = true;
-            for (int rg = 0; rg < kRegions; ++rg) {
-                ptx::mbar_wait(&S.v_full[rg], ph, abort_flag);
-                __syncwarp();
-                if (*abort_flag) { ok = false; break; }
-                ptx::tc_fence_after();
-                if (lane == 0) {
+        // ================= MMA issuer (lane 0 alone) =================
+        // Descriptors are built once; every MMA adds a compile-time offset to the start-address
+        // field (addresses stay below 256 KB, so the 14-bit field never carries).
+        if (lane == 0) {
+            const uint32_t idesc_s = ptx::idesc_f16_f32(128, kHeads, false, false);
+            const uint32_t idesc_pv = ptx::idesc_f16_f32(128, kHeads, true, true);
+            const uint64_t s_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), 16, 1024);
+            const uint64_t s_b0 = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
+            const uint64_t pv_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), kVRegion, 1024);
+            const uint64_t pv_b0 = ptx::sdesc_sw128(ptx::smem_u32(sP), kPBytes, 1024);
+            for (int j = 0; j < ntiles; ++j) {
+                const uint32_t ph = j & 1;
+                if (j > 0 && !ptx::mbar_wait(&S.s_empty, ph ^ 1, abort_flag)) break;
+                bool ok = true;
+                uint64_t ad = s_a0, bd = s_b0;
+#pragma unroll 1
+                for (int rg = 0; rg < kRegions; ++rg) {
+                    if (!ptx::mbar_wait(&S.v_full[rg], ph, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t ad = ptx::sdesc_sw128(v_addr + rg * kVRegion + k * 32, 16, 1024);
-                        const uint64_t bd = ptx::sdesc_sw128(q_addr + rg * kQRegion + k * 32, 16, 1024);
-                        ptx::mma_f16_ss(tmem, ad, bd, idesc_s, (rg | k) != 0);
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        ptx::mma_f16_ss(tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc_s,
+                                        (rg | k) != 0);
+                    ad += (uint64_t)(kVRegion >> 4);
+                    bd += (uint64_t)(kQRegion >> 4);
                 }
-                __syncwarp();
-            }
-            if (!ok) break;
-            if (lane == 0) ptx::mma_commit(&S.s_full);
-            __syncwarp();
-            ptx::mbar_wait(&S.p_full, ph, abort_flag);
-            __syncwarp();
-            if (*abort_flag) break;
-            ptx::tc_fence_after();
-            if (lane == 0) {
+                if (!ok) break;
+                ptx::mma_commit(&S.s_full);
+                if (!ptx::mbar_wait(&S.p_full, ph, abort_flag)) break;
+                ptx::tc_fence_after();
+#pragma unroll 1
                 for (int mb = 0; mb < 4; ++mb) {
+                    uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pv_b0;
 #pragma unroll
                     for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint64_t ad = ptx::sdesc_sw128(v_addr + 2 * mb * kVRegion + kk * 2048, kVRegion, 1024);
-                        const uint64_t bd = ptx::sdesc_sw128(p_addr + kk * 2048, kPBytes, 1024);
-                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, ad, bd, idesc_pv, (j > 0 || kk > 0));
+                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, a2, b2, idesc_pv, (j > 0 || kk > 0));
+                        a2 += (uint64_t)(2048 >> 4);
+                        b2 += (uint64_t)(2048 >> 4);
                     }
                 }
                 ptx::mma_commit(&S.pv_hi_done);
-            }
-            __syncwarp();
-            // low halves of P: P - fp16(P), same accumulators (P is then exact to ~2^-22)
-            ptx::mbar_wait(&S.p_lo_full, ph, abort_flag);
-            __syncwarp();
-            if (*abort_flag) break;
-            ptx::tc_fence_after();
-            if (lane == 0) {
+                // low halves of P: P - fp16(P), same accumulators (P is then exact to ~2^-22)
+                if (!ptx::mbar_wait(&S.p_lo_full, ph, abort_flag)) break;
+                ptx::tc_fence_after();
+#pragma unroll 1
                 for (int mb = 0; mb < 4; ++mb) {
+                    uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pv_b0;
 #pragma unroll
                     for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint64_t ad = ptx::sdesc_sw128(v_addr + 2 * mb * kVRegion + kk * 2048, kVRegion, 1024);
-                        const uint64_t bd = ptx::sdesc_sw128(p_addr + kk * 2048, kPBytes, 1024);
-                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, ad, bd, idesc_pv, 1u);
+                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, a2, b2, idesc_pv, 1u);
+                        a2 += (uint64_t)(2048 >> 4);
+                        b2 += (uint64_t)(2048 >> 4);
                     }
                     ptx::mma_commit(&S.v_empty[2 * mb]);
                     ptx::mma_commit(&S.v_empty[2 * mb + 1]);
                 }
                 ptx::mma_commit(&S.pv_done);
             }
-            __syncwarp();
+            // every issued MMA must have completed before TMEM is released (also after an abort)
+            ptx::mma_commit(&S.drain);
+            ptx::mbar_wait_drain(&S.drain, 0);
         }
-        // every issued MMA must have completed before TMEM is released (also after an abort)
-        if (lane == 0) ptx::mma_commit(&S.drain);
         __syncwarp();
-        ptx::mbar_wait_drain(&S.drain, 0);
     } else {
         // ================= workers: key t = sub*32 + lane; half = channel/head half =========
         const int sub = warp & 3;
