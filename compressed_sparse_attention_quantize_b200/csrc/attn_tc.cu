@@ -304,13 +304,16 @@ attn_tc_kernel(AttnArgs a) {
             const uint64_t pv_b0 = ptx::sdesc_sw128(ptx::smem_u32(sP), kPBytes, 1024);
             for (int j = 0; j < ntiles; ++j) {
                 const uint32_t ph = j & 1;
-                if (j > 0 && !ptx::mbar_wait(&S.s_empty, ph ^ 1, abort_flag)) break;
+                if (j > 0) {
+                    if (!ptx::mbar_wait(&S.s_empty, ph ^ 1, abort_flag)) break;
+                    ptx::tc_fence_after();              // S^T columns: the softmax reads are done
+                }
                 bool ok = true;
                 uint64_t ad = s_a0, bd = s_b0;
 #pragma unroll 1
                 for (int rg = 0; rg < kRegions; ++rg) {
+                    // dequantisers fenced their stores to the async proxy before arriving
                     if (!ptx::mbar_wait(&S.v_full[rg], ph, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         ptx::mma_f16_ss(tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc_s,
@@ -335,7 +338,6 @@ attn_tc_kernel(AttnArgs a) {
                 ptx::mma_commit(&S.pv_hi_done);
                 // low halves of P: P - fp16(P), same accumulators (P is then exact to ~2^-22)
                 if (!ptx::mbar_wait(&S.p_lo_full, ph, abort_flag)) break;
-                ptx::tc_fence_after();
 #pragma unroll 1
                 for (int mb = 0; mb < 4; ++mb) {
                     uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pv_b0;
