@@ -24,9 +24,10 @@
 //
 // Warp roles (9 warps): 0 = TMEM owner + MMA issuer; 1-8 = workers.  Worker warp w owns TMEM
 // sub-partition w%4 (keys 32*(w%4)..+31) and one half: it dequantises channels 256*half..+255
-// of its keys and runs the softmax for heads 32*half..+31.  Hand-offs use mbarriers per V
-// region (64 channels) so dequantising tile j+1 overlaps the P.V products of tile j; the
-// per-head max is only re-reduced when some logit exceeds the running max by 2^8.
+// of its keys and runs the softmax for heads 32*half..+31.  Hand-offs use one mbarrier per
+// channel half (every mbarrier wait costs the issuing thread ~140 cycles, measured), so the
+// dequantisation of one half overlaps the MMAs on the other; the per-head max is only
+// re-reduced when some logit exceeds the running max by 2^8.
 // Every wait is bounded: on expiry the CTA records CSA2_ERR_TIMEOUT, drains, frees TMEM and exits.
 #include "attn.cuh"
 #include "tc_ptx.cuh"
@@ -50,8 +51,8 @@ constexpr int kOCol = 256;                 // O^T accumulators at columns 256..5
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Smem {
-    uint64_t v_full[kRegions];
-    uint64_t v_empty[kRegions];
+    uint64_t v_full[2];                    // per channel half: the half's 4 regions are written
+    uint64_t v_empty[2];                   // per channel half: the P.V products reading it are done
     uint64_t s_full, s_empty, p_full, pv_hi_done, p_lo_full, pv_done, drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -211,7 +212,7 @@ attn_tc_kernel(AttnArgs a) {
 
     // ---------------- setup ----------------
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kRegions; ++i) {
+        for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&S.v_full[i], kWorkers / 2);
             ptx::mbar_init(&S.v_empty[i], 1);
         }
@@ -312,8 +313,9 @@ attn_tc_kernel(AttnArgs a) {
                 uint64_t ad = s_a0, bd = s_b0;
 #pragma unroll 1
                 for (int rg = 0; rg < kRegions; ++rg) {
-                    // dequantisers fenced their stores to the async proxy before arriving
-                    if (!ptx::mbar_wait(&S.v_full[rg], ph, abort_flag)) { ok = false; break; }
+                    // one wait per channel half (an mbarrier wait stalls the issue stream for
+                    // ~140 cycles); dequantisers fenced their stores to the async proxy
+                    if ((rg & 3) == 0 && !ptx::mbar_wait(&S.v_full[rg >> 2], ph, abort_flag)) { ok = false; break; }
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         ptx::mma_f16_ss(tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc_s,
@@ -347,8 +349,7 @@ attn_tc_kernel(AttnArgs a) {
                         a2 += (uint64_t)(2048 >> 4);
                         b2 += (uint64_t)(2048 >> 4);
                     }
-                    ptx::mma_commit(&S.v_empty[2 * mb]);
-                    ptx::mma_commit(&S.v_empty[2 * mb + 1]);
+                    if (mb & 1) ptx::mma_commit(&S.v_empty[mb >> 1]);   // half mb/2 free
                 }
                 ptx::mma_commit(&S.pv_done);
             }
@@ -372,18 +373,19 @@ attn_tc_kernel(AttnArgs a) {
         for (int j = 0; j < ntiles && !aborted; ++j) {
             const uint32_t ph = j & 1;
             // ---- dequantise this thread's half of key t into V (regions 4*half .. 4*half+3)
+            if (j > 0 && !ptx::mbar_wait(&S.v_empty[half], ph ^ 1, abort_flag)) { aborted = true; }
+            if (aborted) break;
 #pragma unroll
             for (int rl = 0; rl < 4; ++rl) {
                 const int rg = half * 4 + rl;
                 uint4 out[8];
                 dequant_region(src, hr, rl, rg, out);
-                if (j > 0 && !ptx::mbar_wait(&S.v_empty[rg], ph ^ 1, abort_flag)) { aborted = true; break; }
                 uint8_t *dst = sV + rg * kVRegion;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + sw128_off(t, c)) = out[c];
-                ptx::fence_async_smem();
-                ptx::mbar_arrive(&S.v_full[rg]);
             }
+            ptx::fence_async_smem();
+            ptx::mbar_arrive(&S.v_full[half]);
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             ptx::mbar_wait(&S.s_full, ph, abort_flag);
             ptx::named_barrier(1, kWorkers);
