@@ -43,28 +43,34 @@ constexpr int kQRegion = kHeads * 128;     // 8 KB
 constexpr int kVRegion = kTile * 128;      // 16 KB
 constexpr int kQBytes = kRegions * kQRegion;         // 64 KB
 constexpr int kVBytes = kRegions * kVRegion;         // 128 KB
-constexpr int kPBytes = kTile * kHeads * 2;          // 16 KB
+constexpr int kPBytes = kTile * kHeads * 2;          // 16 KB (one of P_hi, P_lo)
 constexpr int kThreads = 288;             // warp 0: MMA issuer; warps 1-8: workers
 constexpr int kWorkers = 256;
 constexpr int kTmemCols = 512;
 constexpr int kOCol = 256;                 // O^T accumulators at columns 256..511
+constexpr int kLCol = 64;                  // per-key row-sum partials at columns 64..127
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Smem {
     uint64_t v_full[2];                    // per channel half: the half's 4 regions are written
     uint64_t v_empty[2];                   // per channel half: the P.V products reading it are done
-    uint64_t s_full, s_empty, p_full, pv_hi_done, p_lo_full, pv_done, drain;
+    uint64_t s_full, s_empty, p_full, pv_done, drain;
     uint32_t tmem_base;
     int abort_flag;
     int any_rescale;
     int q_exp_max;
     float m_run[kHeads];
     float alpha[kHeads];
-    float red[4][kHeads];
-    float lsum[4][kHeads];
 };
 
-constexpr int kSmemBytes = kQBytes + kVBytes + kPBytes + (int)sizeof(Smem) + 1024;
+// Scratch that lives in the P_lo buffer while that buffer is free: the per-head max reduction
+// (during a tile's softmax, before P_lo is rewritten) and the final row-sum reduction.
+struct Scratch {
+    float red[4][kHeads];
+    float inv_l[kHeads];
+};
+
+constexpr int kSmemBytes = kQBytes + kVBytes + 2 * kPBytes + (int)sizeof(Smem) + 1024;
 
 // Where key x of row r comes from.
 struct KeySrc {
@@ -194,8 +200,10 @@ attn_tc_kernel(AttnArgs a) {
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *sQ = base;
     uint8_t *sV = base + kQBytes;
-    uint8_t *sP = sV + kVBytes;
-    Smem &S = *reinterpret_cast<Smem *>(sP + kPBytes);
+    uint8_t *sP = sV + kVBytes;                     // P_hi
+    uint8_t *sPlo = sP + kPBytes;                   // P_lo
+    Smem &S = *reinterpret_cast<Smem *>(sPlo + kPBytes);
+    Scratch &X = *reinterpret_cast<Scratch *>(sPlo);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x;                       // query row
@@ -219,8 +227,6 @@ attn_tc_kernel(AttnArgs a) {
         ptx::mbar_init(&S.s_full, 1);
         ptx::mbar_init(&S.s_empty, kWorkers);
         ptx::mbar_init(&S.p_full, kWorkers);
-        ptx::mbar_init(&S.pv_hi_done, 1);
-        ptx::mbar_init(&S.p_lo_full, kWorkers);
         ptx::mbar_init(&S.pv_done, 1);
         ptx::mbar_init(&S.drain, 1);
         S.abort_flag = 0;
@@ -229,7 +235,6 @@ attn_tc_kernel(AttnArgs a) {
         ptx::fence_async_smem();
     }
     if (threadIdx.x < kHeads) S.m_run[threadIdx.x] = -INFINITY;
-    if (threadIdx.x < 4 * kHeads) S.lsum[threadIdx.x / kHeads][threadIdx.x % kHeads] = 0.0f;
     if (warp == 0) {
         ptx::tmem_alloc(&S.tmem_base, kTmemCols);
         ptx::tmem_relinquish();
@@ -303,6 +308,7 @@ attn_tc_kernel(AttnArgs a) {
             const uint64_t s_b0 = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
             const uint64_t pv_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), kVRegion, 1024);
             const uint64_t pv_b0 = ptx::sdesc_sw128(ptx::smem_u32(sP), kPBytes, 1024);
+            const uint64_t pvlo_b0 = ptx::sdesc_sw128(ptx::smem_u32(sPlo), kPBytes, 1024);
             for (int j = 0; j < ntiles; ++j) {
                 const uint32_t ph = j & 1;
                 if (j > 0) {
@@ -337,12 +343,10 @@ attn_tc_kernel(AttnArgs a) {
                         b2 += (uint64_t)(2048 >> 4);
                     }
                 }
-                ptx::mma_commit(&S.pv_hi_done);
-                // low halves of P: P - fp16(P), same accumulators (P is then exact to ~2^-22)
-                if (!ptx::mbar_wait(&S.p_lo_full, ph, abort_flag)) break;
+                // low halves of P (P - fp16(P)) into the same accumulators: P exact to ~2^-22
 #pragma unroll 1
                 for (int mb = 0; mb < 4; ++mb) {
-                    uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pv_b0;
+                    uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pvlo_b0;
 #pragma unroll
                     for (int kk = 0; kk < kTile / 16; ++kk) {
                         ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, a2, b2, idesc_pv, 1u);
@@ -367,6 +371,15 @@ attn_tc_kernel(AttnArgs a) {
         const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
         const float qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-qshift);
         bool aborted = false;
+        // this key's share of the row sums lives in TMEM (lane = key, 32 columns per half)
+        const uint32_t l_addr = lane_addr + kLCol + half * 32;
+        {
+            uint32_t zero[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) zero[i] = 0u;
+            ptx::tmem_st32(l_addr, zero);
+            ptx::tmem_st_wait();
+        }
         KeySrc src = key_source(a, r, b, x_begin + t, x_end, n_sel);
         HalfRow hr;
         prefetch_half(src, half, hr);
@@ -415,10 +428,10 @@ attn_tc_kernel(AttnArgs a) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = z[i];
                 warp_transpose_reduce<false>(v, lane);
-                S.red[sub][half * 32 + lane] = v[0];
+                X.red[sub][half * 32 + lane] = v[0];
                 ptx::named_barrier(1, kWorkers);
                 if (wt < kHeads) {
-                    const float tmax = fmaxf(fmaxf(S.red[0][wt], S.red[1][wt]), fmaxf(S.red[2][wt], S.red[3][wt]));
+                    const float tmax = fmaxf(fmaxf(X.red[0][wt], X.red[1][wt]), fmaxf(X.red[2][wt], X.red[3][wt]));
                     const float mo = S.m_run[wt];
                     float al = 1.0f;
                     if (tmax > mo + kRescaleThreshold) {
@@ -437,15 +450,18 @@ attn_tc_kernel(AttnArgs a) {
                 const float m = S.m_run[half * 32 + i];
                 z[i] = (m == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[i] - m);
             }
-            // this tile's row sums: lane L owns head 32*half + L of its 32 keys
+            // row sums: per key in TMEM, reduced over the keys once at the end
             {
-                float v[32];
+                uint32_t u[32];
+                ptx::tmem_ld32(l_addr, u);
+                ptx::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = z[i];
-                warp_transpose_reduce<true>(v, lane);
-                const int h = half * 32 + lane;
-                const float al = move ? S.alpha[h] : 1.0f;
-                S.lsum[sub][h] = S.lsum[sub][h] * al + v[0];
+                for (int i = 0; i < 32; ++i) {
+                    const float lp = __uint_as_float(u[i]);
+                    u[i] = __float_as_uint((move ? lp * S.alpha[half * 32 + i] : lp) + z[i]);
+                }
+                ptx::tmem_st32(l_addr, u);
+                ptx::tmem_st_wait();
             }
             // P.V of the previous tile completed before this tile's S (the tensor pipe runs in
             // order), so this wait is immediate; it orders the P rewrite and the O^T rescale.
@@ -455,11 +471,12 @@ attn_tc_kernel(AttnArgs a) {
                 if (*abort_flag) { aborted = true; break; }
                 ptx::tc_fence_after();
             }
-            // P^T line of key t, heads of this half: fp16 high half now, low half kept
-            uint32_t plo[16];
+            // P^T line of key t for this half's heads: fp16 high halves to P_hi, low halves
+            // (P - fp16(P)) to P_lo; the max scratch in the P_lo buffer is no longer read
+            ptx::named_barrier(1, kWorkers);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t hi4[4];
+                uint32_t hi4[4], lo4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int i = 8 * c + 2 * k;
@@ -468,10 +485,10 @@ attn_tc_kernel(AttnArgs a) {
                     const float2 back = __half22float2(hp);
                     const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
                     hi4[k] = *reinterpret_cast<const uint32_t *>(&hp);
-                    plo[4 * c + k] = *reinterpret_cast<const uint32_t *>(&lp);
+                    lo4[k] = *reinterpret_cast<const uint32_t *>(&lp);
                 }
-                *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) =
-                    make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                *reinterpret_cast<uint4 *>(sPlo + sw128_off(t, half * 4 + c)) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
             }
             // O^T rescale for heads whose running max moved (columns of this half)
             if (rescale && j > 0) {
@@ -500,16 +517,6 @@ attn_tc_kernel(AttnArgs a) {
                 src = key_source(a, r, b, x_begin + (j + 1) * kTile + t, x_end, n_sel);
                 prefetch_half(src, half, hr);
             }
-            // once the high halves have been consumed, the same buffer takes the low halves
-            ptx::mbar_wait(&S.pv_hi_done, ph, abort_flag);
-            ptx::named_barrier(1, kWorkers);
-            if (*abort_flag) { aborted = true; break; }
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) =
-                    make_uint4(plo[4 * c], plo[4 * c + 1], plo[4 * c + 2], plo[4 * c + 3]);
-            ptx::fence_async_smem();
-            ptx::mbar_arrive(&S.p_lo_full);
         }
         // ---------------- epilogue ----------------
         if (!aborted && ntiles > 0) {
@@ -518,13 +525,28 @@ attn_tc_kernel(AttnArgs a) {
         ptx::named_barrier(1, kWorkers);
         aborted = aborted || *abort_flag != 0;
         ptx::tc_fence_after();
+        // row sums: reduce the per-key partials over this warp's 32 keys, then over the 4
+        // sub-partitions
+        {
+            float v[32];
+            {
+                uint32_t u[32];
+                ptx::tmem_ld32(l_addr, u);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(u[i]);
+            }
+            warp_transpose_reduce<true>(v, lane);
+            if (!aborted) X.red[sub][half * 32 + lane] = v[0];
+        }
+        ptx::named_barrier(1, kWorkers);
         if (!aborted) {
             const bool single = a.splits == 1;
             const int64_t part_idx = ((int64_t)r * a.hgroups + hg) * a.splits + split;
             float *part = a.partials + part_idx * kPartialFloats;
             if (wt < kHeads) {
-                const float l = ntiles > 0 ? S.lsum[0][wt] + S.lsum[1][wt] + S.lsum[2][wt] + S.lsum[3][wt] : 0.0f;
-                S.red[0][wt] = l > 0.0f ? 1.0f / l : 0.0f;       // 1/l for the single-split output
+                const float l = ntiles > 0 ? X.red[0][wt] + X.red[1][wt] + X.red[2][wt] + X.red[3][wt] : 0.0f;
+                X.inv_l[wt] = l > 0.0f ? 1.0f / l : 0.0f;       // 1/l for the single-split output
                 if (!single) {
                     part[wt] = ntiles > 0 ? S.m_run[wt] : -INFINITY;
                     part[kHeads + wt] = l;
@@ -553,7 +575,7 @@ attn_tc_kernel(AttnArgs a) {
                     if (!single) {
                         part[2 * kHeads + h * kLatent + c] = o;
                     } else {
-                        const float val = o * S.red[0][h];
+                        const float val = o * X.inv_l[h];
                         const int64_t oi = ((int64_t)r * a.H + h0 + h) * kLatent + c;
                         if (a.out_dtype == CSA2_DTYPE_F32)
                             reinterpret_cast<float *>(a.out)[oi] = val;
