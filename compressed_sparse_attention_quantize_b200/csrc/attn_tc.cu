@@ -39,6 +39,7 @@ namespace tc {
 constexpr int kTile = 128;                 // keys per tile (MMA M)
 constexpr int kHeads = 64;                 // heads per CTA (MMA N)
 constexpr int kRegions = 8;                // 64-channel blocks of the 512-wide latent
+constexpr int kBlocks = 4;                 // 128-channel blocks (P.V MMA M)
 constexpr int kQRegion = kHeads * 128;     // 8 KB
 constexpr int kVRegion = kTile * 128;      // 16 KB
 constexpr int kQBytes = kRegions * kQRegion;         // 64 KB
@@ -50,21 +51,22 @@ constexpr int kTmemCols = 512;
 constexpr int kOCol = 256;                 // O^T accumulators at columns 256..511
 constexpr int kLCol = 64;                  // per-key row-sum partials at columns 64..127
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int32_t kNoKey = INT32_MIN;
 
 struct Smem {
-    uint64_t v_full[2];                    // per channel half: the half's 4 regions are written
-    uint64_t v_empty[2];                   // per channel half: the P.V products reading it are done
-    uint64_t s_full, s_empty, p_full, pv_done, drain;
+    uint64_t v_full[2];                    // channels 0-255 / 256-511 of the tile are written
+    uint64_t v_empty[kBlocks];             // P.V of 128-channel block mb has completed
+    uint64_t s_full, p_full, pv_done, drain;
     uint32_t tmem_base;
     int abort_flag;
-    int any_rescale;
     int q_exp_max;
     float m_run[kHeads];
     float alpha[kHeads];
 };
 
 // Scratch that lives in the P_lo buffer while that buffer is free: the per-head max reduction
-// (during a tile's softmax, before P_lo is rewritten) and the final row-sum reduction.
+// (during a tile's softmax, after the previous tile's P.V has completed and before P_lo is
+// rewritten) and the final row-sum reduction.
 struct Scratch {
     float red[4][kHeads];
     float inv_l[kHeads];
@@ -72,26 +74,33 @@ struct Scratch {
 
 constexpr int kSmemBytes = kQBytes + kVBytes + 2 * kPBytes + (int)sizeof(Smem) + 1024;
 
-// Where key x of row r comes from.
+// Key x of row r, step 1: the entry number (>= 0), -1 - w for window position w, or kNoKey.
+CSA2_D int32_t entry_of(const AttnArgs &a, int r, int x, int x_end, int n_sel) {
+    if (x >= x_end) return kNoKey;
+    if (x < n_sel) {
+        const int32_t e = a.idx[(int64_t)r * a.K + x];
+        return e < 0 ? kNoKey : e;
+    }
+    return -1 - (x - n_sel);
+}
+
+// Step 2: where the key's bytes are.
 struct KeySrc {
     bool valid, swa;
     const uint8_t *ptr;      // main: 288-byte row; window: 512 E4M3 codes
     float scale;             // window token scale (1 for main entries, 0 if invalid)
 };
 
-CSA2_D KeySrc key_source(const AttnArgs &a, int r, int b, int x, int x_end, int n_sel) {
+CSA2_D KeySrc source_of(const AttnArgs &a, int r, int b, int64_t seq_start, int32_t e) {
     KeySrc k{false, false, nullptr, 0.0f};
-    if (x >= x_end) return k;
-    if (x < n_sel) {
-        const int32_t e = a.idx[(int64_t)r * a.K + x];
-        if (e < 0) return k;
-        k.valid = true;
-        k.ptr = a.kv + (a.seq_start[b] + e) * a.kv_row_stride;
+    if (e == kNoKey) return k;
+    k.valid = true;
+    if (e >= 0) {
+        k.ptr = a.kv + (seq_start + e) * a.kv_row_stride;
         k.scale = 1.0f;
     } else {
-        const int slot = (a.swa_start ? a.swa_start[r] : 0) + (x - n_sel);
+        const int slot = (a.swa_start ? a.swa_start[r] : 0) + (-1 - e);
         const int64_t srow = (int64_t)b * a.swa_cap + slot;
-        k.valid = true;
         k.swa = true;
         k.ptr = a.swa_codes + srow * kLatent;
         k.scale = a.swa_scale[srow];
@@ -121,35 +130,42 @@ CSA2_D uint32_t sw128_off(int row, int c) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
 }
 
-// Prefetched half-row of one key: main entries keep 128 code bytes + 16 scale bytes of the
-// four 64-channel regions of this thread's half; window keys are loaded per region.
-struct HalfRow {
+// The bytes of one main-entry key that a worker dequantises: regions 2mb + hsel (mb = 0..3),
+// i.e. 32 code bytes and 4 scale bytes per region.  Window keys are read per region instead.
+struct RowPart {
     uint4 codes[8];
-    uint4 scales;
+    uint32_t sc[4];
 };
 
-CSA2_D void prefetch_half(const KeySrc &src, int half, HalfRow &hr) {
+CSA2_D void prefetch_part(const KeySrc &src, int hsel, RowPart &rp) {
     if (src.valid && !src.swa) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hr.codes[i] = __ldg(p + half * 8 + i);
-        hr.scales = __ldg(p + 16 + half);
+        for (int mb = 0; mb < kBlocks; ++mb) {
+            rp.codes[2 * mb] = __ldg(p + 2 * (2 * mb + hsel));
+            rp.codes[2 * mb + 1] = __ldg(p + 2 * (2 * mb + hsel) + 1);
+        }
+        const uint4 s0 = __ldg(p + 16), s1 = __ldg(p + 17);     // scale bytes of regions 0-3, 4-7
+        rp.sc[0] = hsel ? s0.y : s0.x;
+        rp.sc[1] = hsel ? s0.w : s0.z;
+        rp.sc[2] = hsel ? s1.y : s1.x;
+        rp.sc[3] = hsel ? s1.w : s1.z;
     } else {                                     // always assigned: no stale registers live
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hr.codes[i] = make_uint4(0u, 0u, 0u, 0u);
-        hr.scales = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < 8; ++i) rp.codes[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rp.sc[i] = 0u;
     }
 }
 
-// Dequantise region `rg` (64 channels) of one key into 8 fp16 chunks.
-CSA2_D void dequant_region(const KeySrc &src, const HalfRow &hr, int rl, int rg, uint4 (&out)[8]) {
+// Dequantise region rg = 2mb + hsel (64 channels) of one key into 8 fp16 chunks.
+CSA2_D void dequant_region(const KeySrc &src, const RowPart &rp, int mb, int rg, uint4 (&out)[8]) {
     if (!src.valid) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) out[c] = make_uint4(0u, 0u, 0u, 0u);
     } else if (!src.swa) {
-        // rl = region index within the half: code bytes 32rl.., scale bytes 4rl..
-        const uint32_t sw = rl == 0 ? hr.scales.x : rl == 1 ? hr.scales.y : rl == 2 ? hr.scales.z : hr.scales.w;
-        const uint4 c0 = hr.codes[2 * rl], c1 = hr.codes[2 * rl + 1];
+        const uint32_t sw = rp.sc[mb];
+        const uint4 c0 = rp.codes[2 * mb], c1 = rp.codes[2 * mb + 1];
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const uint32_t s01 = ptx::e4m3x2_to_f16x2((uint16_t)(sw & 0xFFFFu));
         const uint32_t s23 = ptx::e4m3x2_to_f16x2((uint16_t)(sw >> 16));
@@ -181,6 +197,7 @@ CSA2_D void dequant_region(const KeySrc &src, const HalfRow &hr, int rl, int rg,
     }
 }
 
+// bar.red.or over `threads` threads: a barrier that also tells every thread whether any flag was set.
 CSA2_D bool block_any(bool flag, uint32_t barrier_id, uint32_t threads) {
     uint32_t r;
     asm volatile(
@@ -192,6 +209,65 @@ CSA2_D bool block_any(bool flag, uint32_t barrier_id, uint32_t threads) {
         : "r"((uint32_t)flag), "r"(barrier_id), "r"(threads)
         : "memory");
     return r != 0;
+}
+
+// The MMA issuer (one thread).  Every MMA sequence is straight-line code: an mbarrier wait or any
+// other memory instruction between two MMAs leaves the tensor pipe idle for a few hundred cycles
+// (measured), so each tile has three waits: the two channel halves of V, then P.
+// Kept out of line so that its few live values keep registers of their own.
+__device__ __noinline__ void issue_mmas(uint32_t tmem, uint8_t *sQ, uint8_t *sV, uint8_t *sP, uint8_t *sPlo,
+                                        Smem &S, int ntiles, volatile int *abort_flag) {
+    constexpr uint32_t idesc_s = ptx::idesc_f16_f32(128, kHeads, false, false);
+    constexpr uint32_t idesc_pv = ptx::idesc_f16_f32(128, kHeads, true, true);
+    // S^T = V . Q^T: A = V (K-major), B = Q (K-major); K step = 32 bytes, region = 64 channels
+    const uint64_t s_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), 16, 1024);
+    const uint64_t s_b0 = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
+    // O^T += V^T . P^T: A = V read MN-major (64 channels per 128-byte row, next 64 channels one
+    // region further), B = P^T (MN-major, 64 heads per row); K step = 16 keys = 2048 bytes
+    const uint64_t pv_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), kVRegion, 1024);
+    const uint64_t pv_b0 = ptx::sdesc_sw128(ptx::smem_u32(sP), kPBytes, 1024);
+    const uint64_t pvlo_b0 = ptx::sdesc_sw128(ptx::smem_u32(sPlo), kPBytes, 1024);
+    for (int j = 0; j < ntiles; ++j) {
+        const uint32_t ph = j & 1;
+        // S(j) is issued after P.V(j-1), whose P the softmax warps released before p_full(j-1),
+        // and s_full(j) completes only after P.V(j-1) has: no separate S-buffer hand-off.
+#pragma unroll
+        for (int hv = 0; hv < 2; ++hv) {
+            if (!ptx::mbar_wait(&S.v_full[hv], ph, abort_flag)) goto done;
+#pragma unroll
+            for (int rl = 0; rl < 4; ++rl)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int rg = hv * 4 + rl;
+                    ptx::mma_f16_ss(tmem, s_a0 + (uint64_t)(rg * (kVRegion >> 4) + k * 2),
+                                    s_b0 + (uint64_t)(rg * (kQRegion >> 4) + k * 2), idesc_s, (rg | k) != 0);
+                }
+        }
+        ptx::mma_commit(&S.s_full);
+        if (!ptx::mbar_wait(&S.p_full, ph, abort_flag)) break;
+        ptx::tc_fence_after();
+        // per 128-channel block: fp16(P) then P - fp16(P) (P exact to ~2^-22) into the same
+        // accumulators, then the block's V bytes are released to the dequantisers
+#pragma unroll
+        for (int mb = 0; mb < kBlocks; ++mb) {
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+                ptx::mma_f16_ss(tmem + kOCol + mb * kHeads,
+                                pv_a0 + (uint64_t)(mb * ((2 * kVRegion) >> 4) + kk * (2048 >> 4)),
+                                pv_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+                ptx::mma_f16_ss(tmem + kOCol + mb * kHeads,
+                                pv_a0 + (uint64_t)(mb * ((2 * kVRegion) >> 4) + kk * (2048 >> 4)),
+                                pvlo_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv, 1u);
+            ptx::mma_commit(&S.v_empty[mb]);
+        }
+        ptx::mma_commit(&S.pv_done);
+    }
+done:
+    // every issued MMA must have completed before TMEM is released (also after an abort)
+    ptx::mma_commit(&S.drain);
+    ptx::mbar_wait_drain(&S.drain, 0);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -218,19 +294,29 @@ attn_tc_kernel(AttnArgs a) {
     const int x_end = min(total, x_begin + a.keys_per_split);
     const int ntiles = x_end > x_begin ? (x_end - x_begin + kTile - 1) / kTile : 0;
 
+    // worker roles: key t = sub*32 + lane (TMEM sub-partition = warp % 4); hsel picks the
+    // channel regions 2mb + hsel it dequantises and the heads 32*hsel..+31 of its softmax
+    const int sub = warp & 3;
+    const int hsel = (warp - 1) >> 2;
+    const int t = sub * 32 + lane;
+    const int64_t seq_start = a.seq_start[b];
+    // the first tile's rows are requested before anything else
+    KeySrc src{false, false, nullptr, 0.0f};
+    RowPart rp;
+    if (warp > 0) {
+        src = source_of(a, r, b, seq_start, entry_of(a, r, x_begin + t, x_end, n_sel));
+        prefetch_part(src, hsel, rp);
+    }
+
     // ---------------- setup ----------------
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&S.v_full[i], kWorkers / 2);
-            ptx::mbar_init(&S.v_empty[i], 1);
-        }
+        for (int i = 0; i < 2; ++i) ptx::mbar_init(&S.v_full[i], kWorkers);
+        for (int i = 0; i < kBlocks; ++i) ptx::mbar_init(&S.v_empty[i], 1);
         ptx::mbar_init(&S.s_full, 1);
-        ptx::mbar_init(&S.s_empty, kWorkers);
         ptx::mbar_init(&S.p_full, kWorkers);
         ptx::mbar_init(&S.pv_done, 1);
         ptx::mbar_init(&S.drain, 1);
         S.abort_flag = 0;
-        S.any_rescale = 0;
         S.q_exp_max = 0;
         ptx::fence_async_smem();
     }
@@ -299,78 +385,17 @@ attn_tc_kernel(AttnArgs a) {
 
     if (warp == 0) {
         // ================= MMA issuer (lane 0 alone) =================
-        // Descriptors are built once; every MMA adds a compile-time offset to the start-address
-        // field (addresses stay below 256 KB, so the 14-bit field never carries).
-        if (lane == 0) {
-            const uint32_t idesc_s = ptx::idesc_f16_f32(128, kHeads, false, false);
-            const uint32_t idesc_pv = ptx::idesc_f16_f32(128, kHeads, true, true);
-            const uint64_t s_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), 16, 1024);
-            const uint64_t s_b0 = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
-            const uint64_t pv_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), kVRegion, 1024);
-            const uint64_t pv_b0 = ptx::sdesc_sw128(ptx::smem_u32(sP), kPBytes, 1024);
-            const uint64_t pvlo_b0 = ptx::sdesc_sw128(ptx::smem_u32(sPlo), kPBytes, 1024);
-            for (int j = 0; j < ntiles; ++j) {
-                const uint32_t ph = j & 1;
-                if (j > 0) {
-                    if (!ptx::mbar_wait(&S.s_empty, ph ^ 1, abort_flag)) break;
-                    ptx::tc_fence_after();              // S^T columns: the softmax reads are done
-                }
-                bool ok = true;
-                uint64_t ad = s_a0, bd = s_b0;
-#pragma unroll 1
-                for (int rg = 0; rg < kRegions; ++rg) {
-                    // one wait per channel half (an mbarrier wait stalls the issue stream for
-                    // ~140 cycles); dequantisers fenced their stores to the async proxy
-                    if ((rg & 3) == 0 && !ptx::mbar_wait(&S.v_full[rg >> 2], ph, abort_flag)) { ok = false; break; }
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        ptx::mma_f16_ss(tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc_s,
-                                        (rg | k) != 0);
-                    ad += (uint64_t)(kVRegion >> 4);
-                    bd += (uint64_t)(kQRegion >> 4);
-                }
-                if (!ok) break;
-                ptx::mma_commit(&S.s_full);
-                if (!ptx::mbar_wait(&S.p_full, ph, abort_flag)) break;
-                ptx::tc_fence_after();
-#pragma unroll 1
-                for (int mb = 0; mb < 4; ++mb) {
-                    uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pv_b0;
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, a2, b2, idesc_pv, (j > 0 || kk > 0));
-                        a2 += (uint64_t)(2048 >> 4);
-                        b2 += (uint64_t)(2048 >> 4);
-                    }
-                }
-                // low halves of P (P - fp16(P)) into the same accumulators: P exact to ~2^-22
-#pragma unroll 1
-                for (int mb = 0; mb < 4; ++mb) {
-                    uint64_t a2 = pv_a0 + (uint64_t)mb * (uint64_t)((2 * kVRegion) >> 4), b2 = pvlo_b0;
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        ptx::mma_f16_ss(tmem + kOCol + mb * kHeads, a2, b2, idesc_pv, 1u);
-                        a2 += (uint64_t)(2048 >> 4);
-                        b2 += (uint64_t)(2048 >> 4);
-                    }
-                    if (mb & 1) ptx::mma_commit(&S.v_empty[mb >> 1]);   // half mb/2 free
-                }
-                ptx::mma_commit(&S.pv_done);
-            }
-            // every issued MMA must have completed before TMEM is released (also after an abort)
-            ptx::mma_commit(&S.drain);
-            ptx::mbar_wait_drain(&S.drain, 0);
-        }
+        if (lane == 0) issue_mmas(tmem, sQ, sV, sP, sPlo, S, ntiles, abort_flag);
         __syncwarp();
     } else {
-        // ================= workers: key t = sub*32 + lane; half = channel/head half =========
-        const int sub = warp & 3;
-        const int half = (warp - 1) >> 2;
-        const int t = sub * 32 + lane;
+        // ================= workers =================
+        const int half = hsel;
         const int wt = threadIdx.x - 32;                 // 0..255
         const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
         const float qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-qshift);
-        bool aborted = false;
+        // A wait that fails (abort or timeout) only marks `bad`; every worker keeps taking the
+        // same barriers, and the decision to stop is collective (bar.red.or) once per tile.
+        bool bad = false, aborted = false;
         // this key's share of the row sums lives in TMEM (lane = key, 32 columns per half)
         const uint32_t l_addr = lane_addr + kLCol + half * 32;
         {
@@ -380,29 +405,34 @@ attn_tc_kernel(AttnArgs a) {
             ptx::tmem_st32(l_addr, zero);
             ptx::tmem_st_wait();
         }
-        KeySrc src = key_source(a, r, b, x_begin + t, x_end, n_sel);
-        HalfRow hr;
-        prefetch_half(src, half, hr);
-        for (int j = 0; j < ntiles && !aborted; ++j) {
+        for (int j = 0; j < ntiles; ++j) {
             const uint32_t ph = j & 1;
-            // ---- dequantise this thread's half of key t into V (regions 4*half .. 4*half+3)
-            if (j > 0 && !ptx::mbar_wait(&S.v_empty[half], ph ^ 1, abort_flag)) { aborted = true; }
-            if (aborted) break;
+            // the next tile's entry number is read now and used after the dequantisation
+            const int32_t e_next = (j + 1 < ntiles) ? entry_of(a, r, x_begin + (j + 1) * kTile + t, x_end, n_sel) : kNoKey;
+            // ---- dequantise regions 2mb + hsel of key t; block mb is free once P.V(j-1) has
+            //      finished with it
 #pragma unroll
-            for (int rl = 0; rl < 4; ++rl) {
-                const int rg = half * 4 + rl;
+            for (int mb = 0; mb < kBlocks; ++mb) {
+                if (j > 0 && !ptx::mbar_wait(&S.v_empty[mb], ph ^ 1, abort_flag)) bad = true;
+                const int rg = 2 * mb + hsel;
                 uint4 out[8];
-                dequant_region(src, hr, rl, rg, out);
+                dequant_region(src, rp, mb, rg, out);
                 uint8_t *dst = sV + rg * kVRegion;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + sw128_off(t, c)) = out[c];
+                if (mb & 1) {
+                    ptx::fence_async_smem();
+                    ptx::mbar_arrive(&S.v_full[mb >> 1]);
+                }
             }
-            ptx::fence_async_smem();
-            ptx::mbar_arrive(&S.v_full[half]);
+            const bool cur_valid = src.valid;
+            const float cur_scale = src.scale;
+            // ---- the next tile's rows are requested before the softmax
+            src = source_of(a, r, b, seq_start, e_next);
+            prefetch_part(src, hsel, rp);
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
-            ptx::mbar_wait(&S.s_full, ph, abort_flag);
-            ptx::named_barrier(1, kWorkers);
-            if (*abort_flag) { aborted = true; break; }
+            if (!ptx::mbar_wait(&S.s_full, ph, abort_flag)) bad = true;
+            if (block_any(bad || *abort_flag != 0, 1, kWorkers)) { aborted = true; break; }
             ptx::tc_fence_after();
             float z[32];
             {
@@ -412,17 +442,17 @@ attn_tc_kernel(AttnArgs a) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(u[i]);
             }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&S.s_empty);
-            const float zs = qk_scale * src.scale;
+            const float zs = qk_scale * cur_scale;
             bool over = false;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                z[i] = src.valid ? z[i] * zs : -INFINITY;
+                z[i] = cur_valid ? z[i] * zs : -INFINITY;
                 over |= z[i] > S.m_run[half * 32 + i] + kRescaleThreshold;
             }
-            // the running max moves only when some logit exceeds it by more than 2^8
+            // the running max moves only when some logit exceeds it by more than 2^8.  The max
+            // scratch lives in P_lo, free here: s_full(j) completed after P.V(j-1).
             const bool move = block_any(over, 1, kWorkers);
+            bool rescale = false;
             if (move) {
                 float v[32];
 #pragma unroll
@@ -430,6 +460,7 @@ attn_tc_kernel(AttnArgs a) {
                 warp_transpose_reduce<false>(v, lane);
                 X.red[sub][half * 32 + lane] = v[0];
                 ptx::named_barrier(1, kWorkers);
+                bool moved_here = false;
                 if (wt < kHeads) {
                     const float tmax = fmaxf(fmaxf(X.red[0][wt], X.red[1][wt]), fmaxf(X.red[2][wt], X.red[3][wt]));
                     const float mo = S.m_run[wt];
@@ -437,18 +468,18 @@ attn_tc_kernel(AttnArgs a) {
                     if (tmax > mo + kRescaleThreshold) {
                         S.m_run[wt] = tmax;
                         al = (mo == -INFINITY) ? 0.0f : ptx::ex2(mo - tmax);
-                        if (j > 0 && mo != -INFINITY) S.any_rescale = 1;
+                        moved_here = j > 0 && mo != -INFINITY;
                     }
                     S.alpha[wt] = al;
                 }
-                ptx::named_barrier(1, kWorkers);
+                // barrier for the m_run / alpha writes, and whether any accumulated head moved
+                rescale = block_any(moved_here, 1, kWorkers);
             }
-            const bool rescale = move && S.any_rescale != 0;
             // probabilities (log2 domain)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const float m = S.m_run[half * 32 + i];
-                z[i] = (m == -INFINITY || !src.valid) ? 0.0f : ptx::ex2(z[i] - m);
+                z[i] = (m == -INFINITY || !cur_valid) ? 0.0f : ptx::ex2(z[i] - m);
             }
             // row sums: per key in TMEM, reduced over the keys once at the end
             {
@@ -461,26 +492,17 @@ attn_tc_kernel(AttnArgs a) {
                     u[i] = __float_as_uint((move ? lp * S.alpha[half * 32 + i] : lp) + z[i]);
                 }
                 ptx::tmem_st32(l_addr, u);
-                ptx::tmem_st_wait();
-            }
-            // P.V of the previous tile completed before this tile's S (the tensor pipe runs in
-            // order), so this wait is immediate; it orders the P rewrite and the O^T rescale.
-            if (j > 0) {
-                ptx::mbar_wait(&S.pv_done, ph ^ 1, abort_flag);
-                ptx::named_barrier(1, kWorkers);
-                if (*abort_flag) { aborted = true; break; }
-                ptx::tc_fence_after();
             }
             // P^T line of key t for this half's heads: fp16 high halves to P_hi, low halves
-            // (P - fp16(P)) to P_lo; the max scratch in the P_lo buffer is no longer read
-            ptx::named_barrier(1, kWorkers);
+            // (P - fp16(P)) to P_lo.  P.V(j-1) finished before s_full(j), and the max scratch
+            // in P_lo was last read before the barrier above.
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t hi4[4], lo4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int i = 8 * c + 2 * k;
-                    const float q0 = z[i] * src.scale, q1 = z[i + 1] * src.scale;
+                    const float q0 = z[i] * cur_scale, q1 = z[i + 1] * cur_scale;
                     const __half2 hp = __floats2half2_rn(q0, q1);
                     const float2 back = __half22float2(hp);
                     const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
@@ -491,12 +513,12 @@ attn_tc_kernel(AttnArgs a) {
                 *reinterpret_cast<uint4 *>(sPlo + sw128_off(t, half * 4 + c)) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
             }
             // O^T rescale for heads whose running max moved (columns of this half)
-            if (rescale && j > 0) {
+            if (rescale) {
                 float al[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) al[i] = S.alpha[half * 32 + i];
 #pragma unroll 1
-                for (int mb = 0; mb < 4; ++mb) {
+                for (int mb = 0; mb < kBlocks; ++mb) {
                     uint32_t u[32];
                     const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
                     ptx::tmem_ld32(addr, u);
@@ -505,25 +527,15 @@ attn_tc_kernel(AttnArgs a) {
                     for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * al[i]);
                     ptx::tmem_st32(addr, u);
                 }
-                ptx::tmem_st_wait();
             }
+            ptx::tmem_st_wait();
             ptx::fence_async_smem();
             ptx::tc_fence_before();
-            ptx::named_barrier(1, kWorkers);
-            if (wt == 0) S.any_rescale = 0;
             ptx::mbar_arrive(&S.p_full);
-            // next tile's rows are fetched while the tensor core runs P.V
-            if (j + 1 < ntiles) {
-                src = key_source(a, r, b, x_begin + (j + 1) * kTile + t, x_end, n_sel);
-                prefetch_half(src, half, hr);
-            }
         }
         // ---------------- epilogue ----------------
-        if (!aborted && ntiles > 0) {
-            ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag);
-        }
-        ptx::named_barrier(1, kWorkers);
-        aborted = aborted || *abort_flag != 0;
+        if (!aborted && ntiles > 0 && !ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag)) bad = true;
+        aborted = block_any(aborted || bad || *abort_flag != 0, 1, kWorkers);
         ptx::tc_fence_after();
         // row sums: reduce the per-key partials over this warp's 32 keys, then over the 4
         // sub-partitions
@@ -557,7 +569,7 @@ attn_tc_kernel(AttnArgs a) {
             }
             ptx::named_barrier(1, kWorkers);
 #pragma unroll 1
-            for (int mb = 0; mb < 4; ++mb) {
+            for (int mb = 0; mb < kBlocks; ++mb) {
                 const int c = mb * 128 + t;               // this thread's channel
                 uint32_t u[32];
                 if (ntiles > 0) {
