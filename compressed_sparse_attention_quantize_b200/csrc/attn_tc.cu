@@ -54,7 +54,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int32_t kNoKey = INT32_MIN;
 
 struct Smem {
-    uint64_t v_full[2];                    // channels 0-255 / 256-511 of the tile are written
+    uint64_t v_full[kBlocks];              // 128-channel block mb of the tile is written
     uint64_t v_empty[kBlocks];             // P.V of 128-channel block mb has completed
     uint64_t s_full, p_full, pv_done, drain;
     uint32_t tmem_base;
@@ -213,7 +213,7 @@ CSA2_D bool block_any(bool flag, uint32_t barrier_id, uint32_t threads) {
 
 // The MMA issuer (one thread).  Every MMA sequence is straight-line code: an mbarrier wait or any
 // other memory instruction between two MMAs leaves the tensor pipe idle for a few hundred cycles
-// (measured), so each tile has three waits: the two channel halves of V, then P.
+// (measured), so each tile has five waits: the four 128-channel blocks of V, then P.
 // Kept out of line so that its few live values keep registers of their own.
 __device__ __noinline__ void issue_mmas(uint32_t tmem, uint8_t *sQ, uint8_t *sV, uint8_t *sP, uint8_t *sPlo,
                                         Smem &S, int ntiles, volatile int *abort_flag) {
@@ -232,13 +232,13 @@ __device__ __noinline__ void issue_mmas(uint32_t tmem, uint8_t *sQ, uint8_t *sV,
         // S(j) is issued after P.V(j-1), whose P the softmax warps released before p_full(j-1),
         // and s_full(j) completes only after P.V(j-1) has: no separate S-buffer hand-off.
 #pragma unroll
-        for (int hv = 0; hv < 2; ++hv) {
-            if (!ptx::mbar_wait(&S.v_full[hv], ph, abort_flag)) goto done;
+        for (int mb = 0; mb < kBlocks; ++mb) {
+            if (!ptx::mbar_wait(&S.v_full[mb], ph, abort_flag)) goto done;
 #pragma unroll
-            for (int rl = 0; rl < 4; ++rl)
+            for (int rl = 0; rl < 2; ++rl)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int rg = hv * 4 + rl;
+                    const int rg = mb * 2 + rl;
                     ptx::mma_f16_ss(tmem, s_a0 + (uint64_t)(rg * (kVRegion >> 4) + k * 2),
                                     s_b0 + (uint64_t)(rg * (kQRegion >> 4) + k * 2), idesc_s, (rg | k) != 0);
                 }
@@ -310,7 +310,7 @@ attn_tc_kernel(AttnArgs a) {
 
     // ---------------- setup ----------------
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) ptx::mbar_init(&S.v_full[i], kWorkers);
+        for (int i = 0; i < kBlocks; ++i) ptx::mbar_init(&S.v_full[i], kWorkers);
         for (int i = 0; i < kBlocks; ++i) ptx::mbar_init(&S.v_empty[i], 1);
         ptx::mbar_init(&S.s_full, 1);
         ptx::mbar_init(&S.p_full, kWorkers);
@@ -420,10 +420,8 @@ attn_tc_kernel(AttnArgs a) {
                 uint8_t *dst = sV + rg * kVRegion;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + sw128_off(t, c)) = out[c];
-                if (mb & 1) {
-                    ptx::fence_async_smem();
-                    ptx::mbar_arrive(&S.v_full[mb >> 1]);
-                }
+                ptx::fence_async_smem();
+                ptx::mbar_arrive(&S.v_full[mb]);
             }
             const bool cur_valid = src.valid;
             const float cur_scale = src.scale;

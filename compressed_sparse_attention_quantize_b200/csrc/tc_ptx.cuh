@@ -32,14 +32,17 @@ CSA2_D bool mbar_try(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: gives up after ~2^22 polls (well over a second with the back-off), records
-// CSA2_ERR_TIMEOUT in the device error word and raises the CTA's abort flag.
+// Bounded wait: gives up after 2^22 polls (tenths of a second at least; polls past 2^16 back
+// off with a sleep), records CSA2_ERR_TIMEOUT in the device error word and raises the CTA's
+// abort flag.  The hot waits of the pipelines finish long before the back-off starts: a sleeping
+// waiter would see the phase flip late.
 constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint32_t kSpinBackoff = 1u << 16;
 CSA2_D bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (i > 32) __nanosleep(64);
+        if (i > kSpinBackoff) __nanosleep(64);
     }
     *abort_flag = 1;
     atomicExch(&g_device_error, (int)CSA2_ERR_TIMEOUT);
@@ -51,7 +54,7 @@ CSA2_D bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) 
 CSA2_D bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try(bar, parity)) return true;
-        if (i > 32) __nanosleep(64);
+        if (i > kSpinBackoff) __nanosleep(64);
     }
     atomicExch(&g_device_error, (int)CSA2_ERR_TIMEOUT);
     return false;
