@@ -285,48 +285,72 @@ def breakdown(torch, csa2, runner, steps, flush):
 
 
 def e2e_measure(torch, csa2, runner, steps, warmup, flush):
-    """The metric through csa2_layer_group with host buffers: per step copy every layer's main
-    query (bf16) and indexer query/weights (fp32) from pinned host memory, quantise the indexer
-    queries on the device, run the group, read the last layer's output back."""
+    """The metric through csa2_layer_group with host buffers.  Per step: every layer's main query
+    (bf16) and indexer query/weights (fp32) are copied from pinned host memory on a copy stream,
+    layer by layer (the indexer queries are quantised there too), and each layer of the group
+    waits only for its own inputs (the group's per-layer ready events), so the copies of later
+    layers overlap the work of earlier ones; the last layer's output is read back at the end.
+    Steps do not overlap: the copy stream starts a step after the previous step's work."""
     from compressed_sparse_attention_quantize_b200 import runtime, synth
     wl = runner.wl
+    def pinned_copy(t):
+        # fresh page-locked buffers: copies of tensor.pin_memory() results ran at a third of
+        # the bandwidth of torch.empty(..., pin_memory=True) buffers on the B200 hosts
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
     host = []
     h2d = 0
     for l, m in enumerate(runner.modes):
         ld = runner.layer_data[l]
-        hq = ld["q"].cpu().pin_memory()
+        hq = pinned_copy(ld["q"].cpu())
         e = {"q": hq}
         h2d += hq.numel() * 2
         if m != "U":
             iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
-            e["iq"] = torch.from_numpy(iq).pin_memory()
+            e["iq"] = pinned_copy(torch.from_numpy(iq))
             e["iq_dev"] = torch.empty_like(e["iq"], device=ld["q"].device)
-            e["iw"] = ld["iw"].cpu().pin_memory()
+            e["iw"] = pinned_copy(ld["iw"].cpu())
             h2d += e["iq"].numel() * 4 + e["iw"].numel() * 4
         host.append(e)
     out_last = runner.layer_data[-1]["out"]
-    out_host = torch.empty(out_last.shape, dtype=out_last.dtype).pin_memory()
+    out_host = torch.empty(out_last.shape, dtype=out_last.dtype, pin_memory=True)
     d2h = out_host.numel() * out_host.element_size()
+    cur = torch.cuda.current_stream()
+    copy_stream = torch.cuda.Stream()
+    ready = [torch.cuda.Event() for _ in runner.modes]
+    for ev in ready:
+        ev.record(cur)                       # creates the handles
+    runner.set_layer_events([ev.cuda_event for ev in ready], None)
 
     def step():
-        for l, m in enumerate(runner.modes):
-            ld, e = runner.layer_data[l], host[l]
-            ld["q"].copy_(e["q"], non_blocking=True)
-            if m != "U":
-                e["iq_dev"].copy_(e["iq"], non_blocking=True)
-                ld["iw"].copy_(e["iw"], non_blocking=True)
-                runtime.quantize_fp4_rows(e["iq_dev"], ld["iq_codes"], ld["iq_scales"], 32, 4)
+        copy_stream.wait_stream(cur)
+        with torch.cuda.stream(copy_stream):
+            for l, m in enumerate(runner.modes):
+                ld, e = runner.layer_data[l], host[l]
+                ld["q"].copy_(e["q"], non_blocking=True)
+                if m != "U":
+                    e["iq_dev"].copy_(e["iq"], non_blocking=True)
+                    ld["iw"].copy_(e["iw"], non_blocking=True)
+                    runtime.quantize_fp4_rows(e["iq_dev"], ld["iq_codes"], ld["iq_scales"], 32, 4,
+                                              stream=copy_stream)
+                ready[l].record(copy_stream)
         runner.run()
         out_host.copy_(out_last, non_blocking=True)
 
-    for _ in range(warmup):
-        flush()
-        step()
-    torch.cuda.synchronize()
-    ms = time_steps(torch, step, steps, flush)
+    try:
+        for _ in range(warmup):
+            flush()
+            step()
+        torch.cuda.synchronize()
+        ms = time_steps(torch, step, steps, flush)
+    finally:
+        torch.cuda.synchronize()
+        runner.set_layer_events(None, None)
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": sum(ms) / steps}
+            "ms_per_step": sum(ms) / steps, "overlap": "per-layer input copies on a second stream"}
 
 
 def run_csa2(args, wl):
@@ -346,7 +370,7 @@ def run_csa2(args, wl):
     if rank > 0:
         wl.seed = wl.seed + 1000 * rank          # independent sequences per rank
     hbm_peak, tc_peak, tc_sus, peak_src = _peaks()
-    runner = runtime.GroupRunner(wl, out_dtype=csa2.DTYPE_F32)
+    runner = runtime.GroupRunner(wl, out_dtype=csa2.DTYPE_BF16)
     flush_buf = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device="cuda")
 
     def flush():
@@ -384,7 +408,7 @@ def run_csa2(args, wl):
 
     # per-call breakdown and roofline of the dominant kernel
     bd = breakdown(torch, csa2, runner, max(3, min(args.steps, 10)), flush)
-    ab, af = attn_work(wl, 4)
+    ab, af = attn_work(wl, 2 if runner.out_dtype == csa2.DTYPE_BF16 else 4)
     ib = index_work(wl)
     kernels = {}
     if "sparse_attn" in bd:
@@ -433,7 +457,7 @@ def run_csa2(args, wl):
                 "config": {"workload": wl.name, "batch_per_gpu": wl.B, "ctx_tokens": wl.ctx_tokens[0],
                            "entries_per_seq": wl.n_entries[0], "layers": ",".join(wl.modes),
                            "heads": wl.H, "index_heads": wl.HI, "topk": wl.K, "pool": wl.P,
-                           "swa": 128, "parallelism": f"replicas x{world} (independent sequences)",
+                           "swa": 128, "out": "bf16", "parallelism": f"replicas x{world} (independent sequences)",
                            "l2": "flushed between steps (256 MB write, outside the events)"},
                 "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches), "clocks": clocks}

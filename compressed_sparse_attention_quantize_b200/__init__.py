@@ -66,6 +66,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [
         ("mode", _i32), ("q", _vp), ("iq_codes", _vp), ("iq_scales", _vp), ("iw", _vp),
         ("swa_codes", _vp), ("swa_scale", _vp), ("out", _vp), ("lse", _vp), ("idx_out", _vp),
+        ("ready_event", _vp), ("done_event", _vp),
     ]
 
 

@@ -284,6 +284,10 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     cudaStream_t st = as_stream(stream);
     for (int l = 0; l < n_layers; ++l) {
         const csa2_layer_desc &L = layers[l];
+        if (L.ready_event) {
+            cudaError_t e = cudaStreamWaitEvent(st, reinterpret_cast<cudaEvent_t>(L.ready_event), 0);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
         if (L.mode == CSA2_MODE_FULL) {
             s = csa2_index_topk(CSA2_MODE_FULL, L.iq_codes, L.iq_scales, L.iw, g->B, g->T, g->H_I,
                                 g->k_codes, g->k_code_stride, g->k_scales, g->k_scale_stride,
@@ -309,6 +313,10 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
                              g->swa_len, g->softmax_scale, L.out, g->out_dtype, L.lse, aws,
                              aws_bytes, stream);
         if (s != CSA2_OK) return s;
+        if (L.done_event) {
+            cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(L.done_event), st);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
     }
     return CSA2_OK;
 }

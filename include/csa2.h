@@ -226,6 +226,10 @@ CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t *q, int B, int T, i
  *   REUSE   : takes the preceding layer's selection as is (no indexer work).
  * Every layer then runs csa2_sparse_attn with its own main query and its own window over
  * the shared main KV.  Layers run in order on `stream`.
+ * Per-layer events (optional, cudaEvent_t passed as void*, owned by the caller): the work of
+ * layer l waits on `ready_event` (cudaStreamWaitEvent), e.g. the copy of that layer's query on
+ * another stream, and `done_event` is recorded once layer l's work is queued, e.g. to start
+ * reading its output back while later layers run.  NULL skips either.
  * Rejected (INVALID_ARG): a REUSE or REINDEX layer before any FULL layer; REINDEX with
  * P == 0.
  * ---------------------------------------------------------------------------------- */
@@ -251,6 +255,8 @@ typedef struct csa2_layer_desc {
     void *out;                   /* [B*T][H][D] of out_dtype                           */
     float *lse;                  /* [B*T][H] or NULL                                   */
     int32_t *idx_out;            /* optional copy of this layer's selection [B*T][K]   */
+    void *ready_event;           /* cudaEvent_t or NULL: the layer's kernels wait for it */
+    void *done_event;            /* cudaEvent_t or NULL: recorded after the layer's work */
 } csa2_layer_desc;
 
 CSA2_API csa2_status csa2_layer_group_workspace_size(const csa2_group_desc *g,

@@ -178,6 +178,38 @@ def test_bf16_output():
         assert np.linalg.norm(got - ref) <= 4e-3 * np.linalg.norm(ref)
 
 
+def test_layer_events_same_result():
+    """Per-layer ready/done events (csa2_layer_desc) only order work: the group's outputs with a
+    side stream feeding each layer's query are bit-identical to a plain call."""
+    wl = synth.scaled(synth.workload(2), B=3, n=5000, K=256, P=1200, name="events")
+    r = _run_group(wl)
+    ref = [ld["out"].clone() for ld in r.layer_data]
+    host_q = [ld["q"].cpu().pin_memory() for ld in r.layer_data]
+    for ld in r.layer_data:
+        ld["q"].zero_()
+        ld["out"].zero_()
+    cur = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    ready = [torch.cuda.Event() for _ in r.modes]
+    done = [torch.cuda.Event() for _ in r.modes]
+    for ev in ready + done:
+        ev.record(cur)
+    torch.cuda.synchronize()
+    r.set_layer_events([e.cuda_event for e in ready], [e.cuda_event for e in done])
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):
+        for l, ld in enumerate(r.layer_data):
+            ld["q"].copy_(host_q[l], non_blocking=True)
+            ready[l].record(side)
+    r.run()
+    for l in range(len(r.modes)):
+        done[l].synchronize()
+    torch.cuda.synchronize()
+    r.set_layer_events(None, None)
+    for l, ld in enumerate(r.layer_data):
+        assert torch.equal(ld["out"], ref[l]), l
+
+
 @pytest.mark.parametrize("cfg,rows", [(1, [0, 17, 31]), (2, [0, 15]), (3, [0, 3]), (4, [0, 1000, 4095])])
 def test_full_size_sampled(cfg, rows):
     """Full-size workloads in the bench's launch configuration; sampled rows vs the oracle."""
