@@ -425,9 +425,6 @@ attn_tc_kernel(AttnArgs a) {
             }
             const bool cur_valid = src.valid;
             const float cur_scale = src.scale;
-            // ---- the next tile's rows are requested before the softmax
-            src = source_of(a, r, b, seq_start, e_next);
-            prefetch_part(src, hsel, rp);
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             if (!ptx::mbar_wait(&S.s_full, ph, abort_flag)) bad = true;
             if (block_any(bad || *abort_flag != 0, 1, kWorkers)) { aborted = true; break; }
@@ -530,6 +527,10 @@ attn_tc_kernel(AttnArgs a) {
             ptx::fence_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&S.p_full);
+            // ---- the next tile's rows are requested while the tensor core runs P.V (not
+            //      earlier: live across the softmax they would push its registers into spills)
+            src = source_of(a, r, b, seq_start, e_next);
+            prefetch_part(src, hsel, rp);
         }
         // ---------------- epilogue ----------------
         if (!aborted && ntiles > 0 && !ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag)) bad = true;

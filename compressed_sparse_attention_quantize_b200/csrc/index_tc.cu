@@ -15,8 +15,10 @@
 // Operands in shared memory, K-major without swizzle: a 32-byte row of FP4 codes is two 16-byte
 // planes (elements 0-31 and 32-63), rows 16 bytes apart inside a plane.  D: 128 lanes (keys) x
 // N columns (4 per head, N rounded up to 16) fp32 in TMEM.  Each thread keeps the key rows of
-// the next 4 tiles in flight in registers; a CTA uses 128 TMEM columns and 56 KB of shared
-// memory so at most 4 CTAs share an SM and TMEM allocation never waits.
+// next tiles in flight: for a contiguous key range (Full mode) one thread streams the raw
+// 32-byte rows of the next kStages tiles into a shared-memory ring with bulk copies; for a
+// gathered pool (Reindex) every thread keeps its key rows of the next kDepth tiles in registers.
+// Shared memory is reserved so that TMEM allocation never waits (at most 512 / columns CTAs).
 #include "common.cuh"
 #include "index_api.cuh"
 #include "tc_ptx.cuh"
@@ -28,7 +30,9 @@ constexpr int kTile = 128;
 constexpr int kThreads = 128;
 constexpr int kMaxN = 4 * CSA2_MAX_INDEX_HEADS;      // 64 columns
 constexpr int kTilesPerCta = 8;                      // 1024 keys per CTA
-constexpr int kDepth = 2;                            // tiles of key rows in flight per thread
+constexpr int kDepth = 2;                            // gathered tiles in flight per thread
+constexpr int kStages = 8;                           // contiguous tiles in flight per CTA
+constexpr int kRingBytes = kStages * kTile * 32;     // raw key rows, 32 bytes each
 
 struct Args {
     const uint8_t *q_codes, *q_scales;
@@ -56,6 +60,7 @@ struct __align__(16) Smem {
     float qs[CSA2_MAX_INDEX_HEADS * 4];// query block scales
     float w[CSA2_MAX_INDEX_HEADS];
     uint64_t done, drain;
+    uint64_t full[kStages];            // ring stage s holds its tile's key rows
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -95,9 +100,10 @@ CSA2_D void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t i
         : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 8)
+__global__ void __launch_bounds__(kThreads, 6)
 index_score_tc_kernel(Args a) {
     __shared__ Smem S;
+    extern __shared__ __align__(128) uint8_t ring[];     // kStages x 128 raw key rows (contiguous mode)
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int r = a.row0 + blockIdx.y;
     const int b = r / a.T;
@@ -116,6 +122,7 @@ index_score_tc_kernel(Args a) {
     if (t == 0) {
         ptx::mbar_init(&S.done, 1);
         ptx::mbar_init(&S.drain, 1);
+        for (int i = 0; i < kStages; ++i) ptx::mbar_init(&S.full[i], 1);
         S.abort_flag = 0;
         ptx::fence_async_smem();
     }
@@ -160,76 +167,137 @@ index_score_tc_kernel(Args a) {
     volatile int *abort_flag = &S.abort_flag;
     const int64_t sbase = a.seq_start[b];
 
-    // key rows of tile i for this thread
-    auto key_row = [&](int i, uint4 &c0, uint4 &c1, uint32_t &sc, bool &valid) {
-        const int64_t j = j0 + (int64_t)i * kTile + t;
-        valid = j < n;
-        c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
-        sc = 0u;
-        if (valid) {
-            const int64_t e = sbase + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
-            const uint4 *kc = reinterpret_cast<const uint4 *>(a.k_codes + e * a.k_code_stride);
-            c0 = __ldg(kc);
-            c1 = __ldg(kc + 1);
-            const uint8_t *ks = a.k_scales + e * a.k_scale_stride;
-            sc = (uint32_t)__ldg(ks) | ((uint32_t)__ldg(ks + 1) << 8) | ((uint32_t)__ldg(ks + 2) << 16) |
-                 ((uint32_t)__ldg(ks + 3) << 24);
-        }
-    };
-
-    uint4 c0[kDepth], c1[kDepth];
-    uint32_t sc[kDepth];
-    bool valid[kDepth];
-#pragma unroll
-    for (int k = 0; k < kDepth; ++k) key_row(k, c0[k], c1[k], sc[k], valid[k]);
     const uint64_t adesc = sdesc_noswizzle(ptx::smem_u32(S.a), kTile * 16, 128);
-    bool aborted = false;
-    for (int i0 = 0; i0 < ntiles && !aborted; i0 += kDepth) {
-#pragma unroll
-        for (int k = 0; k < kDepth; ++k) {
-            const int i = i0 + k;
-            if (i >= ntiles) break;
-            // stage tile i: the previous MMA has completed and every thread has read its D
-            *reinterpret_cast<uint4 *>(S.a + t * 16) = c0[k];
-            *reinterpret_cast<uint4 *>(S.a + kTile * 16 + t * 16) = c1[k];
-            ptx::fence_async_smem();
-            ptx::tc_fence_before();
-            __syncthreads();
-            if (t == 0) {
-                ptx::tc_fence_after();
-                mma_mxf4(tmem, adesc, bdesc, idesc, sf, sf);
-                ptx::mma_commit(&S.done);
-            }
-            const uint32_t sc_this = sc[k];
-            const bool valid_this = valid[k];
-            if (i + kDepth < ntiles) key_row(i + kDepth, c0[k], c1[k], sc[k], valid[k]);
-            ptx::mbar_wait(&S.done, i & 1, abort_flag);
-            if (__syncthreads_or(*abort_flag != 0)) { aborted = true; break; }
+
+    // One tile: stage this thread's key row in the two 16-byte planes, one MMA, then the
+    // fixed-order epilogue.  Returns false when the CTA gives up (collective).
+    auto run_tile = [&](int i, const uint4 &k0, const uint4 &k1, uint32_t sc_this, bool valid_this) -> bool {
+        *reinterpret_cast<uint4 *>(S.a + t * 16) = k0;
+        *reinterpret_cast<uint4 *>(S.a + kTile * 16 + t * 16) = k1;
+        ptx::fence_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+        if (t == 0) {
             ptx::tc_fence_after();
-            float sk[4];
+            mma_mxf4(tmem, adesc, bdesc, idesc, sf, sf);
+            ptx::mma_commit(&S.done);
+        }
+        ptx::mbar_wait(&S.done, i & 1, abort_flag);
+        if (__syncthreads_or(*abort_flag != 0)) return false;
+        ptx::tc_fence_after();
+        float sk[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
-            float acc = 0.0f;
-            for (int hb = 0; hb * 8 < H; ++hb) {
-                uint32_t u[32];
-                ptx::tmem_ld32(lane_addr + hb * 32, u);
-                ptx::tmem_ld_wait();
+        for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
+        float acc = 0.0f;
+        for (int hb = 0; hb * 8 < H; ++hb) {
+            uint32_t u[32];
+            ptx::tmem_ld32(lane_addr + hb * 32, u);
+            ptx::tmem_ld_wait();
 #pragma unroll
-                for (int hh = 0; hh < 8; ++hh) {
-                    const int h = hb * 8 + hh;
-                    if (h < H) {
-                        float p[4];
+            for (int hh = 0; hh < 8; ++hh) {
+                const int h = hb * 8 + hh;
+                if (h < H) {
+                    float p[4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[h * 4 + q], sk[q]));
-                        const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
-                        const float rl = dot > 0.0f ? dot : 0.0f;
-                        acc = __fadd_rn(acc, __fmul_rn(S.w[h], rl));
-                    }
+                    for (int q = 0; q < 4; ++q)
+                        p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[h * 4 + q], sk[q]));
+                    const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
+                    const float rl = dot > 0.0f ? dot : 0.0f;
+                    acc = __fadd_rn(acc, __fmul_rn(S.w[h], rl));
                 }
             }
-            if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
-            if (valid_this) a.scores[(int64_t)blockIdx.y * a.score_stride + j0 + (int64_t)i * kTile + t] = acc;
+        }
+        if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
+        if (valid_this) a.scores[(int64_t)blockIdx.y * a.score_stride + j0 + (int64_t)i * kTile + t] = acc;
+        return true;
+    };
+
+    // the four E4M3 block scales of key j (0 past the end)
+    auto scale_of = [&](int i) -> uint32_t {
+        const int64_t j = j0 + (int64_t)i * kTile + t;
+        if (i >= ntiles || j >= n) return 0u;
+        const int64_t e = sbase + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
+        const uint8_t *ks = a.k_scales + e * a.k_scale_stride;
+        if ((a.k_scale_stride & 3) == 0) return __ldg(reinterpret_cast<const uint32_t *>(ks));
+        return (uint32_t)__ldg(ks) | ((uint32_t)__ldg(ks + 1) << 8) | ((uint32_t)__ldg(ks + 2) << 16) |
+               ((uint32_t)__ldg(ks + 3) << 24);
+    };
+
+    bool aborted = false;
+    const bool contiguous = a.pool == nullptr && a.k_code_stride == 32;
+    if (contiguous) {
+        // ---- Full mode: the CTA's keys are consecutive rows; thread 0 keeps kStages tiles of raw
+        //      rows in flight with bulk copies (only the rows that exist are copied)
+        const uint8_t *src0 = a.k_codes + (sbase + j0) * 32;
+        auto issue = [&](int i) {
+            const int st = i % kStages;
+            const int64_t jt = (int64_t)i * kTile;
+            const uint32_t bytes = (uint32_t)min((int64_t)kTile, n - j0 - jt) * 32u;
+            ptx::mbar_arrive_expect_tx(&S.full[st], bytes);
+            ptx::bulk_load_g2s(ring + st * kTile * 32, src0 + jt * 32, bytes, &S.full[st]);
+        };
+        int issued = 0;
+        if (t == 0)
+            for (; issued < kStages && issued < ntiles; ++issued) issue(issued);
+        uint32_t s0 = scale_of(0), s1 = scale_of(1), s2 = scale_of(2);
+        int i = 0;
+        for (; i < ntiles; ++i) {
+            const int st = i % kStages;
+            ptx::mbar_wait(&S.full[st], (uint32_t)(i / kStages) & 1u, abort_flag);   // a miss aborts below
+            const bool valid_this = j0 + (int64_t)i * kTile + t < n;
+            uint4 k0 = make_uint4(0u, 0u, 0u, 0u), k1 = k0;
+            if (valid_this) {
+                const uint4 *row = reinterpret_cast<const uint4 *>(ring + st * kTile * 32 + t * 32);
+                k0 = row[0];
+                k1 = row[1];
+            }
+            const uint32_t sc_this = s0;
+            s0 = s1;
+            s1 = s2;
+            s2 = scale_of(i + 3);
+            if (!run_tile(i, k0, k1, sc_this, valid_this)) { aborted = true; break; }
+            // every thread has read stage st (run_tile synchronised after staging)
+            if (t == 0 && issued < ntiles) issue(issued++);
+        }
+        if (aborted && t == 0) {       // let the copies still in flight land before exiting
+            for (int k = i; k < issued; ++k)
+                ptx::mbar_wait_drain(&S.full[k % kStages], (uint32_t)(k / kStages) & 1u);
+        }
+    } else {
+        // ---- gathered keys (Reindex pool) or strided rows: kDepth tiles in registers per thread
+        auto key_row = [&](int i, uint4 &c0, uint4 &c1, bool &valid) {
+            const int64_t j = j0 + (int64_t)i * kTile + t;
+            valid = j < n;
+            c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
+            if (valid) {
+                const int64_t e = sbase + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
+                const uint4 *kc = reinterpret_cast<const uint4 *>(a.k_codes + e * a.k_code_stride);
+                c0 = __ldg(kc);
+                c1 = __ldg(kc + 1);
+            }
+        };
+        uint4 c0[kDepth], c1[kDepth];
+        uint32_t sc[kDepth];
+        bool valid[kDepth];
+#pragma unroll
+        for (int k = 0; k < kDepth; ++k) {
+            key_row(k, c0[k], c1[k], valid[k]);
+            sc[k] = scale_of(k);
+        }
+        for (int i0 = 0; i0 < ntiles && !aborted; i0 += kDepth) {
+#pragma unroll
+            for (int k = 0; k < kDepth; ++k) {
+                const int i = i0 + k;
+                if (i >= ntiles) break;
+                const uint4 k0 = c0[k], k1 = c1[k];
+                const uint32_t sc_this = sc[k];
+                const bool valid_this = valid[k];
+                if (i + kDepth < ntiles) {
+                    key_row(i + kDepth, c0[k], c1[k], valid[k]);
+                    sc[k] = scale_of(i + kDepth);
+                }
+                if (!run_tile(i, k0, k1, sc_this, valid_this)) { aborted = true; break; }
+            }
         }
     }
     if (aborted && t == 0) {           // drain the tensor pipe before TMEM is released
@@ -270,7 +338,8 @@ cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, flo
     // reserve shared memory so that at most 512/cols CTAs are resident on an SM
     const int per_sm = 512 / (int)cols;
     const int smem_total = (227 * 1024) / per_sm - 1024;
-    const int dyn = smem_total - (int)sizeof(itc::Smem);
+    // (and at least the bulk-copy ring of the contiguous path)
+    const int dyn = max(smem_total - (int)sizeof(itc::Smem), itc::kRingBytes);
     static int attr_dyn = -1;
     if (attr_dyn != dyn) {
         cudaError_t e = cudaFuncSetAttribute(itc::index_score_tc_kernel,

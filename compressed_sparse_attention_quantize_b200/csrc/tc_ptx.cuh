@@ -60,6 +60,20 @@ CSA2_D bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     return false;
 }
 
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global memory
+// into this CTA's shared memory; completes `bytes` transactions on the mbarrier `bar`.
+CSA2_D void bulk_load_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// Arrive once and add `bytes` to the transaction count the current phase waits for.
+CSA2_D void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------------------
 // fences
 // ---------------------------------------------------------------------------------------
