@@ -51,6 +51,13 @@ def _peaks():
 # ------------------------------------------------------------------------------------------
 # algorithmic work per call (bytes that must move; flops of the contraction)
 # ------------------------------------------------------------------------------------------
+# DRAM bytes (read + write) of one attn_tc_kernel launch on this workload, from an ncu capture of
+# the current kernel (dram__bytes_read.sum + dram__bytes_write.sum); set to None whenever the
+# kernel changes until it is captured again.
+ATTN_TRAFFIC_BYTES = 29_122_560 + 61_696
+ATTN_TRAFFIC_SOURCE = "ncu --set full capture, profiles/attn_tc_decode128k_b32.md"
+
+
 def attn_work(wl, out_bytes):
     """Bytes and flops of one csa2_sparse_attn call over the workload."""
     from compressed_sparse_attention_quantize_b200 import synth
@@ -430,7 +437,7 @@ def run_csa2(args, wl):
         k = kernels[dom]
         roof = {"kernel": "csa2_sparse_attn", "bound": "tensor", "achieved": k["achieved_tflops"],
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": k["achieved_tflops"] / tc_peak,
-                "traffic": None, "peak_source": f"{peak_src} bf16_tflops (fp16 MMA runs at the same rate)",
+                "traffic": ATTN_TRAFFIC_BYTES, "traffic_source": ATTN_TRAFFIC_SOURCE, "peak_source": f"{peak_src} bf16_tflops (fp16 MMA runs at the same rate)",
                 "hbm_achieved_gbs": k["achieved_gbs"], "hbm_frac": k["achieved_gbs"] / hbm_peak}
     elif dom == "index_topk":
         k = kernels[dom]

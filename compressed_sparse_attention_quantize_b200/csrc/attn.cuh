@@ -30,9 +30,6 @@ struct AttnArgs {
 // Floats of one tensor-core split partial: running max[64], row sum[64], O[64][512].
 constexpr int kPartialFloats = 2 * 64 + 64 * 512;
 
-cudaError_t launch_attn_simt(AttnArgs a, cudaStream_t st);
-size_t simt_workspace_bytes(int rows, int H, int K);
-
 cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st);
 size_t tc_workspace_bytes(int rows, int H, int K);
 

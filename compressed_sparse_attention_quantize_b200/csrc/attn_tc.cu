@@ -607,36 +607,82 @@ attn_tc_kernel(AttnArgs a) {
     }
 }
 
-// Merge split partials (log2-domain maxima): one CTA of 128 threads per (row, head).
-__global__ void attn_tc_merge_kernel(AttnArgs a) {
+// Merge split partials (log2-domain maxima): one CTA of 128 threads per (row, head).  Warp 0
+// turns the splits' (m, l) into weights exp2(m - M) (one split per lane, up to 64 splits), then
+// every thread adds its 4 channels of the splits in split order with independent loads.
+constexpr int kMaxMergeSplits = 64;
+static_assert((CSA2_MAX_TOPK + CSA2_SWA_WINDOW + kTile - 1) / kTile <= kMaxMergeSplits, "splits <= tiles");
+
+__global__ void __launch_bounds__(128) attn_tc_merge_kernel(AttnArgs a) {
+    __shared__ float fw[kMaxMergeSplits];
+    __shared__ float inv_total;
     const int r = blockIdx.x, h = blockIdx.y;
     const int hg = h / kHeads, hl = h % kHeads;
     const float *base = a.partials + ((int64_t)r * a.hgroups + hg) * a.splits * kPartialFloats;
-    float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, base[s * kPartialFloats + hl]);
-    float L = 0.0f;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < a.splits; ++s) {
-        const float *p = base + s * kPartialFloats;
-        const float ls = p[kHeads + hl];
-        if (!(ls > 0.0f)) continue;
-        const float f = exp2f(p[hl] - M);
-        L += ls * f;
-        const float4 o = *reinterpret_cast<const float4 *>(p + 2 * kHeads + hl * kLatent + threadIdx.x * 4);
-        acc[0] += o.x * f; acc[1] += o.y * f; acc[2] += o.z * f; acc[3] += o.w * f;
+    const int ns = min(a.splits, kMaxMergeSplits);
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        float m[2], l[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int sidx = lane + 32 * k;
+            m[k] = sidx < ns ? base[sidx * kPartialFloats + hl] : -INFINITY;
+            l[k] = sidx < ns ? base[sidx * kPartialFloats + kHeads + hl] : 0.0f;
+        }
+        float M = fmaxf(m[0], m[1]);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float f[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) f[k] = (l[k] > 0.0f) ? exp2f(m[k] - M) : 0.0f;
+        // L in split order: gather the terms to lane 0 order-preservingly through shared memory
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            if (lane + 32 * k < ns) fw[lane + 32 * k] = f[k];
+        __syncwarp();
+        if (lane == 0) {
+            float L = 0.0f;
+            for (int sidx = 0; sidx < ns; ++sidx) {
+                const float ls = base[sidx * kPartialFloats + kHeads + hl];
+                if (ls > 0.0f) L += ls * fw[sidx];
+            }
+            inv_total = L > 0.0f ? 1.0f / L : 0.0f;
+            if (a.lse) a.lse[(int64_t)r * a.H + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        }
     }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float *o = base + 2 * kHeads + hl * kLatent + threadIdx.x * 4;
+    int sidx = 0;
+    for (; sidx + 4 <= ns; sidx += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = *reinterpret_cast<const float4 *>(o + (int64_t)(sidx + k) * kPartialFloats);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float f = fw[sidx + k];
+            if (f != 0.0f) {
+                acc[0] += v[k].x * f; acc[1] += v[k].y * f; acc[2] += v[k].z * f; acc[3] += v[k].w * f;
+            }
+        }
+    }
+    for (; sidx < ns; ++sidx) {
+        const float f = fw[sidx];
+        if (f != 0.0f) {
+            const float4 v = *reinterpret_cast<const float4 *>(o + (int64_t)sidx * kPartialFloats);
+            acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
+        }
+    }
+    const float inv = inv_total;
     const int64_t oi = ((int64_t)r * a.H + h) * kLatent + threadIdx.x * 4;
     if (a.out_dtype == CSA2_DTYPE_F32) {
         *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + oi) =
             make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
     } else {
-        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.out) + oi;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) o[i] = __float2bfloat16_rn(acc[i] * inv);
+        __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(reinterpret_cast<__nv_bfloat16 *>(a.out) + oi);
+        o2[0] = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+        o2[1] = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
     }
-    if (threadIdx.x == 0 && a.lse)
-        a.lse[(int64_t)r * a.H + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
 }  // namespace tc

@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 6)
 index_score_tc_kernel(Args a) {
     __shared__ Smem S;
     extern __shared__ __align__(128) uint8_t ring[];     // kStages x 128 raw key rows (contiguous mode)
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int t = threadIdx.x, warp = t >> 5;
     const int r = a.row0 + blockIdx.y;
     const int b = r / a.T;
     const int64_t n = min(candidates(a, r), a.score_stride);

@@ -8,21 +8,17 @@
 // [A] page "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径", section
 //   "压缩吸收注意力（二代）": the first layer picks 2048 blocks and keeps a candidate pool.
 //
-// Score I[r,j] = sum_h w_h * relu(q_h . k_j) in fp32.  Per 16-channel block the partial is
-// exact in any order (all terms are multiples of s_q*s_k/4 and the block needs <= 20
-// significant bits), so it is accumulated with fma; the four blocks and the heads are then
-// added in a fixed left-to-right order with explicitly rounded adds and multiplies.  This
-// reproduces the reference order bit for bit, so the selected sets match exactly.
-//
-// Selection is a 4-pass, 8-bit radix select on order-preserving keys, then one compaction
-// pass in entry order: entries above the threshold key, plus the lowest-indexed entries
-// equal to it, written in ascending index order.
+// Scores come from the tensor-core kernel in index_tc.cu (bit-identical to the reference's
+// fixed fp32 order) into a bounded row-chunked buffer; selection runs on 8-CTA clusters
+// (topk_cluster.cu) or, for rows longer than a cluster holds, on one CTA per row here: a 4-pass,
+// 8-bit radix select on order-preserving keys, then one compaction pass in entry order
+// (entries above the threshold key, plus the lowest-indexed entries equal to it, written in
+// ascending index order).
 #include "common.cuh"
 #include "index_api.cuh"
 
 namespace csa2 {
 
-constexpr int kScoreThreads = 256;
 constexpr int kSelectThreads = 1024;
 
 struct ScoreArgs {
@@ -57,55 +53,6 @@ CSA2_D int64_t row_candidates(const ScoreArgs &a, int r) {
         if (n < 0) n = 0;
     }
     return n;
-}
-
-__global__ void __launch_bounds__(kScoreThreads)
-index_score_kernel(ScoreArgs a) {
-    const int r = a.row0 + blockIdx.y;
-    const int b = r / a.T;
-    __shared__ float qv[CSA2_MAX_INDEX_HEADS * 64];
-    __shared__ float wv[CSA2_MAX_INDEX_HEADS];
-    for (int i = threadIdx.x; i < a.H * 64; i += blockDim.x) {
-        const int h = i >> 6, c = i & 63;
-        const uint8_t byte = a.q_codes[((int64_t)r * a.H + h) * 32 + (c >> 1)];
-        const uint32_t code = (c & 1) ? (byte >> 4) : (byte & 15u);
-        qv[i] = e2m1_to_f32(code) * e4m3_to_f32(a.q_scales[((int64_t)r * a.H + h) * 4 + (c >> 4)]);
-    }
-    for (int i = threadIdx.x; i < a.H; i += blockDim.x) wv[i] = a.w[(int64_t)r * a.H + i];
-    __syncthreads();
-
-    const int64_t n = row_candidates(a, r);
-    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= n || j >= a.score_stride) return;         // score_stride == max_n bounds the row
-    const int64_t e = a.seq_start[b] + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
-    const uint4 *kc = reinterpret_cast<const uint4 *>(a.k_codes + e * a.k_code_stride);
-    const uint4 c0 = __ldg(kc), c1 = __ldg(kc + 1);
-    const uint8_t *ksp = a.k_scales + e * a.k_scale_stride;
-    float ks[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) ks[i] = e4m3_to_f32(__ldg(ksp + i));
-    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    float kv[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-        kv[c] = e2m1_to_f32((words[c >> 3] >> ((c & 7) * 4)) & 15u) * ks[c >> 4];
-
-    float acc = 0.0f;
-    for (int h = 0; h < a.H; ++h) {
-        float p[4];
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-            float s = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) s = fmaf(qv[h * 64 + blk * 16 + i], kv[blk * 16 + i], s);
-            p[blk] = s;                                        // exact
-        }
-        const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
-        const float rl = dot > 0.0f ? dot : 0.0f;
-        acc = __fadd_rn(acc, __fmul_rn(wv[h], rl));
-    }
-    if (acc == 0.0f) acc = 0.0f;                               // -0 -> +0
-    a.scores[(int64_t)blockIdx.y * a.score_stride + j] = acc;
 }
 
 // ---------------------------------------------------------------------------------------

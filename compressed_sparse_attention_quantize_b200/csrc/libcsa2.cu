@@ -3,7 +3,6 @@
 #include "index_topk.cu"
 #include "index_tc.cu"
 #include "topk_cluster.cu"
-#include "attn_simt.cu"
 #include "attn_tc.cu"
 #include "attn_dispatch.cu"
 #include "api.cu"
