@@ -67,6 +67,9 @@ def lib():
         L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
         L.oracle_quantize_fp4.restype = None
         L.oracle_quantize_fp4.argtypes = [f32p, ctypes.c_int64, ctypes.c_int, u8p, u8p]
+        L.oracle_compress_fp4.restype = None
+        L.oracle_compress_fp4.argtypes = [f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_void_p, u8p, u8p]
         L.oracle_dequantize_fp4.restype = None
         L.oracle_dequantize_fp4.argtypes = [u8p, u8p, ctypes.c_int64, ctypes.c_int, f64p]
         L.oracle_quantize_fp8_token.restype = None
@@ -127,6 +130,28 @@ def quantize_fp4(x: np.ndarray):
     codes = np.empty((rows, dim // 2), np.uint8)
     scales = np.empty((rows, dim // 16), np.uint8)
     lib().oracle_quantize_fp4(x, rows, dim, codes, scales)
+    return codes, scales
+
+
+def compress_fp4(x: np.ndarray, ratio: int, w: np.ndarray = None):
+    """[B: CSA2：三层压缩一次吃满] every `ratio` tokens -> one entry, as the weighted sum
+    sum_i w[e, i] * x[ratio*e + i] in fp32 (token order, no fused multiply-add; w=None is the
+    mean), then FP4-quantised like quantize_fp4.
+
+    x: float32 [entries*ratio, dim]; w: float32 [entries, ratio] or None.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    tokens, dim = x.shape
+    assert dim % 16 == 0 and tokens % ratio == 0
+    entries = tokens // ratio
+    wp = None
+    if w is not None:
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        assert w.shape == (entries, ratio)
+        wp = w.ctypes.data
+    codes = np.empty((entries, dim // 2), np.uint8)
+    scales = np.empty((entries, dim // 16), np.uint8)
+    lib().oracle_compress_fp4(x, entries, ratio, dim, wp, codes, scales)
     return codes, scales
 
 

@@ -148,6 +148,35 @@ void oracle_quantize_fp4(const float *x, int64_t rows, int dim,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Sequence compressor + quantise-on-write.  [B §CSA2：三层压缩一次吃满]:   */
+/* every m tokens become one entry (V4's CSA compresses along the sequence; */
+/* its weights are learned and not on the pages).  With caller-supplied     */
+/* per-token weights w[e][i], entry e = sum_{i<m} w[e][i] * x[m e + i]:      */
+/* fp32, tokens in order, each product and each sum rounded once (no fused  */
+/* multiply-add).  w == NULL means the plain mean, w = 1/m.  The entry then */
+/* goes through the FP4 quantiser above.                                    */
+/* ------------------------------------------------------------------------ */
+void oracle_compress_fp4(const float *x, int64_t entries, int ratio, int dim,
+                         const float *w, uint8_t *codes, uint8_t *scales)
+{
+    float *row = (float *)malloc(sizeof(float) * (size_t)dim);
+    const float mean_w = 1.0f / (float)ratio;
+    for (int64_t e = 0; e < entries; ++e) {
+        for (int c = 0; c < dim; ++c) {
+            float acc = 0.0f;
+            for (int i = 0; i < ratio; ++i) {
+                const float wi = w ? w[e * ratio + i] : mean_w;
+                const float prod = wi * x[(e * ratio + i) * (int64_t)dim + c];
+                acc = (i == 0) ? prod : acc + prod;
+            }
+            row[c] = acc;
+        }
+        oracle_quantize_fp4(row, 1, dim, codes + e * (dim / 2), scales + e * (dim / 16));
+    }
+    free(row);
+}
+
 /* Dequantised FP4 value of channel c of one row (exact in fp64 and fp32). */
 static double fp4_value(const uint8_t *codes, const uint8_t *scales, int c)
 {
