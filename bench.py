@@ -383,17 +383,24 @@ def run_csa2(args, wl):
     def flush():
         flush_buf.fill_(1)
 
+    # the timed step replays the whole layer group as one CUDA graph (--eager: one C call per step)
+    step_fn = runner.run
+    graph_kernels = 0
+    if not args.eager:
+        graph_kernels = runner.capture()
+        step_fn = runner.replay
     for _ in range(args.warmup):
         flush()
-        runner.run()
+        step_fn()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = csa2.csa2_launch_count()
     with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clk:
-        ms = time_steps(torch, runner.run, args.steps, flush)
-    launches = csa2.csa2_launch_count() - launches0
+        ms = time_steps(torch, step_fn, args.steps, flush)
+    # graph replays do not pass through the library's launch counter: count the graph's kernels
+    launches = csa2.csa2_launch_count() - launches0 + graph_kernels * args.steps
     clocks = clk.summary()
     total_ms = sum(ms)
     if world > 1:
@@ -464,7 +471,8 @@ def run_csa2(args, wl):
                 "config": {"workload": wl.name, "batch_per_gpu": wl.B, "ctx_tokens": wl.ctx_tokens[0],
                            "entries_per_seq": wl.n_entries[0], "layers": ",".join(wl.modes),
                            "heads": wl.H, "index_heads": wl.HI, "topk": wl.K, "pool": wl.P,
-                           "swa": 128, "out": "bf16", "parallelism": f"replicas x{world} (independent sequences)",
+                           "swa": 128, "out": "bf16", "step": "eager" if args.eager else "cuda graph",
+                           "parallelism": f"replicas x{world} (independent sequences)",
                            "l2": "flushed between steps (256 MB write, outside the events)"},
                 "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches), "clocks": clocks}
@@ -482,6 +490,8 @@ def main():
     ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time one csa2_layer_group call per step "
+                    "instead of replaying it as a CUDA graph")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only (no breakdown, e2e or CPU baseline): for profiler captures")
     ap.add_argument("--entries", type=int, default=0,

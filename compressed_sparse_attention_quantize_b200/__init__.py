@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 
 __all__ = [
     "CSA2Error", "lib", "library_path",
-    "csa2_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
+    "csa2_quantize_kv", "csa2_compress_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
     "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
@@ -89,6 +89,9 @@ def lib():
     L.csa2_version.argtypes = []
     L.csa2_quantize_kv.restype = _i32
     L.csa2_quantize_kv.argtypes = [_i32, _vp, _i32, _i64, _i32, _i64, _vp, _i64, _vp, _i64, _vp, _vp]
+    L.csa2_compress_quantize_kv.restype = _i32
+    L.csa2_compress_quantize_kv.argtypes = [_vp, _i32, _i64, _i32, _i32, _i64, _vp, _i64, _vp, _i64,
+                                            _vp, _i64, _vp, _vp]
     L.csa2_index_topk_workspace_size.restype = _i32
     L.csa2_index_topk_workspace_size.argtypes = [_i32, _i32, _i64, _i32, _i32, ctypes.POINTER(_sz)]
     L.csa2_index_topk.restype = _i32
@@ -161,6 +164,13 @@ def csa2_quantize_kv(fmt, x, x_dtype, rows, dim, x_stride, codes, code_stride, s
                      dst_rows=None, stream=None) -> None:
     _check(lib().csa2_quantize_kv(fmt, _ptr(x), x_dtype, rows, dim, x_stride, _ptr(codes), code_stride,
                                   _ptr(scales), scale_stride, _ptr(dst_rows), _stream(stream)))
+
+
+def csa2_compress_quantize_kv(x, x_dtype, entries, ratio, dim, x_stride, w, w_stride, codes,
+                              code_stride, scales, scale_stride, dst_rows=None, stream=None) -> None:
+    _check(lib().csa2_compress_quantize_kv(_ptr(x), x_dtype, entries, ratio, dim, x_stride, _ptr(w),
+                                           w_stride, _ptr(codes), code_stride, _ptr(scales),
+                                           scale_stride, _ptr(dst_rows), _stream(stream)))
 
 
 def csa2_index_topk_workspace_size(mode, rows, max_n, K, P) -> int:

@@ -8,6 +8,8 @@
 #include "attn.cuh"
 
 namespace csa2 {
+cudaError_t launch_compress_fp4(const void *, int, int64_t, int, int, int64_t, const float *, int64_t,
+                                uint8_t *, int64_t, uint8_t *, int64_t, const int64_t *, cudaStream_t);
 cudaError_t launch_quant_fp4(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
                              uint8_t *, int64_t, const int64_t *, cudaStream_t);
 cudaError_t launch_quant_fp8_token(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
@@ -109,7 +111,7 @@ const char *csa2_status_string(csa2_status s) {
     return "CSA2: unknown status";
 }
 
-int csa2_version(void) { return 1; }
+int csa2_version(void) { return 2; }
 
 const char *csa2_last_error_string(void) { return t_last_error; }
 
@@ -134,6 +136,21 @@ csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, 
     return cuda_status(launch_quant_fp8_token(x, x_dtype, rows, dim, x_stride, codes, code_stride,
                                               (uint8_t *)scales, scale_stride, dst_rows,
                                               as_stream(stream)));
+}
+
+csa2_status csa2_compress_quantize_kv(const void *x, int x_dtype, int64_t entries, int ratio, int dim,
+                                      int64_t x_stride, const float *w, int64_t w_stride,
+                                      uint8_t *codes, int64_t code_stride, uint8_t *scales,
+                                      int64_t scale_stride, const int64_t *dst_rows, void *stream) {
+    if (x_dtype != CSA2_DTYPE_F32 && x_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
+    if (entries == 0) return CSA2_OK;
+    if (entries < 0 || ratio < 1 || ratio > CSA2_MAX_COMPRESS_RATIO || dim <= 0 || (dim % 16) ||
+        dim > 65536 || x_stride < dim)
+        return CSA2_ERR_SHAPE;
+    if (!x || !codes || !scales) return CSA2_ERR_INVALID_ARG;
+    if ((w && w_stride < ratio) || code_stride < dim / 2 || scale_stride < dim / 16) return CSA2_ERR_SHAPE;
+    return cuda_status(launch_compress_fp4(x, x_dtype, entries, ratio, dim, x_stride, w, w_stride, codes,
+                                           code_stride, scales, scale_stride, dst_rows, as_stream(stream)));
 }
 
 csa2_status csa2_index_topk_workspace_size(int mode, int rows, int64_t max_n, int K, int P,

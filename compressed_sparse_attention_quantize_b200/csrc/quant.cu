@@ -24,6 +24,32 @@ CSA2_D float load_as_f32<float>(const float *p) { return __ldg(p); }
 template <>
 CSA2_D float load_as_f32<uint16_t>(const uint16_t *p) { return bf16_bits_to_f32(__ldg(p)); }
 
+// FP4 quantisation of one 16-channel block: 8 code bytes at cd, one E4M3 scale at *sd.
+CSA2_D void quantize_block16(const float (&v)[16], uint8_t *cd, uint8_t *sd) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const uint32_t sc = e4m3_code_mag_rne(__fdiv_rn(amax, 6.0f));
+    const float s = e4m3_to_f32(sc);
+    uint32_t packed[2] = {0u, 0u};
+    if (s != 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float q = __fdiv_rn(fabsf(v[i]), s);
+            uint32_t c = e2m1_code_mag_rne(q) | (signbit(v[i]) ? 8u : 0u);
+            packed[i >> 3] |= c << ((i & 7) * 4);
+        }
+    }
+    // 8 code bytes; alignment of cd is only guaranteed to 1 byte in general
+    if ((((uintptr_t)cd) & 7u) == 0) {
+        *reinterpret_cast<uint2 *>(cd) = make_uint2(packed[0], packed[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cd[i] = (uint8_t)(packed[i >> 2] >> ((i & 3) * 8));
+    }
+    *sd = (uint8_t)sc;
+}
+
 // One thread per 16-channel block.
 template <typename T>
 __global__ void quant_fp4_kernel(const T *__restrict__ x, int64_t rows, int dim, int64_t x_stride,
@@ -38,33 +64,42 @@ __global__ void quant_fp4_kernel(const T *__restrict__ x, int64_t rows, int dim,
         const int b = (int)(t - r * nblk);
         const T *xr = x + r * x_stride + b * 16;
         float v[16];
-        float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            v[i] = load_as_f32<T>(xr + i);
-            amax = fmaxf(amax, fabsf(v[i]));
-        }
-        const uint32_t sc = e4m3_code_mag_rne(__fdiv_rn(amax, 6.0f));
-        const float s = e4m3_to_f32(sc);
-        uint32_t packed[2] = {0u, 0u};
-        if (s != 0.0f) {
+        for (int i = 0; i < 16; ++i) v[i] = load_as_f32<T>(xr + i);
+        const int64_t d = dst_rows ? dst_rows[r] : r;
+        quantize_block16(v, codes + d * code_stride + b * 8, scales + d * scale_stride + b);
+    }
+}
+
+// Sequence compressor + quantise-on-write ([B] section "CSA2：三层压缩一次吃满": every m tokens
+// become one entry).  Entry e = sum_k w[e][k] * x[m*e + k] in fp32, tokens in order, every
+// product and sum rounded once (no fused multiply-add); w == NULL is the mean (w = 1/m).
+// One thread per (entry, 16-channel block).
+template <typename T>
+__global__ void compress_fp4_kernel(const T *__restrict__ x, int64_t entries, int ratio, int dim,
+                                    int64_t x_stride, const float *__restrict__ w, int64_t w_stride,
+                                    uint8_t *__restrict__ codes, int64_t code_stride,
+                                    uint8_t *__restrict__ scales, int64_t scale_stride,
+                                    const int64_t *__restrict__ dst_rows) {
+    const int nblk = dim >> 4;
+    const int64_t total = entries * nblk;
+    const float mean_w = __fdiv_rn(1.0f, (float)ratio);
+    for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
+         t += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = t / nblk;
+        const int b = (int)(t - e * nblk);
+        float v[16];
+        for (int k = 0; k < ratio; ++k) {
+            const float wk = w ? __ldg(w + e * w_stride + k) : mean_w;
+            const T *xr = x + (e * ratio + k) * x_stride + b * 16;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float q = __fdiv_rn(fabsf(v[i]), s);
-                uint32_t c = e2m1_code_mag_rne(q) | (signbit(v[i]) ? 8u : 0u);
-                packed[i >> 3] |= c << ((i & 7) * 4);
+                const float prod = __fmul_rn(wk, load_as_f32<T>(xr + i));
+                v[i] = k == 0 ? prod : __fadd_rn(v[i], prod);
             }
         }
-        const int64_t d = dst_rows ? dst_rows[r] : r;
-        uint8_t *cd = codes + d * code_stride + b * 8;
-        // 8 code bytes; alignment of cd is only guaranteed to 1 byte in general
-        if ((((uintptr_t)cd) & 7u) == 0) {
-            *reinterpret_cast<uint2 *>(cd) = make_uint2(packed[0], packed[1]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cd[i] = (uint8_t)(packed[i >> 2] >> ((i & 3) * 8));
-        }
-        scales[d * scale_stride + b] = (uint8_t)sc;
+        const int64_t d = dst_rows ? dst_rows[e] : e;
+        quantize_block16(v, codes + d * code_stride + b * 8, scales + d * scale_stride + b);
     }
 }
 
@@ -127,6 +162,26 @@ cudaError_t launch_quant_fp4(const void *x, int x_dtype, int64_t rows, int dim, 
         quant_fp4_kernel<uint16_t><<<(unsigned)blocks, threads, 0, st>>>(
             (const uint16_t *)x, rows, dim, x_stride, codes, code_stride, scales, scale_stride,
             dst_rows);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compress_fp4(const void *x, int x_dtype, int64_t entries, int ratio, int dim,
+                                int64_t x_stride, const float *w, int64_t w_stride, uint8_t *codes,
+                                int64_t code_stride, uint8_t *scales, int64_t scale_stride,
+                                const int64_t *dst_rows, cudaStream_t st) {
+    const int64_t total = entries * (dim / 16);
+    const int threads = 256;
+    int64_t blocks = ceil_div(total, threads);
+    if (blocks > 148 * 64) blocks = 148 * 64;
+    if (x_dtype == CSA2_DTYPE_F32)
+        compress_fp4_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
+            (const float *)x, entries, ratio, dim, x_stride, w, w_stride, codes, code_stride, scales,
+            scale_stride, dst_rows);
+    else
+        compress_fp4_kernel<uint16_t><<<(unsigned)blocks, threads, 0, st>>>(
+            (const uint16_t *)x, entries, ratio, dim, x_stride, w, w_stride, codes, code_stride, scales,
+            scale_stride, dst_rows);
     note_launches(1);
     return cudaGetLastError();
 }

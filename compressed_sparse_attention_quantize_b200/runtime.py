@@ -144,3 +144,26 @@ class GroupRunner:
 
     def run(self, stream=None) -> None:
         csa2_layer_group(self.g, self.layer_descs, self.workspace, self.ws_bytes, stream)
+
+    def capture(self) -> int:
+        """Record one call of the layer group into a CUDA graph (after a warm-up call, so the
+        library's one-time attribute set-up happens outside the capture); ``replay()`` then
+        launches the whole group with one graph launch.  Returns the number of library kernels
+        the graph holds.  The graph reads the current contents of the runner's buffers."""
+        from . import csa2_launch_count
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.run()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        n0 = csa2_launch_count()
+        with torch.cuda.graph(graph):
+            self.run()
+        self.graph = graph
+        self.graph_kernels = csa2_launch_count() - n0
+        return self.graph_kernels
+
+    def replay(self) -> None:
+        self.graph.replay()

@@ -67,6 +67,7 @@ typedef enum csa2_status {
 #define CSA2_MAX_POOL     32768
 #define CSA2_MAX_HEADS    128     /* main query heads; a multiple of 16          */
 #define CSA2_SWA_WINDOW   128     /* at most this many window tokens per query   */
+#define CSA2_MAX_COMPRESS_RATIO 64 /* tokens per compressed entry                  */
 
 /* Human-readable name of a status code (static string, never NULL). */
 CSA2_API const char *csa2_status_string(csa2_status s);
@@ -103,6 +104,32 @@ CSA2_API csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64
                              int64_t x_stride, uint8_t *codes, int64_t code_stride,
                              void *scales, int64_t scale_stride, const int64_t *dst_rows,
                              void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_compress_quantize_kv -- sequence compressor fused with the FP4 quantise-on-write.
+ *
+ * [B] section "CSA2：三层压缩一次吃满": along the sequence every m tokens are compressed into
+ * one entry (V4's CSA does this with learned weights, which are not on the pages).  Here the
+ * caller supplies the per-token weights:
+ *     entry e = sum_{k<m} w[e][k] * x[m*e + k]
+ * in fp32, tokens in order k = 0..m-1, each product and each sum rounded once (no fused
+ * multiply-add); w == NULL takes the mean, w = 1/m (an IEEE fp32 quotient).  The entry is then
+ * quantised exactly as csa2_quantize_kv with CSA2_FMT_FP4_E2M1_E4M3S16 and written to
+ * destination row d = dst_rows ? dst_rows[e] : e (dim/2 code bytes at codes + d*code_stride,
+ * dim/16 E4M3 scale bytes at scales + d*scale_stride).
+ *
+ * x: entries*m token rows of dim elements of x_dtype (CSA2_DTYPE_F32 or CSA2_DTYPE_BF16), token
+ *    row t at x + t*x_stride elements.  w: NULL or fp32 [entries][w_stride] (w_stride >= m).
+ * Errors: INVALID_ARG (NULL x/codes/scales, unknown dtype), SHAPE (entries < 0, m < 1 or
+ *   m > CSA2_MAX_COMPRESS_RATIO, dim <= 0, not a multiple of 16 or > 65536, x_stride < dim,
+ *   w_stride < m, code_stride < dim/2, scale_stride < dim/16), CUDA.
+ * entries == 0 is a no-op returning CSA2_OK (checked after x_dtype).
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_compress_quantize_kv(const void *x, int x_dtype, int64_t entries, int ratio,
+                                      int dim, int64_t x_stride, const float *w,
+                                      int64_t w_stride, uint8_t *codes, int64_t code_stride,
+                                      uint8_t *scales, int64_t scale_stride,
+                                      const int64_t *dst_rows, void *stream);
 
 /* ------------------------------------------------------------------------------------
  * csa2_index_topk -- indexer scoring + top-K block selection for Full and Reindex layers.

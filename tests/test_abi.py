@@ -66,6 +66,22 @@ def test_quantize_validation(L):
     assert q(1, 16, 0, 4, 512, 512, 16, 512, 18, 4, None, None) == ALIGN
 
 
+def test_compress_validation(L):
+    c = L.csa2_compress_quantize_kv
+    # x, dtype, entries, ratio, dim, x_stride, w, w_stride, codes, code_stride, scales, scale_stride, dst, stream
+    assert c(16, 5, 4, 4, 512, 512, None, 0, 16, 256, 16, 32, None, None) == INVALID      # dtype
+    assert c(None, 0, 0, 4, 512, 512, None, 0, None, 256, None, 32, None, None) == OK      # entries == 0
+    assert c(16, 0, -1, 4, 512, 512, None, 0, 16, 256, 16, 32, None, None) == SHAPE
+    assert c(16, 0, 4, 0, 512, 512, None, 0, 16, 256, 16, 32, None, None) == SHAPE        # ratio < 1
+    assert c(16, 0, 4, 65, 512, 512, None, 0, 16, 256, 16, 32, None, None) == SHAPE       # ratio > max
+    assert c(16, 0, 4, 4, 500, 512, None, 0, 16, 256, 16, 32, None, None) == SHAPE        # dim % 16
+    assert c(16, 0, 4, 4, 512, 511, None, 0, 16, 256, 16, 32, None, None) == SHAPE        # x_stride
+    assert c(16, 0, 4, 4, 512, 512, 16, 3, 16, 256, 16, 32, None, None) == SHAPE          # w_stride < m
+    assert c(16, 0, 4, 4, 512, 512, None, 0, 16, 255, 16, 32, None, None) == SHAPE        # code_stride
+    assert c(16, 0, 4, 4, 512, 512, None, 0, 16, 256, 16, 31, None, None) == SHAPE        # scale_stride
+    assert c(None, 0, 4, 4, 512, 512, None, 0, 16, 256, 16, 32, None, None) == INVALID    # NULL x
+
+
 def _attn(L, **kw):
     a = dict(q=16, B=1, T=1, H=64, D=512, kv=16, kv_row_stride=288, seq_start=16, idx=16, cnt=None,
              K=64, swa_codes=16, swa_scale=16, swa_cap=128, swa_start=None, swa_len=16,

@@ -62,6 +62,41 @@ def test_quantize_fp4_scatter_rows():
     assert not codes.cpu().numpy()[[2, 10, 19]].any()
 
 
+@pytest.mark.parametrize("dtype,ratio,weighted", [("f32", 4, True), ("bf16", 4, True), ("f32", 4, False),
+                                                    ("f32", 3, True), ("bf16", 1, False), ("f32", 16, True)])
+def test_compress_fp4_bitexact(dtype, ratio, weighted):
+    """Compressor + quantise-on-write vs the oracle: packed 288-byte rows written at scattered
+    destinations; padded token rows and a padded weight matrix."""
+    rng = np.random.default_rng(200 + ratio)
+    entries, dim = 523, 512
+    x = rng.standard_normal((entries * ratio, dim)).astype(np.float32)
+    x[:, rng.choice(dim, 4, replace=False)] *= 8.0                  # outlier channels
+    x[::7] *= np.float32(1e-3)
+    xpad = np.zeros((entries * ratio, dim + 32), np.float32)
+    xpad[:, :dim] = x
+    xt = torch.from_numpy(xpad).cuda()
+    if dtype == "bf16":
+        xt = xt.to(torch.bfloat16)
+        x = xt[:, :dim].float().cpu().numpy()
+    w = None
+    wt = None
+    if weighted:
+        w = rng.uniform(-0.5, 1.0, (entries, ratio)).astype(np.float32)
+        wpad = np.zeros((entries, ratio + 3), np.float32)
+        wpad[:, :ratio] = w
+        wt = torch.from_numpy(wpad).cuda()
+    dst = torch.from_numpy(rng.permutation(entries + 40)[:entries].astype(np.int64)).cuda()
+    rows = torch.zeros((entries + 40, 288), dtype=torch.uint8, device="cuda")
+    csa2.csa2_compress_quantize_kv(xt, csa2.DTYPE_BF16 if dtype == "bf16" else csa2.DTYPE_F32, entries,
+                                   ratio, dim, xt.stride(0), wt, ratio + 3, rows, 288, rows[:, 256:], 288,
+                                   dst_rows=dst)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.compress_fp4(x, ratio, w)
+    got = rows.cpu().numpy()[dst.cpu().numpy()]
+    assert np.array_equal(got[:, :256], oc)
+    assert np.array_equal(got[:, 256:], os_)
+
+
 def test_quantize_fp8_token_bitexact():
     rng = np.random.default_rng(102)
     x = _special_rows(rng, 300, 512)
@@ -206,6 +241,21 @@ def test_layer_events_same_result():
         done[l].synchronize()
     torch.cuda.synchronize()
     r.set_layer_events(None, None)
+    for l, ld in enumerate(r.layer_data):
+        assert torch.equal(ld["out"], ref[l]), l
+
+
+def test_graph_replay_same_result():
+    """The layer group captured in a CUDA graph and replayed gives the eager call's outputs."""
+    wl = synth.scaled(synth.workload(2), B=3, n=4000, K=256, P=1000, name="graph")
+    r = _run_group(wl)
+    ref = [ld["out"].clone() for ld in r.layer_data]
+    kernels = r.capture()
+    assert kernels >= len(r.modes)
+    for ld in r.layer_data:
+        ld["out"].zero_()
+    r.replay()
+    torch.cuda.synchronize()
     for l, ld in enumerate(r.layer_data):
         assert torch.equal(ld["out"], ref[l]), l
 
