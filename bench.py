@@ -331,8 +331,8 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
         ev.record(cur)                       # creates the handles
     runner.set_layer_events([ev.cuda_event for ev in ready], None)
 
-    def step():
-        copy_stream.wait_stream(cur)
+    def body(main):
+        copy_stream.wait_stream(main)
         with torch.cuda.stream(copy_stream):
             for l, m in enumerate(runner.modes):
                 ld, e = runner.layer_data[l], host[l]
@@ -346,8 +346,23 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
         runner.run()
         out_host.copy_(out_last, non_blocking=True)
 
+    graph = None
     try:
         for _ in range(warmup):
+            flush()
+            body(cur)
+        torch.cuda.synchronize()
+        # the whole step (both streams, copies included) as one CUDA graph, as the device step is
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                body(torch.cuda.current_stream())
+            torch.cuda.synchronize()
+            graph = g
+        except Exception:                  # capture refused: time the eager step instead
+            torch.cuda.synchronize()
+        step = graph.replay if graph is not None else (lambda: body(cur))
+        for _ in range(2):
             flush()
             step()
         torch.cuda.synchronize()
@@ -357,7 +372,8 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
         runner.set_layer_events(None, None)
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": sum(ms) / steps, "overlap": "per-layer input copies on a second stream"}
+            "ms_per_step": sum(ms) / steps, "overlap": "per-layer input copies on a second stream",
+            "step": "cuda graph" if graph is not None else "eager"}
 
 
 def run_csa2(args, wl):
