@@ -137,8 +137,26 @@ struct RowPart {
     uint32_t sc[4];
 };
 
+// 32 bytes in one 256-bit load (p 32-byte aligned), read-only path
+CSA2_D void ldg_32B(const void *p, uint4 &lo, uint4 &hi) {
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+}
+
 CSA2_D void prefetch_part(const KeySrc &src, int hsel, RowPart &rp) {
-    if (src.valid && !src.swa) {
+    if (src.valid && !src.swa && (reinterpret_cast<uintptr_t>(src.ptr) & 31u) == 0) {
+        // aligned rows: one 256-bit load per region and one for the 32 scale bytes (5 requests
+        // instead of 10 -- the gather's request count throttled the load pipe)
+#pragma unroll
+        for (int mb = 0; mb < kBlocks; ++mb) ldg_32B(src.ptr + 32 * (2 * mb + hsel), rp.codes[2 * mb], rp.codes[2 * mb + 1]);
+        uint4 s0, s1;
+        ldg_32B(src.ptr + 256, s0, s1);
+        rp.sc[0] = hsel ? s0.y : s0.x;
+        rp.sc[1] = hsel ? s0.w : s0.z;
+        rp.sc[2] = hsel ? s1.y : s1.x;
+        rp.sc[3] = hsel ? s1.w : s1.z;
+    } else if (src.valid && !src.swa) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
 #pragma unroll
         for (int mb = 0; mb < kBlocks; ++mb) {
@@ -425,24 +443,28 @@ attn_tc_kernel(AttnArgs a) {
             }
             const bool cur_valid = src.valid;
             const float cur_scale = src.scale;
+            // ---- the next tile's rows are requested now, while the tensor core is idle until P
+            //      is ready (issued during P.V they slowed its operand reads); the softmax below
+            //      works on 16 heads at a time so these registers stay live without spilling
+            src = source_of(a, r, b, seq_start, e_next);
+            prefetch_part(src, hsel, rp);
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             if (!ptx::mbar_wait(&S.s_full, ph, abort_flag)) bad = true;
             if (block_any(bad || *abort_flag != 0, 1, kWorkers)) { aborted = true; break; }
             ptx::tc_fence_after();
-            float z[32];
-            {
-                uint32_t u[32];
-                ptx::tmem_ld32(lane_addr + half * 32, u);
-                ptx::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(u[i]);
-            }
             const float zs = qk_scale * cur_scale;
+            const uint32_t s_addr = lane_addr + half * 32;
             bool over = false;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                z[i] = cur_valid ? z[i] * zs : -INFINITY;
-                over |= z[i] > S.m_run[half * 32 + i] + kRescaleThreshold;
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t u[16];
+                ptx::tmem_ld16(s_addr + hh * 16, u);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float zi = cur_valid ? __uint_as_float(u[i]) * zs : -INFINITY;
+                    over |= zi > S.m_run[half * 32 + hh * 16 + i] + kRescaleThreshold;
+                }
             }
             // the running max moves only when some logit exceeds it by more than 2^8.  The max
             // scratch lives in P_lo, free here: s_full(j) completed after P.V(j-1).
@@ -450,8 +472,13 @@ attn_tc_kernel(AttnArgs a) {
             bool rescale = false;
             if (move) {
                 float v[32];
+                {
+                    uint32_t u[32];
+                    ptx::tmem_ld32(s_addr, u);
+                    ptx::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = z[i];
+                    for (int i = 0; i < 32; ++i) v[i] = cur_valid ? __uint_as_float(u[i]) * zs : -INFINITY;
+                }
                 warp_transpose_reduce<false>(v, lane);
                 X.red[sub][half * 32 + lane] = v[0];
                 ptx::named_barrier(1, kWorkers);
@@ -470,42 +497,51 @@ attn_tc_kernel(AttnArgs a) {
                 // barrier for the m_run / alpha writes, and whether any accumulated head moved
                 rescale = block_any(moved_here, 1, kWorkers);
             }
-            // probabilities (log2 domain)
+            // per 16 heads: probabilities (log2 domain), row sums (per key in TMEM, reduced over
+            // the keys once at the end), and the P^T line of key t: fp16 high halves to P_hi, low
+            // halves (P - fp16(P)) to P_lo.  P.V(j-1) finished before s_full(j), and the max
+            // scratch in P_lo was last read before the barrier above.
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float m = S.m_run[half * 32 + i];
-                z[i] = (m == -INFINITY || !cur_valid) ? 0.0f : ptx::ex2(z[i] - m);
-            }
-            // row sums: per key in TMEM, reduced over the keys once at the end
-            {
-                uint32_t u[32];
-                ptx::tmem_ld32(l_addr, u);
-                ptx::tmem_ld_wait();
+            for (int hh = 0; hh < 2; ++hh) {
+                float z[16];
+                {
+                    uint32_t u[16];
+                    ptx::tmem_ld16(s_addr + hh * 16, u);
+                    ptx::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float lp = __uint_as_float(u[i]);
-                    u[i] = __float_as_uint((move ? lp * S.alpha[half * 32 + i] : lp) + z[i]);
+                    for (int i = 0; i < 16; ++i) {
+                        const float m = S.m_run[half * 32 + hh * 16 + i];
+                        z[i] = (m == -INFINITY || !cur_valid) ? 0.0f : ptx::ex2(__uint_as_float(u[i]) * zs - m);
+                    }
                 }
-                ptx::tmem_st32(l_addr, u);
-            }
-            // P^T line of key t for this half's heads: fp16 high halves to P_hi, low halves
-            // (P - fp16(P)) to P_lo.  P.V(j-1) finished before s_full(j), and the max scratch
-            // in P_lo was last read before the barrier above.
+                {
+                    uint32_t u[16];
+                    ptx::tmem_ld16(l_addr + hh * 16, u);
+                    ptx::tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t hi4[4], lo4[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int i = 8 * c + 2 * k;
-                    const float q0 = z[i] * cur_scale, q1 = z[i + 1] * cur_scale;
-                    const __half2 hp = __floats2half2_rn(q0, q1);
-                    const float2 back = __half22float2(hp);
-                    const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
-                    hi4[k] = *reinterpret_cast<const uint32_t *>(&hp);
-                    lo4[k] = *reinterpret_cast<const uint32_t *>(&lp);
+                    for (int i = 0; i < 16; ++i) {
+                        const float lp = __uint_as_float(u[i]);
+                        u[i] = __float_as_uint((move ? lp * S.alpha[half * 32 + hh * 16 + i] : lp) + z[i]);
+                    }
+                    ptx::tmem_st16(l_addr + hh * 16, u);
                 }
-                *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-                *reinterpret_cast<uint4 *>(sPlo + sw128_off(t, half * 4 + c)) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t hi4[4], lo4[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int i = 8 * c2 + 2 * k;
+                        const float q0 = z[i] * cur_scale, q1 = z[i + 1] * cur_scale;
+                        const __half2 hp = __floats2half2_rn(q0, q1);
+                        const float2 back = __half22float2(hp);
+                        const __half2 lp = __floats2half2_rn(q0 - back.x, q1 - back.y);
+                        hi4[k] = *reinterpret_cast<const uint32_t *>(&hp);
+                        lo4[k] = *reinterpret_cast<const uint32_t *>(&lp);
+                    }
+                    const int c = hh * 2 + c2;
+                    *reinterpret_cast<uint4 *>(sP + sw128_off(t, half * 4 + c)) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                    *reinterpret_cast<uint4 *>(sPlo + sw128_off(t, half * 4 + c)) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+                }
             }
             // O^T rescale for heads whose running max moved (columns of this half)
             if (rescale) {
@@ -527,10 +563,6 @@ attn_tc_kernel(AttnArgs a) {
             ptx::fence_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&S.p_full);
-            // ---- the next tile's rows are requested while the tensor core runs P.V (not
-            //      earlier: live across the softmax they would push its registers into spills)
-            src = source_of(a, r, b, seq_start, e_next);
-            prefetch_part(src, hsel, rp);
         }
         // ---------------- epilogue ----------------
         if (!aborted && ntiles > 0 && !ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag)) bad = true;
