@@ -736,18 +736,39 @@ static int num_sms() {
     return g_num_sms;
 }
 
-// Split plan: enough CTAs to fill the SMs once (one CTA per SM), splitting on tile boundaries.
+// Split plan (one CTA per SM).  Each CTA costs a fixed part (Q staging, first loads, epilogue:
+// about 1.8 tile times, measured) plus its tiles; splits add merge work (about 0.009 tile times
+// per row and split, plus the merge launch).  The remainder split is the slowest-varying grid
+// index, so its short CTAs are the ones that wait for an SM when the grid exceeds the SMs.
+// Pick the tiles per split with the smallest estimated finish time.
 void tc_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_split) {
     hgroups = (H + tc::kHeads - 1) / tc::kHeads;
     const int max_keys = K + CSA2_SWA_WINDOW;
     const int tiles = (max_keys + tc::kTile - 1) / tc::kTile;
-    const int ctas = rows * hgroups;
-    int s = num_sms() / (ctas > 0 ? ctas : 1);
-    if (s < 1) s = 1;
-    if (s > tiles) s = tiles;
-    const int tiles_per = (tiles + s - 1) / s;
-    splits = (tiles + tiles_per - 1) / tiles_per;
-    keys_per_split = tiles_per * tc::kTile;
+    const int per_split = rows * hgroups;                     // CTAs of one split index
+    const int nsm = num_sms();
+    const double fixed = 1.8, merge_per = 0.009, merge_launch = 0.3;
+    double best = 1e30;
+    int best_tp = tiles;
+    for (int tp = 1; tp <= tiles; ++tp) {
+        const int sp = (tiles + tp - 1) / tp;
+        const int last = tiles - (sp - 1) * tp;
+        const long long ctas = (long long)per_split * sp;
+        double t;
+        if (ctas <= nsm) {
+            t = fixed + tp;
+        } else if (ctas - nsm <= per_split) {                 // only remainder CTAs wait
+            t = fixed + tp;
+            const double second = 2.0 * (fixed + last);
+            if (second > t) t = second;
+        } else {
+            t = (double)((ctas + nsm - 1) / nsm) * (fixed + tp);
+        }
+        if (sp > 1) t += merge_launch + merge_per * (double)per_split * sp;
+        if (t < best - 1e-9) { best = t; best_tp = tp; }
+    }
+    splits = (tiles + best_tp - 1) / best_tp;
+    keys_per_split = best_tp * tc::kTile;
 }
 
 size_t tc_workspace_bytes(int rows, int H, int K) {
