@@ -250,7 +250,9 @@ static csa2_status group_layout(const csa2_group_desc *g, const csa2_layer_desc 
         if (iw2 > iw) iw = iw2;
     }
     *attn_off = off + iw;
-    off += iw + attn_ws(rows, g->H, g->K);
+    // two attention workspaces: layer l merges its splits from slot l % 2 on a second stream
+    // while layer l + 1 runs
+    off += iw + attn_ws(rows, g->H, g->K) * (n > 1 ? 2 : 1);
     *total = off;
     return CSA2_OK;
 }
@@ -260,6 +262,30 @@ csa2_status csa2_layer_group_workspace_size(const csa2_group_desc *g, const csa2
     if (!bytes) return CSA2_ERR_INVALID_ARG;
     size_t a, b, c, d;
     return group_layout(g, layers, n_layers, &a, &b, &c, &d, bytes);
+}
+
+// Per host thread and device: the stream the layer group runs its split merges on, and the
+// events that order them (a thread's group calls never share them with another thread's).
+struct GroupAux {
+    cudaStream_t side = nullptr;
+    cudaEvent_t attn_done = nullptr, merge_done[2] = {nullptr, nullptr};
+};
+static cudaError_t group_aux(GroupAux **out) {
+    static thread_local GroupAux aux[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    GroupAux &a = aux[dev];
+    if (!a.side) {
+        e = cudaStreamCreateWithFlags(&a.side, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&a.attn_done, cudaEventDisableTiming);
+        for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&a.merge_done[i], cudaEventDisableTiming);
+        if (e != cudaSuccess) { a.side = nullptr; return e; }
+    }
+    *out = &a;
+    return cudaSuccess;
 }
 
 csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *layers, int n_layers,
@@ -297,8 +323,14 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     void *iws = ws + iws_off;
     const size_t iws_bytes = attn_off - iws_off;
     void *aws = ws + attn_off;
-    const size_t aws_bytes = total - attn_off;
+    const size_t aws_one = attn_ws(rows, g->H, g->K);
     cudaStream_t st = as_stream(stream);
+    GroupAux *aux = nullptr;
+    {
+        cudaError_t e = group_aux(&aux);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    bool merge_pending[2] = {false, false};
     for (int l = 0; l < n_layers; ++l) {
         const csa2_layer_desc &L = layers[l];
         if (L.ready_event) {
@@ -325,15 +357,41 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
                                             cudaMemcpyDeviceToDevice, st);
             if (e != cudaSuccess) return cuda_status(e);
         }
-        s = csa2_sparse_attn(L.q, g->B, g->T, g->H, g->D, g->kv, g->kv_row_stride, g->seq_start, idx,
-                             cnt, g->K, L.swa_codes, L.swa_scale, g->swa_cap, g->swa_start,
-                             g->swa_len, g->softmax_scale, L.out, g->out_dtype, L.lse, aws,
-                             aws_bytes, stream);
-        if (s != CSA2_OK) return s;
+        // attention on `st`; its split merge on the side stream, overlapping the next layers.
+        // Layer l uses workspace slot l % 2: before overwriting it, wait for layer l - 2's merge.
+        const int slot = n_layers > 1 ? (l & 1) : 0;
+        if (l >= 2 && merge_pending[slot]) {
+            cudaError_t e = cudaStreamWaitEvent(st, aux->merge_done[slot], 0);
+            if (e != cudaSuccess) return cuda_status(e);
+            merge_pending[slot] = false;
+        }
+        AttnArgs a;
+        a.q = L.q; a.rows = rows; a.T = g->T; a.H = g->H; a.K = g->K;
+        a.kv = g->kv; a.kv_row_stride = g->kv_row_stride; a.seq_start = g->seq_start;
+        a.idx = idx; a.cnt = cnt;
+        a.swa_codes = L.swa_codes; a.swa_scale = L.swa_scale; a.swa_cap = g->swa_cap;
+        a.swa_start = g->swa_start; a.swa_len = g->swa_len;
+        a.softmax_scale = g->softmax_scale; a.out = L.out; a.out_dtype = g->out_dtype; a.lse = L.lse;
+        a.partials = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(aws) + slot * aws_one);
+        a.splits = 1;
+        bool merged = false;
+        cudaError_t e = launch_attn_tc_side_merge(a, st, aux->side, aux->attn_done, &merged);
+        if (e != cudaSuccess) return cuda_status(e);
+        if (merged) {
+            e = cudaEventRecord(aux->merge_done[slot], aux->side);
+            if (e != cudaSuccess) return cuda_status(e);
+            merge_pending[slot] = true;
+        }
         if (L.done_event) {
-            cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(L.done_event), st);
+            e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(L.done_event), merged ? aux->side : st);
             if (e != cudaSuccess) return cuda_status(e);
         }
+    }
+    // the group completes on `stream`: join every merge still running on the side stream
+    for (int i = 0; i < 2; ++i) {
+        if (!merge_pending[i]) continue;
+        cudaError_t e = cudaStreamWaitEvent(st, aux->merge_done[i], 0);
+        if (e != cudaSuccess) return cuda_status(e);
     }
     return CSA2_OK;
 }

@@ -31,6 +31,8 @@ struct AttnArgs {
 constexpr int kPartialFloats = 2 * 64 + 64 * 512;
 
 cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st);
+cudaError_t launch_attn_tc_side_merge(AttnArgs a, cudaStream_t st, cudaStream_t side, cudaEvent_t attn_done,
+                                      bool *merged);
 size_t tc_workspace_bytes(int rows, int H, int K);
 
 // Dispatch used by the C ABI.

@@ -778,6 +778,35 @@ size_t tc_workspace_bytes(int rows, int H, int K) {
     return (size_t)rows * hg * sp * kPartialFloats * sizeof(float) + 256;
 }
 
+// As launch_attn_tc, but the split merge runs on `side` once the attention kernel has finished
+// (`attn_done` is recorded on `st` and waited on `side`); returns in *merged whether a merge was
+// queued on `side`.
+cudaError_t launch_attn_tc_side_merge(AttnArgs a, cudaStream_t st, cudaStream_t side, cudaEvent_t attn_done,
+                                      bool *merged) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             tc::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    tc_plan(a.rows, a.H, a.K, a.hgroups, a.splits, a.keys_per_split);
+    dim3 grid(a.rows, a.hgroups, a.splits);
+    tc::attn_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a);
+    int n = 1;
+    *merged = false;
+    if (a.splits > 1) {
+        cudaError_t e = cudaEventRecord(attn_done, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, attn_done, 0);
+        if (e != cudaSuccess) return e;
+        tc::attn_tc_merge_kernel<<<dim3(a.rows, a.H), 128, 0, side>>>(a);
+        ++n;
+        *merged = true;
+    }
+    note_launches(n);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st) {
     static bool attr_set = false;
     if (!attr_set) {
