@@ -291,6 +291,41 @@ def breakdown(torch, csa2, runner, steps, flush):
     return {k: v for k, v in times.items() if v}
 
 
+class gpu_local_cpus:
+    """Run the enclosed code on the CPUs NVML reports as local to the current GPU (read-only
+    NVML query), then restore the affinity.  Page-locked buffers allocated and first touched
+    inside land on the GPU's NUMA node, which decides the host<->device copy bandwidth."""
+
+    def __init__(self, torch):
+        self.torch = torch
+        self.saved = None
+        self.used = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            props = self.torch.cuda.get_device_properties(self.torch.cuda.current_device())
+            busid = f"{props.pci_domain_id:04x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+            words = (os.cpu_count() + 63) // 64
+            mask = pynvml.nvmlDeviceGetCpuAffinity(h, words)
+            cpus = {w * 64 + b for w, m in enumerate(mask) for b in range(64) if (int(m) >> b) & 1}
+            cpus &= set(os.sched_getaffinity(0))
+            if cpus:
+                self.saved = os.sched_getaffinity(0)
+                os.sched_setaffinity(0, cpus)
+                self.used = True
+        except Exception:
+            self.saved = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            os.sched_setaffinity(0, self.saved)
+        return False
+
+
 def e2e_measure(torch, csa2, runner, steps, warmup, flush):
     """The metric through csa2_layer_group with host buffers.  Per step: every layer's main query
     (bf16) and indexer query/weights (fp32) are copied from pinned host memory on a copy stream,
@@ -309,20 +344,22 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
 
     host = []
     h2d = 0
-    for l, m in enumerate(runner.modes):
-        ld = runner.layer_data[l]
-        hq = pinned_copy(ld["q"].cpu())
-        e = {"q": hq}
-        h2d += hq.numel() * 2
-        if m != "U":
-            iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
-            e["iq"] = pinned_copy(torch.from_numpy(iq))
-            e["iq_dev"] = torch.empty_like(e["iq"], device=ld["q"].device)
-            e["iw"] = pinned_copy(ld["iw"].cpu())
-            h2d += e["iq"].numel() * 4 + e["iw"].numel() * 4
-        host.append(e)
-    out_last = runner.layer_data[-1]["out"]
-    out_host = torch.empty(out_last.shape, dtype=out_last.dtype, pin_memory=True)
+    with gpu_local_cpus(torch) as local:
+        for l, m in enumerate(runner.modes):
+            ld = runner.layer_data[l]
+            hq = pinned_copy(ld["q"].cpu())
+            e = {"q": hq}
+            h2d += hq.numel() * 2
+            if m != "U":
+                iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
+                e["iq"] = pinned_copy(torch.from_numpy(iq))
+                e["iq_dev"] = torch.empty_like(e["iq"], device=ld["q"].device)
+                e["iw"] = pinned_copy(ld["iw"].cpu())
+                h2d += e["iq"].numel() * 4 + e["iw"].numel() * 4
+            host.append(e)
+        out_last = runner.layer_data[-1]["out"]
+        out_host = torch.empty(out_last.shape, dtype=out_last.dtype, pin_memory=True)
+        out_host.zero_()
     d2h = out_host.numel() * out_host.element_size()
     cur = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
@@ -373,7 +410,8 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": sum(ms) / steps, "overlap": "per-layer input copies on a second stream",
-            "step": "cuda graph" if graph is not None else "eager"}
+            "step": "cuda graph" if graph is not None else "eager",
+            "host_buffers": "GPU-local NUMA node" if local.used else "default placement"}
 
 
 def run_csa2(args, wl):

@@ -17,6 +17,8 @@ from typing import Optional, Sequence
 __all__ = [
     "CSA2Error", "lib", "library_path",
     "csa2_quantize_kv", "csa2_compress_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
+    "csa2_index_topk_scored", "csa2_topk_merge_shards", "csa2_topk_merge_shards_workspace_size",
+    "csa2_attn_merge_shards", "csa2_sparse_attn_shard",
     "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
@@ -92,6 +94,18 @@ def lib():
     L.csa2_compress_quantize_kv.restype = _i32
     L.csa2_compress_quantize_kv.argtypes = [_vp, _i32, _i64, _i32, _i32, _i64, _vp, _i64, _vp, _i64,
                                             _vp, _i64, _vp, _vp]
+    L.csa2_index_topk_scored.restype = _i32
+    L.csa2_index_topk_scored.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _vp, _i64, _vp, _vp, _i64,
+                                         _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
+    L.csa2_topk_merge_shards_workspace_size.restype = _i32
+    L.csa2_topk_merge_shards_workspace_size.argtypes = [_i32, _i32, _i32, ctypes.POINTER(_sz)]
+    L.csa2_topk_merge_shards.restype = _i32
+    L.csa2_topk_merge_shards.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
+    L.csa2_sparse_attn_shard.restype = _i32
+    L.csa2_sparse_attn_shard.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _i32,
+                                         _vp, _vp, _i32, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+    L.csa2_attn_merge_shards.restype = _i32
+    L.csa2_attn_merge_shards.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp]
     L.csa2_index_topk_workspace_size.restype = _i32
     L.csa2_index_topk_workspace_size.argtypes = [_i32, _i32, _i64, _i32, _i32, ctypes.POINTER(_sz)]
     L.csa2_index_topk.restype = _i32
@@ -171,6 +185,43 @@ def csa2_compress_quantize_kv(x, x_dtype, entries, ratio, dim, x_stride, w, w_st
     _check(lib().csa2_compress_quantize_kv(_ptr(x), x_dtype, entries, ratio, dim, x_stride, _ptr(w),
                                            w_stride, _ptr(codes), code_stride, _ptr(scales),
                                            scale_stride, _ptr(dst_rows), _stream(stream)))
+
+
+def csa2_index_topk_scored(q_codes, q_scales, w, B, T, H_I, k_codes, k_code_stride, k_scales,
+                           k_scale_stride, seq_start, n_entries, max_n, q_pos, K, out_idx, out_cnt,
+                           out_scores, workspace, ws_bytes, stream=None) -> None:
+    _check(lib().csa2_index_topk_scored(_ptr(q_codes), _ptr(q_scales), _ptr(w), B, T, H_I, _ptr(k_codes),
+                                        k_code_stride, _ptr(k_scales), k_scale_stride, _ptr(seq_start),
+                                        _ptr(n_entries), max_n, _ptr(q_pos), K, _ptr(out_idx), _ptr(out_cnt),
+                                        _ptr(out_scores), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def csa2_topk_merge_shards_workspace_size(G, rows, K_in) -> int:
+    out = _sz(0)
+    _check(lib().csa2_topk_merge_shards_workspace_size(G, rows, K_in, ctypes.byref(out)))
+    return out.value
+
+
+def csa2_topk_merge_shards(scores, ids, id_offset, cnt, G, rows, K_in, K, out_idx, out_cnt, workspace,
+                           ws_bytes, stream=None) -> None:
+    _check(lib().csa2_topk_merge_shards(_ptr(scores), _ptr(ids), _ptr(id_offset), _ptr(cnt), G, rows, K_in, K,
+                                        _ptr(out_idx), _ptr(out_cnt), _ptr(workspace), ws_bytes,
+                                        _stream(stream)))
+
+
+def csa2_sparse_attn_shard(q, B, T, H, D, kv, kv_row_stride, seq_start, shard_lo, shard_n, idx, cnt, K,
+                           swa_codes, swa_scale, swa_cap, swa_start, swa_len, softmax_scale, out, lse,
+                           workspace, ws_bytes, stream=None) -> None:
+    _check(lib().csa2_sparse_attn_shard(_ptr(q), B, T, H, D, _ptr(kv), kv_row_stride, _ptr(seq_start),
+                                        _ptr(shard_lo), _ptr(shard_n), _ptr(idx), _ptr(cnt), K, _ptr(swa_codes),
+                                        _ptr(swa_scale), swa_cap, _ptr(swa_start), _ptr(swa_len),
+                                        ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                        ws_bytes, _stream(stream)))
+
+
+def csa2_attn_merge_shards(outs, lses, G, rows, H, D, out, out_dtype, lse=None, stream=None) -> None:
+    _check(lib().csa2_attn_merge_shards(_ptr(outs), _ptr(lses), G, rows, H, D, _ptr(out), out_dtype, _ptr(lse),
+                                        _stream(stream)))
 
 
 def csa2_index_topk_workspace_size(mode, rows, max_n, K, P) -> int:

@@ -8,6 +8,13 @@
 #include "attn.cuh"
 
 namespace csa2 {
+size_t topk_merge_workspace_bytes(int G, int rows, int K_in);
+int64_t topk_cluster_max_n();
+cudaError_t launch_topk_merge_shards(const float *, const int32_t *, const int64_t *, const int32_t *, int, int,
+                                     int, int, int32_t *, int32_t *, void *, cudaStream_t);
+cudaError_t launch_attn_merge_shards(const float *, const float *, int, int, int, int, void *, int, float *,
+                                     cudaStream_t);
+
 cudaError_t launch_compress_fp4(const void *, int, int64_t, int, int, int64_t, const float *, int64_t,
                                 uint8_t *, int64_t, uint8_t *, int64_t, const int64_t *, cudaStream_t);
 cudaError_t launch_quant_fp4(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
@@ -186,7 +193,62 @@ csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uint8_t *q_s
     L.K = K; L.out_idx = out_idx; L.out_cnt = out_cnt;
     L.P = P; L.out_pool = out_pool; L.out_pool_len = out_pool_len;
     L.workspace = workspace; L.ws_bytes = ws_bytes;
+    L.out_scores = nullptr;
     return cuda_status(launch_index_topk(L, as_stream(stream)));
+}
+
+csa2_status csa2_index_topk_scored(const uint8_t *q_codes, const uint8_t *q_scales, const float *w, int B,
+                                   int T, int H_I, const uint8_t *k_codes, int64_t k_code_stride,
+                                   const uint8_t *k_scales, int64_t k_scale_stride,
+                                   const int64_t *seq_start, const int32_t *n_entries, int64_t max_n,
+                                   const int32_t *q_pos, int K, int32_t *out_idx, int32_t *out_cnt,
+                                   float *out_scores, void *workspace, size_t ws_bytes, void *stream) {
+    if (!out_scores) return CSA2_ERR_INVALID_ARG;
+    csa2_status s = check_index_args(CSA2_MODE_FULL, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_stride,
+                                     k_scales, k_scale_stride, seq_start, n_entries, max_n, nullptr,
+                                     nullptr, 0, K, out_idx, 0, nullptr);
+    if (s != CSA2_OK) return s;
+    const int rows = B * T;
+    if (!workspace || ws_bytes < index_ws(CSA2_MODE_FULL, rows, max_n, K, 0)) return CSA2_ERR_WORKSPACE;
+    IndexLaunch L;
+    L.mode = CSA2_MODE_FULL; L.q_codes = q_codes; L.q_scales = q_scales; L.w = w;
+    L.B = B; L.T = T; L.H = H_I;
+    L.k_codes = k_codes; L.k_code_stride = k_code_stride;
+    L.k_scales = k_scales; L.k_scale_stride = k_scale_stride;
+    L.seq_start = seq_start; L.n_entries = n_entries; L.max_n = max_n; L.q_pos = q_pos;
+    L.pool = nullptr; L.pool_len = nullptr; L.P_in = 0;
+    L.K = K; L.out_idx = out_idx; L.out_cnt = out_cnt;
+    L.P = 0; L.out_pool = nullptr; L.out_pool_len = nullptr;
+    L.workspace = workspace; L.ws_bytes = ws_bytes;
+    L.out_scores = out_scores;
+    return cuda_status(launch_index_topk(L, as_stream(stream)));
+}
+
+csa2_status csa2_topk_merge_shards_workspace_size(int G, int rows, int K_in, size_t *bytes) {
+    if (!bytes) return CSA2_ERR_INVALID_ARG;
+    if (G <= 0 || rows <= 0 || K_in <= 0) return CSA2_ERR_SHAPE;
+    *bytes = topk_merge_workspace_bytes(G, rows, K_in);
+    return CSA2_OK;
+}
+
+csa2_status csa2_topk_merge_shards(const float *scores, const int32_t *ids, const int64_t *id_offset,
+                                   const int32_t *cnt, int G, int rows, int K_in, int K, int32_t *out_idx,
+                                   int32_t *out_cnt, void *workspace, size_t ws_bytes, void *stream) {
+    if (!scores || !ids || !cnt || !out_idx) return CSA2_ERR_INVALID_ARG;
+    if (G <= 0 || rows <= 0 || K_in <= 0 || K < 1 || K > CSA2_MAX_TOPK) return CSA2_ERR_SHAPE;
+    if ((int64_t)G * K_in > topk_cluster_max_n()) return CSA2_ERR_UNSUPPORTED;
+    if (!workspace || ws_bytes < topk_merge_workspace_bytes(G, rows, K_in)) return CSA2_ERR_WORKSPACE;
+    return cuda_status(launch_topk_merge_shards(scores, ids, id_offset, cnt, G, rows, K_in, K, out_idx, out_cnt,
+                                                workspace, as_stream(stream)));
+}
+
+csa2_status csa2_attn_merge_shards(const float *outs, const float *lses, int G, int rows, int H, int D,
+                                   void *out, int out_dtype, float *lse, void *stream) {
+    if (!outs || !lses || !out) return CSA2_ERR_INVALID_ARG;
+    if (out_dtype != CSA2_DTYPE_F32 && out_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
+    if (G <= 0 || rows <= 0 || H <= 0 || D <= 0 || (D % 4)) return CSA2_ERR_SHAPE;
+    if ((((uintptr_t)outs) & 15u) || (((uintptr_t)out) & 15u)) return CSA2_ERR_ALIGN;
+    return cuda_status(launch_attn_merge_shards(outs, lses, G, rows, H, D, out, out_dtype, lse, as_stream(stream)));
 }
 
 csa2_status csa2_sparse_attn_workspace_size(int rows, int H, int K, size_t *bytes) {
@@ -211,10 +273,36 @@ csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D, cons
     AttnArgs a;
     a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
     a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start;
+    a.shard_lo = nullptr; a.shard_n = nullptr;
     a.idx = idx; a.cnt = cnt;
     a.swa_codes = swa_codes; a.swa_scale = swa_scale; a.swa_cap = swa_cap;
     a.swa_start = swa_start; a.swa_len = swa_len;
     a.softmax_scale = softmax_scale; a.out = out; a.out_dtype = out_dtype; a.lse = lse;
+    a.partials = reinterpret_cast<float *>(workspace);
+    a.splits = 1;
+    return cuda_status(launch_attn(a, as_stream(stream)));
+}
+
+csa2_status csa2_sparse_attn_shard(const uint16_t *q, int B, int T, int H, int D, const uint8_t *kv,
+                                   int64_t kv_row_stride, const int64_t *seq_start, const int64_t *shard_lo,
+                                   const int32_t *shard_n, const int32_t *idx, const int32_t *cnt, int K,
+                                   const uint8_t *swa_codes, const float *swa_scale, int swa_cap,
+                                   const int32_t *swa_start, const int32_t *swa_len, float softmax_scale,
+                                   float *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    if (!shard_lo || !shard_n || !lse) return CSA2_ERR_INVALID_ARG;
+    csa2_status s = check_attn_args(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, K, swa_codes,
+                                    swa_scale, swa_cap, swa_len, out, CSA2_DTYPE_F32);
+    if (s != CSA2_OK) return s;
+    const int rows = B * T;
+    if (!workspace || ws_bytes < attn_ws(rows, H, K)) return CSA2_ERR_WORKSPACE;
+    AttnArgs a;
+    a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
+    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start;
+    a.shard_lo = shard_lo; a.shard_n = shard_n;
+    a.idx = idx; a.cnt = cnt;
+    a.swa_codes = swa_codes; a.swa_scale = swa_scale; a.swa_cap = swa_cap;
+    a.swa_start = swa_start; a.swa_len = swa_len;
+    a.softmax_scale = softmax_scale; a.out = out; a.out_dtype = CSA2_DTYPE_F32; a.lse = lse;
     a.partials = reinterpret_cast<float *>(workspace);
     a.splits = 1;
     return cuda_status(launch_attn(a, as_stream(stream)));
@@ -368,6 +456,7 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
         AttnArgs a;
         a.q = L.q; a.rows = rows; a.T = g->T; a.H = g->H; a.K = g->K;
         a.kv = g->kv; a.kv_row_stride = g->kv_row_stride; a.seq_start = g->seq_start;
+        a.shard_lo = nullptr; a.shard_n = nullptr;
         a.idx = idx; a.cnt = cnt;
         a.swa_codes = L.swa_codes; a.swa_scale = L.swa_scale; a.swa_cap = g->swa_cap;
         a.swa_start = g->swa_start; a.swa_len = g->swa_len;

@@ -10,6 +10,8 @@ struct AttnArgs {
     const uint8_t *kv;          // main entries, kv_row_stride bytes apart
     int64_t kv_row_stride;
     const int64_t *seq_start;
+    const int64_t *shard_lo;    // context shards: [B] first global entry of this shard (NULL: none)
+    const int32_t *shard_n;     //   [B] entries in the shard; selected ids outside it are skipped
     const int32_t *idx;         // [rows][K]
     const int32_t *cnt;         // [rows] or NULL
     const uint8_t *swa_codes;   // [B][swa_cap][512]

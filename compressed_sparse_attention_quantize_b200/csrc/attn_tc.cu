@@ -94,6 +94,11 @@ struct KeySrc {
 CSA2_D KeySrc source_of(const AttnArgs &a, int r, int b, int64_t seq_start, int32_t e) {
     KeySrc k{false, false, nullptr, 0.0f};
     if (e == kNoKey) return k;
+    if (e >= 0 && a.shard_lo) {                   // context shard: global entry -> this shard's row
+        const int64_t le = (int64_t)e - a.shard_lo[b];
+        if (le < 0 || le >= a.shard_n[b]) return k;
+        e = (int32_t)le;
+    }
     k.valid = true;
     if (e >= 0) {
         k.ptr = a.kv + (seq_start + e) * a.kv_row_stride;

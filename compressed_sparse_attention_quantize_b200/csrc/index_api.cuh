@@ -29,6 +29,7 @@ struct IndexLaunch {
     int32_t *out_pool_len;
     void *workspace;
     size_t ws_bytes;
+    float *out_scores;          // FULL: scores of the selected entries [rows][K] (NULL: none)
 };
 
 // Scratch bytes for `rows` query rows with up to `n` candidates each.

@@ -215,6 +215,8 @@ cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, flo
                                   int64_t score_stride, cudaStream_t st);
 
 int64_t topk_cluster_max_n();
+cudaError_t launch_gather_scores(const float *scores, int64_t score_stride, const int32_t *idx, int K,
+                                 int row0, int nrows, float *out_scores, cudaStream_t st);
 cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const int32_t *cand,
                                 int cand_stride, const int32_t *n_entries, const int32_t *q_pos,
                                 const int32_t *pool_len, int T, int row0, int nrows, int K,
@@ -251,6 +253,8 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
                                                 sa.q_pos, sa.pool_len, sa.T, sa.row0, nr, L.K, L.out_idx,
                                                 L.out_cnt, reindex ? 0 : L.P, L.out_pool, L.out_pool_len,
                                                 max_n, st);
+            if (e == cudaSuccess && L.out_scores && !reindex)
+                e = launch_gather_scores(scores, sa.score_stride, L.out_idx, L.K, sa.row0, nr, L.out_scores, st);
             if (e != cudaSuccess) return e;
             continue;
         }
@@ -267,6 +271,8 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
         select_kernel<<<nr, kSelectThreads, 0, st>>>(se);
         note_launches(1);
         cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess && L.out_scores && !reindex)
+            e = launch_gather_scores(scores, sa.score_stride, L.out_idx, L.K, sa.row0, nr, L.out_scores, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -73,5 +73,7 @@ extern "C" csa2_status csa2_sparse_attn_noalloc(const uint16_t *q, int B, int T,
     a.softmax_scale = softmax_scale; a.out = out; a.out_dtype = out_dtype; a.lse = lse;
     a.partials = reinterpret_cast<float *>(scratch);
     a.splits = 1;
+    a.shard_lo = nullptr;
+    a.shard_n = nullptr;
     return cuda_status(launch_attn_tc(a, reinterpret_cast<cudaStream_t>(stream)));
 }

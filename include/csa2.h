@@ -294,6 +294,82 @@ CSA2_API csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer
                              int n_layers, void *workspace, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------
+ * Context parallelism: one long sequence whose compressed entries are split into
+ * consecutive shards, one per GPU ([A] section "压缩吸收注意力（二代）": the top 2048 blocks
+ * of the whole context, score descending, entry index ascending on ties; [B] section
+ * "CSA2：三层压缩一次吃满": one joint softmax over the selection).  Each GPU runs
+ * csa2_index_topk_scored and csa2_sparse_attn on its own shard; the caller all-gathers the
+ * results (NCCL) and merges them with the two calls below.  The global top-K lies inside the
+ * union of the shards' top-K lists, so the merged selection equals the single-GPU one.
+ *
+ * csa2_index_topk_scored -- csa2_index_topk in FULL mode (no pool) that also writes the
+ *   fp32 score of every selected entry: out_scores [B*T][K], -inf in padded slots.  Same
+ *   arguments, workspace and errors as csa2_index_topk; INVALID_ARG if out_scores is NULL.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_index_topk_scored(const uint8_t *q_codes, const uint8_t *q_scales,
+                                   const float *w, int B, int T, int H_I,
+                                   const uint8_t *k_codes, int64_t k_code_stride,
+                                   const uint8_t *k_scales, int64_t k_scale_stride,
+                                   const int64_t *seq_start, const int32_t *n_entries,
+                                   int64_t max_n, const int32_t *q_pos, int K,
+                                   int32_t *out_idx, int32_t *out_cnt, float *out_scores,
+                                   void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_topk_merge_shards -- top-K of the union of G shards' scored candidate lists.
+ *   scores, ids: [G][rows][K_in]; shard g's list for row r holds cnt[g*rows + r] valid
+ *   candidates first (ids ascending).  id_offset: [G][rows] int64 added to shard g's ids
+ *   (the shard's first global entry; NULL adds nothing).  After the offset, shard g's ids
+ *   must all lie below shard g+1's.
+ *   Output as csa2_index_topk: the selected ids ascending in out_idx [rows][K], -1 padded,
+ *   out_cnt [rows] (nullable) = min(K, candidates).  Order: score descending, id ascending.
+ *   workspace: csa2_topk_merge_shards_workspace_size(G, rows, K_in) bytes.
+ * Errors: INVALID_ARG (NULL scores/ids/cnt/out_idx), SHAPE (G, rows, K_in <= 0, K < 1 or
+ *   K > CSA2_MAX_TOPK), UNSUPPORTED (G*K_in above the selection's 262144 candidates),
+ *   WORKSPACE, CUDA.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_topk_merge_shards_workspace_size(int G, int rows, int K_in, size_t *bytes);
+CSA2_API csa2_status csa2_topk_merge_shards(const float *scores, const int32_t *ids,
+                                   const int64_t *id_offset, const int32_t *cnt, int G, int rows,
+                                   int K_in, int K,
+                                   int32_t *out_idx, int32_t *out_cnt, void *workspace,
+                                   size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_sparse_attn_shard -- csa2_sparse_attn over one shard's part of the selection: idx
+ *   holds GLOBAL entry numbers; entry e of sequence b is used only if it lies in the shard,
+ *   shard_lo[b] <= e < shard_lo[b] + shard_n[b], and is read from this GPU's cache row
+ *   seq_start[b] + e - shard_lo[b].  The window keys are taken as given (pass swa_len = 0 on
+ *   every shard but the one that holds the window).  Output fp32 out [B*T][H][D] and the
+ *   natural-log lse [B*T][H] (required): the inputs of csa2_attn_merge_shards.  Other
+ *   arguments, workspace and errors as csa2_sparse_attn; INVALID_ARG if shard_lo, shard_n or
+ *   lse is NULL.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_sparse_attn_shard(const uint16_t *q, int B, int T, int H, int D,
+                                   const uint8_t *kv, int64_t kv_row_stride,
+                                   const int64_t *seq_start, const int64_t *shard_lo,
+                                   const int32_t *shard_n, const int32_t *idx, const int32_t *cnt,
+                                   int K, const uint8_t *swa_codes, const float *swa_scale,
+                                   int swa_cap, const int32_t *swa_start, const int32_t *swa_len,
+                                   float softmax_scale, float *out, float *lse, void *workspace,
+                                   size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_attn_merge_shards -- log-sum-exp merge of G shards' attention results (each the
+ *   fp32 output and natural-log LSE of csa2_sparse_attn over that shard's part of the key
+ *   set): out = sum_g exp(lse_g - M) out_g / L, lse = M + ln L, M = max_g lse_g,
+ *   L = sum_g exp(lse_g - M), shards added in order g = 0..G-1.  A shard with lse = -inf
+ *   (no keys) contributes nothing.
+ *   outs: fp32 [G][rows][H][D] (16-byte aligned); lses: [G][rows][H]; out: [rows][H][D] of
+ *   out_dtype (16-byte aligned); lse: [rows][H] or NULL.
+ * Errors: INVALID_ARG (NULL outs/lses/out, unknown dtype), SHAPE (G, rows, H, D <= 0, D not a
+ *   multiple of 4), ALIGN, CUDA.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_attn_merge_shards(const float *outs, const float *lses, int G, int rows,
+                                   int H, int D, void *out, int out_dtype, float *lse,
+                                   void *stream);
+
+/* ------------------------------------------------------------------------------------
  * csa2_device_error -- reads (and clears) the library's device-side error word for the
  * current device: 0 when no bounded wait has expired since the last call, otherwise a
  * csa2_status code.  Synchronises `stream` first.
