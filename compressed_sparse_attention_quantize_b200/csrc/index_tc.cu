@@ -29,7 +29,6 @@ namespace itc {
 constexpr int kTile = 128;
 constexpr int kThreads = 128;
 constexpr int kMaxN = 4 * CSA2_MAX_INDEX_HEADS;      // 64 columns
-constexpr int kTilesPerCta = 8;                      // 1024 keys per CTA
 constexpr int kDepth = 2;                            // gathered tiles in flight per thread
 constexpr int kStages = 8;                           // contiguous tiles in flight per CTA
 constexpr int kRingBytes = kStages * kTile * 32;     // raw key rows, 32 bytes each
@@ -52,6 +51,7 @@ struct Args {
     float *scores;
     int64_t score_stride;
     uint32_t tmem_cols;
+    int tiles_per_cta;                 // consecutive 128-key tiles of a row per CTA
 };
 
 struct __align__(16) Smem {
@@ -108,9 +108,9 @@ index_score_tc_kernel(Args a) {
     const int r = a.row0 + blockIdx.y;
     const int b = r / a.T;
     const int64_t n = min(candidates(a, r), a.score_stride);
-    const int64_t j0 = (int64_t)blockIdx.x * kTilesPerCta * kTile;
+    const int64_t j0 = (int64_t)blockIdx.x * a.tiles_per_cta * kTile;
     if (j0 >= n) return;                                  // uniform per CTA: nothing allocated yet
-    const int ntiles = (int)min((int64_t)kTilesPerCta, (n - j0 + kTile - 1) / kTile);
+    const int ntiles = (int)min((int64_t)a.tiles_per_cta, (n - j0 + kTile - 1) / kTile);
     const int H = a.H;
     const int N = ((4 * H + 15) / 16) * 16;
     const uint32_t tmem_cols = a.tmem_cols;
@@ -329,24 +329,50 @@ cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, flo
     a.row0 = row0;
     a.scores = scores;
     a.score_stride = score_stride;
-    const int64_t per_cta = (int64_t)itc::kTilesPerCta * itc::kTile;
     // TMEM per CTA: D (N columns) + 32 columns of unit scale factors
     const int N = ((4 * L.H + 15) / 16) * 16;
     uint32_t cols = 32;
     while (cols < (uint32_t)(N + 32)) cols <<= 1;
     a.tmem_cols = cols;
     // reserve shared memory so that at most 512/cols CTAs are resident on an SM
+    // (and at least the bulk-copy ring of the contiguous path)
     const int per_sm = 512 / (int)cols;
     const int smem_total = (227 * 1024) / per_sm - 1024;
-    // (and at least the bulk-copy ring of the contiguous path)
     const int dyn = max(smem_total - (int)sizeof(itc::Smem), itc::kRingBytes);
     static int attr_dyn = -1;
+    static int resident = 0;
     if (attr_dyn != dyn) {
         cudaError_t e = cudaFuncSetAttribute(itc::index_score_tc_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
         if (e != cudaSuccess) return e;
         attr_dyn = dyn;
+        // resident CTAs per SM, from TMEM columns, shared memory (1 KB reserved per CTA) and
+        // registers (the occupancy query does not account for this kernel's limits)
+        int dev = 0, nsm = 148, smem_sm = 228 * 1024;
+        if (cudaGetDevice(&dev) == cudaSuccess) {
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+            cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        }
+        cudaFuncAttributes fa;
+        int regs = 72;
+        size_t stat = sizeof(itc::Smem);
+        if (cudaFuncGetAttributes(&fa, itc::index_score_tc_kernel) == cudaSuccess) {
+            regs = fa.numRegs > 0 ? fa.numRegs : regs;
+            stat = fa.sharedSizeBytes;
+        }
+        int blocks = per_sm;
+        blocks = min(blocks, smem_sm / (int)(stat + (size_t)dyn + 1024));
+        blocks = min(blocks, 65536 / (regs * itc::kThreads));
+        resident = max(blocks, 1) * nsm;
     }
+    // tiles per CTA: the fewest that fit every row's tiles into one wave of resident CTAs (a
+    // partial second wave would cost a whole CTA time); with more rows than resident CTAs, 8
+    const int64_t tiles_row = ceil_div(score_stride, (int64_t)itc::kTile);
+    const int64_t per_row_ctas = resident / (nrows > 0 ? nrows : 1);
+    int64_t tpc = per_row_ctas > 0 ? ceil_div(tiles_row, per_row_ctas) : 8;
+    if (tpc < 1) tpc = 1;
+    a.tiles_per_cta = (int)tpc;
+    const int64_t per_cta = tpc * itc::kTile;
     dim3 grid((unsigned)ceil_div(score_stride, per_cta), (unsigned)nrows);
     itc::index_score_tc_kernel<<<grid, itc::kThreads, dyn, st>>>(a);
     note_launches(1);
