@@ -64,28 +64,33 @@ struct Shared {
     int remaining;
 };
 
-// Block-wide exclusive count of a flag in thread order (kThreads threads, kThreads/32 warps;
-// warp 0 scans one partial per warp and zero for lanes beyond the warp count).
-static_assert(kThreads % 32 == 0 && kThreads <= 1024, "block_excl needs whole warps, at most 32");
+static_assert(kThreads % 32 == 0 && kThreads <= 1024, "block scans need whole warps, at most 32");
 static_assert(kThreads >= 256, "one thread per histogram bin");
-CSA2_D int block_excl(bool f, int *ws, int &total) {
+// Block-wide exclusive sum of per-thread counts in thread order (warp 0 scans one partial per
+// warp and zero for lanes beyond the warp count); total = the block's sum.
+CSA2_D int block_excl_sum(int v, int *ws, int &total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) ws[warp] = __popc(bal);
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    if (lane == 31) ws[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int v = lane < kThreads / 32 ? ws[lane] : 0;
-        int incl = v;
+        const int w = lane < kThreads / 32 ? ws[lane] : 0;
+        int wincl = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += x;
+            const int x = __shfl_up_sync(0xffffffffu, wincl, o);
+            if (lane >= o) wincl += x;
         }
-        ws[lane] = incl - v;
-        if (lane == 31) ws[32] = incl;
+        ws[lane] = wincl - w;
+        if (lane == 31) ws[32] = wincl;
     }
     __syncthreads();
-    const int res = ws[warp] + __popc(bal & ((1u << lane) - 1u));
+    const int res = ws[warp] + incl - v;
     total = ws[32];
     __syncthreads();
     return res;
@@ -183,26 +188,29 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
         out_base += g + take;
         eq_before += e;
     }
-    // ordered compaction of this chunk
-    int run_out = 0, run_eq = 0;
-    for (int base = 0; base < chunk_len; base += kThreads) {
-        const int i = base + threadIdx.x;
-        uint32_t key = 0u;
-        if (i < chunk_len) key = keys[i];
-        const bool g = i < chunk_len && key > thr;
-        const bool e = i < chunk_len && key == thr;
-        int eq_tot;
-        const int er = block_excl(e, S.warp_sums, eq_tot);
-        const bool sel = g || (e && eq_before + run_eq + er < need_eq);
-        int sel_tot;
-        const int pos = block_excl(sel, S.warp_sums, sel_tot);
+    // ordered compaction of this chunk: thread t owns the consecutive keys [t*per, (t+1)*per),
+    // so two block scans (equal keys before it, selections before it) place every output
+    const int per = ((chunk_len + kThreads - 1) / kThreads) | 1;     // odd: a warp's lanes hit 32 banks
+    const int i0 = min(chunk_len, threadIdx.x * per), i1 = min(chunk_len, i0 + per);
+    int my_gt = 0, my_eq = 0;
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t key = keys[i];
+        my_gt += key > thr;
+        my_eq += key == thr;
+    }
+    int eq_tot;
+    const int eq_pre = block_excl_sum(my_eq, S.warp_sums, eq_tot);
+    const int take = min(my_eq, max(0, need_eq - (eq_before + eq_pre)));     // my equal keys taken
+    int sel_tot;
+    int o = out_base + block_excl_sum(my_gt + take, S.warp_sums, sel_tot);
+    int eq_seen = 0;
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t key = keys[i];
+        const bool sel = key > thr || (key == thr && eq_seen++ < take);
         if (sel) {
-            const int64_t j = chunk_base + i;
-            const int o = out_base + run_out + pos;
-            if (o < k) out[o] = ids ? ids[j] : (int32_t)j;     // never past the row's k slots
+            if (o < k) out[o] = ids ? ids[chunk_base + i] : (int32_t)(chunk_base + i);   // never past k
+            ++o;
         }
-        run_out += sel_tot;
-        run_eq += eq_tot;
     }
     cl.sync();                                      // counts may be reused by the next selection
 }
