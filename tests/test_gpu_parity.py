@@ -266,3 +266,81 @@ def test_full_size_sampled(cfg, rows):
     wl = synth.workload(cfg)
     r = _run_group(wl)
     _check_rows(r, wl, rows)
+
+
+def test_topk_heavy_ties_full_pool_reindex():
+    """Selections where exact score ties straddle the K-th and P-th places.
+
+    Keys of sequence 0 repeat with period 13, so its ~30000 scores take 13 values and the
+    2048th and 3000th places fall inside tie classes; sequence 4 has zero head weights, so all
+    of its scores are +0.  Ties are broken by entry index ascending ([A] section
+    "压缩吸收注意力（二代）" orders the selection by score; the index order on ties is the
+    reading both sides share).  Also: a distinct-key row with a ragged tail, a row with exactly
+    K entries and an empty row.  Full mode emits the pool; a Reindex pass re-scores it with a
+    second query.  Codes and scales are drawn directly (no quantisation step on either side).
+    """
+    rng = np.random.default_rng(4242)
+    H_I, K, P = 8, 2048, 3000
+    n = [30000, 4097, 2048, 0, 30000]
+    B = len(n)
+    starts = np.concatenate([[0], np.cumsum(n)[:-1]]).astype(np.int64)
+    total = int(sum(n))
+    kc = rng.integers(0, 256, (total, 32), dtype=np.uint8)
+    ks = rng.integers(0x28, 0x49, (total, 4), dtype=np.uint8)
+    base_c, base_s = kc[:13].copy(), ks[:13].copy()
+    j = np.arange(n[0]) % 13
+    kc[:n[0]], ks[:n[0]] = base_c[j], base_s[j]
+
+    def query(seed):
+        r = np.random.default_rng(seed)
+        qc = r.integers(0, 256, (B, H_I, 32), dtype=np.uint8)
+        qs = r.integers(0x28, 0x49, (B, H_I, 4), dtype=np.uint8)
+        w = r.uniform(0, 1, (B, H_I)).astype(np.float32)
+        w[2] = 0.0
+        w[4] = 0.0
+        return qc, qs, w
+
+    dev = torch.device("cuda")
+    g_kc, g_ks = torch.from_numpy(kc).to(dev), torch.from_numpy(ks).to(dev)
+    g_start = torch.from_numpy(starts).to(dev)
+    g_n = torch.tensor(n, dtype=torch.int32, device=dev)
+    max_n = max(n)
+
+    qc, qs, w = query(1)
+    idx = torch.empty((B, K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+    pool = torch.empty((B, P), dtype=torch.int32, device=dev)
+    pool_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = torch.empty(csa2.csa2_index_topk_workspace_size(csa2.MODE_FULL, B, max_n, K, P), dtype=torch.uint8,
+                     device=dev)
+    csa2.csa2_index_topk(csa2.MODE_FULL, torch.from_numpy(qc).to(dev), torch.from_numpy(qs).to(dev),
+                         torch.from_numpy(w).to(dev), B, 1, H_I, g_kc, 32, g_ks, 4, g_start, g_n, max_n, None,
+                         None, None, 0, K, idx, cnt, P, pool, pool_len, ws, ws.numel())
+    torch.cuda.synchronize()
+    o_pools = []
+    for b in range(B):
+        s0 = int(starts[b])
+        oi, oc, op, opl, s = oracle.full_index(qc[b], qs[b], w[b], kc[s0:s0 + n[b]], ks[s0:s0 + n[b]], n[b], K, P)
+        if b == 0:
+            kth = np.sort(s)[::-1][K - 1]
+            assert np.count_nonzero(s == kth) > 1 and np.count_nonzero(s > kth) < K   # a tie straddles K
+        assert int(cnt[b]) == oc and np.array_equal(idx[b].cpu().numpy(), oi), f"top-K row {b}"
+        assert int(pool_len[b]) == opl and np.array_equal(pool[b].cpu().numpy(), op), f"pool row {b}"
+        o_pools.append((op, opl))
+    assert np.array_equal(idx[4].cpu().numpy(), np.arange(K, dtype=np.int32))
+
+    qc2, qs2, w2 = query(2)
+    w2[4] = rng.uniform(0, 1, H_I).astype(np.float32)
+    idx2 = torch.empty((B, K), dtype=torch.int32, device=dev)
+    cnt2 = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws2 = torch.empty(csa2.csa2_index_topk_workspace_size(csa2.MODE_REINDEX, B, max_n, K, P), dtype=torch.uint8,
+                      device=dev)
+    csa2.csa2_index_topk(csa2.MODE_REINDEX, torch.from_numpy(qc2).to(dev), torch.from_numpy(qs2).to(dev),
+                         torch.from_numpy(w2).to(dev), B, 1, H_I, g_kc, 32, g_ks, 4, g_start, g_n, max_n, None,
+                         pool, pool_len, P, K, idx2, cnt2, 0, None, None, ws2, ws2.numel())
+    torch.cuda.synchronize()
+    for b in range(B):
+        s0 = int(starts[b])
+        op, opl = o_pools[b]
+        oi, oc = oracle.reindex(qc2[b], qs2[b], w2[b], kc[s0:s0 + n[b]], ks[s0:s0 + n[b]], op, opl, K)
+        assert int(cnt2[b]) == oc and np.array_equal(idx2[b].cpu().numpy(), oi), f"reindex row {b}"
