@@ -9,8 +9,9 @@
 // column (h, b) carries head h's codes for block b and zeros elsewhere -- and every block scale
 // fed to the MMA is 1.0, so each output is a sum of 16 exact products (multiples of 1/4, at most
 // 576): exact in fp32.  The epilogue multiplies by the two E4M3 scales (exact) and adds blocks
-// and heads in the fixed order of the reference (explicitly rounded adds and multiplies), so
-// the scores -- and therefore the selected sets -- are bit-identical to it.
+// and heads in the fixed order that csa2.h defines (explicitly rounded adds and multiplies), so
+// the scores -- and therefore the selected sets -- are bit-identical to any implementation of
+// that order (the oracle's is one).
 //
 // Operands in shared memory, K-major without swizzle: a 32-byte row of FP4 codes is two 16-byte
 // planes (elements 0-31 and 32-63), rows 16 bytes apart inside a plane.  D: 128 lanes (keys) x

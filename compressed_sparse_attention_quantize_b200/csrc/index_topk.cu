@@ -8,8 +8,8 @@
 // [A] page "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径", section
 //   "压缩吸收注意力（二代）": the first layer picks 2048 blocks and keeps a candidate pool.
 //
-// Scores come from the tensor-core kernel in index_tc.cu (bit-identical to the reference's
-// fixed fp32 order) into a bounded row-chunked buffer; selection runs on 8-CTA clusters
+// Scores come from the tensor-core kernel in index_tc.cu (bit-identical to the fixed fp32
+// summation order that csa2.h defines) into a bounded row-chunked buffer; selection runs on 8-CTA clusters
 // (topk_cluster.cu) or, for rows longer than a cluster holds, on one CTA per row here: a 4-pass,
 // 8-bit radix select on order-preserving keys, then one compaction pass in entry order
 // (entries above the threshold key, plus the lowest-indexed entries equal to it, written in

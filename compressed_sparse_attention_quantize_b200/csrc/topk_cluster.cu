@@ -11,7 +11,9 @@
 // shared memory (identical totals -> identical decisions, no broadcast needed).  Compaction:
 // each CTA publishes how many of its keys are above / equal to the threshold; the CTA's output
 // offset and its share of the "equal" keys (lowest indices first) follow from the lower-ranked
-// CTAs' counts; inside the CTA a block scan writes the selected ids in ascending order.
+// CTAs' counts.  Inside the CTA each thread owns a consecutive run of keys; two block scans
+// (equal keys before the thread, then selections before it) give every thread its output
+// offset, so the selected ids come out in ascending order.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
