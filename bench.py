@@ -520,7 +520,7 @@ def run_csa2(args, wl):
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "fp4(e2m1)+e4m3 storage; f32 compute",
+                "scaling": "weak", "vs_baseline": None, "dtype": "f16 MMA (attention), fp4 MMA (indexer), f32 accumulate",
                 "data": "synthetic (seeded; shapes and distributions of the workload)",
                 "config": {"workload": wl.name, "batch_per_gpu": wl.B, "ctx_tokens": wl.ctx_tokens[0],
                            "entries_per_seq": wl.n_entries[0], "layers": ",".join(wl.modes),
