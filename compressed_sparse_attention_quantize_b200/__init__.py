@@ -20,7 +20,7 @@ __all__ = [
     "csa2_index_topk_scored", "csa2_topk_merge_shards", "csa2_topk_merge_shards_workspace_size",
     "csa2_attn_merge_shards", "csa2_sparse_attn_shard",
     "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_noalloc",
-    "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error",
+    "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error", "csa2_selftest_bounded_wait",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
     "FMT_FP4", "FMT_FP8_TOKEN", "DTYPE_F32", "DTYPE_BF16", "MODE_FULL", "MODE_REINDEX",
     "MODE_REUSE",
@@ -128,6 +128,8 @@ def lib():
                                    _sz, _vp]
     L.csa2_device_error.restype = _i32
     L.csa2_device_error.argtypes = [_vp]
+    L.csa2_selftest_bounded_wait.restype = _i32
+    L.csa2_selftest_bounded_wait.argtypes = [_i32, _vp]
     L.csa2_last_error_string.restype = ctypes.c_char_p
     L.csa2_last_error_string.argtypes = []
     L.csa2_launch_count.restype = ctypes.c_uint64
@@ -289,6 +291,12 @@ def csa2_layer_group(g: GroupDesc, layers: Sequence[LayerDesc], workspace, ws_by
 
 def csa2_device_error(stream=None) -> int:
     return lib().csa2_device_error(_stream(stream))
+
+
+def csa2_selftest_bounded_wait(skip_arrival: bool, stream=None) -> None:
+    """Launch the bounded-wait self-test; with skip_arrival the next csa2_device_error
+    returns CSA2_ERR_TIMEOUT (6)."""
+    _check(lib().csa2_selftest_bounded_wait(1 if skip_arrival else 0, _stream(stream)))
 
 
 def csa2_launch_count() -> int:

@@ -15,6 +15,7 @@ cudaError_t launch_topk_merge_shards(const float *, const int32_t *, const int64
 cudaError_t launch_attn_merge_shards(const float *, const float *, int, int, int, int, void *, int, float *,
                                      cudaStream_t);
 
+cudaError_t launch_selftest_bounded_wait(int, cudaStream_t);
 cudaError_t launch_compress_fp4(const void *, int, int64_t, int, int, int64_t, const float *, int64_t,
                                 uint8_t *, int64_t, uint8_t *, int64_t, const int64_t *, cudaStream_t);
 cudaError_t launch_quant_fp4(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
@@ -483,6 +484,10 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
         if (e != cudaSuccess) return cuda_status(e);
     }
     return CSA2_OK;
+}
+
+csa2_status csa2_selftest_bounded_wait(int skip_arrival, void *stream) {
+    return cuda_status(launch_selftest_bounded_wait(skip_arrival != 0, as_stream(stream)));
 }
 
 csa2_status csa2_device_error(void *stream) {

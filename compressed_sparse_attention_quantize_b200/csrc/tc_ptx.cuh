@@ -38,8 +38,9 @@ CSA2_D bool mbar_try(uint64_t *bar, uint32_t parity) {
 // waiter would see the phase flip late.
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr uint32_t kSpinBackoff = 1u << 16;
+template <uint32_t kLimit = kSpinLimit>
 CSA2_D bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    for (uint32_t i = 0; i < kLimit; ++i) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
         if (i > kSpinBackoff) __nanosleep(64);

@@ -377,6 +377,19 @@ CSA2_API csa2_status csa2_attn_merge_shards(const float *outs, const float *lses
 CSA2_API csa2_status csa2_device_error(void *stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa2_selftest_bounded_wait -- failure-detection self-test of the bounded device-side wait
+ * that the pipelined kernels use (no page defines it; it checks this library's own error
+ * path).  Launches one CTA on `stream`: a producer thread arrives on an mbarrier that a
+ * consumer thread waits for, then waits for the consumer's reply.  skip_arrival != 0 makes the
+ * producer skip its arrival, so the consumer's wait gives up after 2^10 polls, the device
+ * error word becomes CSA2_ERR_TIMEOUT (read it with csa2_device_error) and the kernel
+ * exits.  Nothing traps or faults, and the context stays usable.  With skip_arrival == 0 the
+ * handshake completes and the error word is untouched.
+ * Errors: CUDA (launch failure).
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_selftest_bounded_wait(int skip_arrival, void *stream);
+
+/* ------------------------------------------------------------------------------------
  * csa2_last_error_string -- description of the last CUDA runtime error a call of this
  * library met on the calling host thread (the reason behind CSA2_ERR_CUDA), or "" if none.
  * ---------------------------------------------------------------------------------- */
