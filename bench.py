@@ -326,6 +326,42 @@ class gpu_local_cpus:
         return False
 
 
+def topk_side_reference(torch, csa2, wl, flush, reps=10):
+    """torch.topk next to the library's top-K on the same fp32 score buffer (side reference only).
+
+    Scores: [rows][n] uniform on [0, 1), seeded; K of n per row.  The library's side is
+    csa2_topk_merge_shards with one shard holding the whole row, which also returns the
+    selection in ascending index order.  Both selections are checked to have the same
+    K-th largest score per row."""
+    rows, n, K = wl.B * wl.T, int(max(wl.n_entries)), wl.K
+    g = torch.Generator(device="cuda")
+    g.manual_seed(int(wl.seed) + 77)
+    scores = torch.rand((1, rows, n), generator=g, device="cuda", dtype=torch.float32)
+    ids = torch.arange(n, dtype=torch.int32, device="cuda").repeat(1, rows, 1).contiguous()
+    cnt = torch.full((1, rows), n, dtype=torch.int32, device="cuda")
+    idx = torch.empty((rows, K), dtype=torch.int32, device="cuda")
+    out_cnt = torch.empty((rows,), dtype=torch.int32, device="cuda")
+    ws = torch.empty(csa2.csa2_topk_merge_shards_workspace_size(1, rows, n), dtype=torch.uint8, device="cuda")
+    res = {}
+
+    def ours():
+        csa2.csa2_topk_merge_shards(scores, ids, None, cnt, 1, rows, n, K, idx, out_cnt, ws, ws.numel())
+
+    def theirs():
+        res["t"] = torch.topk(scores[0], K, dim=1, sorted=False)
+
+    for f in (ours, theirs):
+        f()
+    t_ours = time_steps(torch, ours, reps, flush)
+    t_torch = time_steps(torch, theirs, reps, flush)
+    kth_ours = scores[0].gather(1, idx.long()).min(dim=1).values
+    kth_torch = res["t"].values.min(dim=1).values
+    return {"scores": f"[{rows}][{n}] fp32 uniform [0,1)", "k": K,
+            "csa2_topk_ms": statistics.median(t_ours), "torch_topk_ms": statistics.median(t_torch),
+            "kth_value_equal": bool(torch.equal(kth_ours, kth_torch)),
+            "note": "csa2_topk_merge_shards (one shard) vs torch.topk(sorted=False); L2 flushed before each call"}
+
+
 def e2e_measure(torch, csa2, runner, steps, warmup, flush):
     """The metric through csa2_layer_group with host buffers.  Per step: every layer's main query
     (bf16) and indexer query/weights (fp32) are copied from pinned host memory on a copy stream,
@@ -517,6 +553,11 @@ def run_csa2(args, wl):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, runner.softmax_scale)
 
+    try:
+        side = topk_side_reference(torch, csa2, wl, flush)
+    except Exception as exc:                 # a side reference never costs the main line
+        side = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -529,7 +570,7 @@ def run_csa2(args, wl):
                            "parallelism": f"replicas x{world} (independent sequences)",
                            "l2": "flushed between steps (256 MB write, outside the events)"},
                 "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": int(launches), "clocks": clocks}
+                "gpu_launches": int(launches), "clocks": clocks, "topk_side_reference": side}
         print(json.dumps(line), flush=True)
     del runner
     if world > 1:
