@@ -535,7 +535,8 @@ def run_csa2(args, wl):
         roof = {"kernel": "csa2_sparse_attn", "bound": "tensor", "achieved": k["achieved_tflops"],
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": k["achieved_tflops"] / tc_peak,
                 "traffic": ATTN_TRAFFIC_BYTES, "traffic_source": ATTN_TRAFFIC_SOURCE, "peak_source": f"{peak_src} bf16_tflops (fp16 MMA runs at the same rate)",
-                "hbm_achieved_gbs": k["achieved_gbs"], "hbm_frac": k["achieved_gbs"] / hbm_peak}
+                "hbm_achieved_gbs": k["achieved_gbs"], "hbm_frac": k["achieved_gbs"] / hbm_peak,
+                "hbm_frac_of_nominal_8tbs": k["achieved_gbs"] / 8000.0}
     elif dom == "index_topk":
         k = kernels[dom]
         roof = {"kernel": "csa2_index_topk", "bound": "hbm", "achieved": k["achieved_gbs"],
