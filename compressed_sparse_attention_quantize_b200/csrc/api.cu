@@ -28,6 +28,8 @@ cudaError_t launch_quant_fp8_token(const void *, int, int64_t, int, int64_t, uin
 
 #include <atomic>
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace csa2 {
 static std::atomic<uint64_t> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -44,6 +46,18 @@ inline csa2_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return CSA2_OK;
     snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
     return CSA2_ERR_CUDA;
+}
+// Host-timeline ranges for profilers: every public call, and each layer inside a group.  NVTX3
+// is header-only; without an attached tool the push and pop are no-ops.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
+inline const char *layer_range_name(int mode) {
+    return mode == CSA2_MODE_FULL ? "csa2 layer: Full" : mode == CSA2_MODE_REINDEX ? "csa2 layer: Reindex"
+                                                                                   : "csa2 layer: Reuse";
 }
 constexpr size_t kAlign = 256;
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -128,6 +142,7 @@ uint64_t csa2_launch_count(void) { return g_launches.load(std::memory_order_rela
 csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
                              int64_t x_stride, uint8_t *codes, int64_t code_stride, void *scales,
                              int64_t scale_stride, const int64_t *dst_rows, void *stream) {
+    const Range range("csa2_quantize_kv");
     if (fmt != CSA2_FMT_FP4_E2M1_E4M3S16 && fmt != CSA2_FMT_FP8_E4M3_TOKEN) return CSA2_ERR_INVALID_ARG;
     if (x_dtype != CSA2_DTYPE_F32 && x_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
     if (rows == 0) return CSA2_OK;                               // no-op, whatever the strides
@@ -150,6 +165,7 @@ csa2_status csa2_compress_quantize_kv(const void *x, int x_dtype, int64_t entrie
                                       int64_t x_stride, const float *w, int64_t w_stride,
                                       uint8_t *codes, int64_t code_stride, uint8_t *scales,
                                       int64_t scale_stride, const int64_t *dst_rows, void *stream) {
+    const Range range("csa2_compress_quantize_kv");
     if (x_dtype != CSA2_DTYPE_F32 && x_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
     if (entries == 0) return CSA2_OK;
     if (entries < 0 || ratio < 1 || ratio > CSA2_MAX_COMPRESS_RATIO || dim <= 0 || (dim % 16) ||
@@ -177,6 +193,7 @@ csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uint8_t *q_s
                             int P_in, int K, int32_t *out_idx, int32_t *out_cnt, int P,
                             int32_t *out_pool, int32_t *out_pool_len, void *workspace,
                             size_t ws_bytes, void *stream) {
+    const Range range("csa2_index_topk");
     csa2_status s = check_index_args(mode, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_stride,
                                      k_scales, k_scale_stride, seq_start, n_entries, max_n, pool,
                                      pool_len, P_in, K, out_idx, P, out_pool);
@@ -204,6 +221,7 @@ csa2_status csa2_index_topk_scored(const uint8_t *q_codes, const uint8_t *q_scal
                                    const int64_t *seq_start, const int32_t *n_entries, int64_t max_n,
                                    const int32_t *q_pos, int K, int32_t *out_idx, int32_t *out_cnt,
                                    float *out_scores, void *workspace, size_t ws_bytes, void *stream) {
+    const Range range("csa2_index_topk_scored");
     if (!out_scores) return CSA2_ERR_INVALID_ARG;
     csa2_status s = check_index_args(CSA2_MODE_FULL, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_stride,
                                      k_scales, k_scale_stride, seq_start, n_entries, max_n, nullptr,
@@ -235,6 +253,7 @@ csa2_status csa2_topk_merge_shards_workspace_size(int G, int rows, int K_in, siz
 csa2_status csa2_topk_merge_shards(const float *scores, const int32_t *ids, const int64_t *id_offset,
                                    const int32_t *cnt, int G, int rows, int K_in, int K, int32_t *out_idx,
                                    int32_t *out_cnt, void *workspace, size_t ws_bytes, void *stream) {
+    const Range range("csa2_topk_merge_shards");
     if (!scores || !ids || !cnt || !out_idx) return CSA2_ERR_INVALID_ARG;
     if (G <= 0 || rows <= 0 || K_in <= 0 || K < 1 || K > CSA2_MAX_TOPK) return CSA2_ERR_SHAPE;
     if ((int64_t)G * K_in > topk_cluster_max_n()) return CSA2_ERR_UNSUPPORTED;
@@ -245,6 +264,7 @@ csa2_status csa2_topk_merge_shards(const float *scores, const int32_t *ids, cons
 
 csa2_status csa2_attn_merge_shards(const float *outs, const float *lses, int G, int rows, int H, int D,
                                    void *out, int out_dtype, float *lse, void *stream) {
+    const Range range("csa2_attn_merge_shards");
     if (!outs || !lses || !out) return CSA2_ERR_INVALID_ARG;
     if (out_dtype != CSA2_DTYPE_F32 && out_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
     if (G <= 0 || rows <= 0 || H <= 0 || D <= 0 || (D % 4)) return CSA2_ERR_SHAPE;
@@ -266,6 +286,7 @@ csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D, cons
                              const int32_t *swa_len, float softmax_scale, void *out,
                              int out_dtype, float *lse, void *workspace, size_t ws_bytes,
                              void *stream) {
+    const Range range("csa2_sparse_attn");
     csa2_status s = check_attn_args(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, K, swa_codes,
                                     swa_scale, swa_cap, swa_len, out, out_dtype);
     if (s != CSA2_OK) return s;
@@ -290,6 +311,7 @@ csa2_status csa2_sparse_attn_shard(const uint16_t *q, int B, int T, int H, int D
                                    const uint8_t *swa_codes, const float *swa_scale, int swa_cap,
                                    const int32_t *swa_start, const int32_t *swa_len, float softmax_scale,
                                    float *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    const Range range("csa2_sparse_attn_shard");
     if (!shard_lo || !shard_n || !lse) return CSA2_ERR_INVALID_ARG;
     csa2_status s = check_attn_args(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, K, swa_codes,
                                     swa_scale, swa_cap, swa_len, out, CSA2_DTYPE_F32);
@@ -379,6 +401,7 @@ static cudaError_t group_aux(GroupAux **out) {
 
 csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *layers, int n_layers,
                              void *workspace, size_t ws_bytes, void *stream) {
+    const Range range("csa2_layer_group");
     size_t idx_off, pool_off, iws_off, attn_off, total;
     csa2_status s = group_layout(g, layers, n_layers, &idx_off, &pool_off, &iws_off, &attn_off, &total);
     if (s != CSA2_OK) return s;
@@ -422,6 +445,7 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     bool merge_pending[2] = {false, false};
     for (int l = 0; l < n_layers; ++l) {
         const csa2_layer_desc &L = layers[l];
+        const Range layer_range(layer_range_name(L.mode));
         if (L.ready_event) {
             cudaError_t e = cudaStreamWaitEvent(st, reinterpret_cast<cudaEvent_t>(L.ready_event), 0);
             if (e != cudaSuccess) return cuda_status(e);
