@@ -201,6 +201,10 @@ CSA2_API csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uin
  *   swa_start[r] .. swa_start[r]+swa_len[r]-1 of its sequence (swa_start NULL = 0);
  *   out [B*T][H][D] of out_dtype (CSA2_DTYPE_F32 or CSA2_DTYPE_BF16); lse f32 [B*T][H]
  *   or NULL.
+ * Caller contract (not checked on the device): every non-negative id in idx names an entry
+ *   of its own sequence (id < that sequence's entry count, so the row lies inside kv), and
+ *   swa_start[r] + swa_len[r] <= swa_cap.  csa2_index_topk's outputs always satisfy the
+ *   first condition.
  * Limits: D == 512; H a multiple of 16, 16 <= H <= CSA2_MAX_HEADS; 1 <= K <=
  *   CSA2_MAX_TOPK; swa_len <= CSA2_SWA_WINDOW; kv and kv_row_stride 16-byte aligned.
  * Workspace: csa2_sparse_attn_workspace_size(B*T, H, K, &bytes).
