@@ -58,13 +58,22 @@ ATTN_TRAFFIC_BYTES = 29_462_272 + 256_256
 ATTN_TRAFFIC_SOURCE = "ncu --set full capture, profiles/attn_tc_decode128k_b32.md"
 
 
+def visible_counts(wl, b):
+    """Entries each query of sequence b can select, for the byte and flop accounting: entry j
+    covers tokens 4j..4j+3 and is visible at token p when 4j + 3 <= p (decode: all)."""
+    import numpy as np
+    if wl.prefill_start is None:
+        return np.array([wl.n_entries[b]], np.int64)
+    return np.minimum((wl.q_pos(b) + 1) // 4, wl.n_entries[b])
+
+
 def attn_work(wl, out_bytes):
     """Bytes and flops of one csa2_sparse_attn call over the workload."""
     from compressed_sparse_attention_quantize_b200 import synth
     byts = 0
     flops = 0
     for b in range(wl.B):
-        nvis = wl.n_visible(b)
+        nvis = visible_counts(wl, b)
         _, swl = synth.swa_window(wl, b)
         for t in range(wl.T):
             sel = min(wl.K, int(nvis[t]))
@@ -78,7 +87,7 @@ def index_work(wl):
     """Bytes of one Full-mode csa2_index_topk call (keys scanned + queries + selection written)."""
     byts = 0
     for b in range(wl.B):
-        nvis = wl.n_visible(b)
+        nvis = visible_counts(wl, b)
         for t in range(wl.T):
             byts += int(nvis[t]) * 36 + wl.HI * 40 + wl.K * 4
             if wl.P:

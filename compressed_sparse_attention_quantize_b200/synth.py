@@ -59,12 +59,6 @@ class Workload:
             return np.array([self.ctx_tokens[b] - 1], np.int64)
         return self.prefill_start + np.arange(self.T, dtype=np.int64)
 
-    def n_visible(self, b: int) -> np.ndarray:
-        """Entries visible to each query of sequence b (entry j covers tokens 4j..4j+3)."""
-        if self.prefill_start is None:
-            return np.array([self.n_entries[b]], np.int64)
-        return np.minimum((self.q_pos(b) + 1) // TOKENS_PER_ENTRY, self.n_entries[b])
-
     def swa_tokens(self) -> int:
         """Sliding-window slots held per sequence per layer."""
         if self.prefill_start is None:

@@ -285,6 +285,27 @@ def attention(q_bf16: np.ndarray, kv_rows: np.ndarray, idx: np.ndarray,
 
 
 # --------------------------------------------------------------------------
+# causal visibility (prefill)
+# --------------------------------------------------------------------------
+TOKENS_PER_ENTRY = 4
+
+
+def visible_entries(q_pos: Optional[int], n_entries: int) -> int:
+    """Number of compressed entries a query may select.
+
+    [B: CSA2：三层压缩一次吃满]: along the sequence every few tokens (4 in these workloads)
+    become one compressed entry.  Reading: entry j summarises tokens 4j..4j+3 and exists for
+    the query at absolute token position p only when all four are known, i.e. when
+    4j + 3 <= p.  Decode (q_pos None): the query follows the whole context, so every entry
+    is visible.  Written out as the definition: count the entries j < n_entries that pass.
+    """
+    if q_pos is None:
+        return int(n_entries)
+    j = np.arange(int(n_entries), dtype=np.int64)
+    return int(np.count_nonzero(TOKENS_PER_ENTRY * j + (TOKENS_PER_ENTRY - 1) <= int(q_pos)))
+
+
+# --------------------------------------------------------------------------
 # layer group (mode table)
 # --------------------------------------------------------------------------
 FULL, REINDEX, REUSE = "F", "I", "U"

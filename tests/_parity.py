@@ -50,7 +50,8 @@ class OracleSeq:
             else:
                 L = self.layer(l)
                 inputs.append((L["qc"][t], L["qs"][t], L["w"][t]))
-        n_vis = int(wl.n_visible(self.b)[t])
+        qp = None if wl.prefill_start is None else int(wl.q_pos(self.b)[t])
+        n_vis = oracle.visible_entries(qp, wl.n_entries[self.b])
         return oracle.layer_group_indices(modes, inputs, self.k_codes, self.k_scales, n_vis, wl.K,
                                           wl.P)
 

@@ -194,7 +194,7 @@ def test_prefill_scaled():
     r = _run_group(wl)
     _check_rows(r, wl, [0, 1, 2, 3, 47, 95])
     # causal: no selected entry lies beyond the query's visible range
-    nv = wl.n_visible(0)
+    nv = [oracle.visible_entries(int(p), wl.n_entries[0]) for p in wl.q_pos(0)]
     idx = r.layer_data[0]["idx"].cpu().numpy()
     for t in range(wl.T):
         assert idx[t].max() < nv[t]

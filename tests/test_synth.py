@@ -22,8 +22,8 @@ def test_workloads():
     w3 = synth.workload(3)
     assert w3.B == 4 and all(131072 <= n <= 262144 for n in w3.n_entries)
     w4 = synth.workload(4)
-    nv = w4.n_visible(0)
-    assert nv[0] == 32768 and nv[-1] == 33792
+    qp = w4.q_pos(0)
+    assert qp[0] == 4 * 32768 and qp[-1] == 4 * 32768 + 4095
     st, ln = synth.swa_window(w4, 0)
     assert st[0] == 0 and ln[0] == 128 and st[-1] == 4095
     w1 = synth.workload(1)
