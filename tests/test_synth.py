@@ -29,3 +29,18 @@ def test_workloads():
     w1 = synth.workload(1)
     st, ln = synth.swa_window(w1, 0)
     assert ln[0] == 128 and w1.modes == ("F", "U", "U", "U", "U", "U")
+
+
+def test_window_extents_follow_the_reading():
+    """Window slots [start, start + len) of query t hold tokens max(0, p - 127) .. p (prefill:
+    slot s holds token prefill_start - 127 + s); decode sees the whole filled ring."""
+    wl = synth.scaled(synth.workload(4), n=2000, T=96, K=256, name="prefill_scaled")
+    first = wl.prefill_start - (synth.SWA_WINDOW - 1)
+    st, ln = synth.swa_window(wl, 0)
+    for t, p in enumerate(wl.q_pos(0)):
+        tokens = first + np.arange(st[t], st[t] + ln[t])
+        assert tokens[0] == max(0, int(p) - 127) and tokens[-1] == p and ln[t] == min(128, int(p) + 1)
+        assert st[t] + ln[t] <= wl.swa_tokens()
+    w1 = synth.workload(1)
+    st, ln = synth.swa_window(w1, 3)
+    assert st[0] == 0 and ln[0] == 128
