@@ -6,16 +6,20 @@ selected entries plus the sliding window).  The arithmetic lives in
 ``csa2_oracle.c``; this module loads it with ctypes and composes the layer
 modes in plain Python.
 
-Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this package.  It imports nothing from the CUDA
-library and the library never imports it.
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline and
+reference legs of ``bench.py`` may import this package.  It imports nothing
+from the CUDA library and the library never imports it.
 
 Sources (web pages about the DeepSeek V4.1 Flash report):
   [A] "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径"
   [B] "DeepSeek V4.1 Flash 如何靠压缩 KV 缓存实现小模型干翻大模型"
 
 Every function here is pinned by a ``-m "not gpu"`` test in
-``tests/test_oracle_*.py`` except where its docstring says "parity unpinned".
+``tests/test_oracle_*.py``.  Parity unpinned: the pool that ``full_index``
+builds (the top-min(P, n) of the Full layer's own order) is pinned as that
+reading (it holds the top-K; Reindex over the whole context gives the Full
+selection), but the pages do not say how the model forms or refreshes its
+pool, so nothing pins the reading itself.
 """
 from __future__ import annotations
 

@@ -13,9 +13,14 @@
  *
  * Precision.  The pages fix the storage formats (E2M1 codes, one E4M3 scale
  * per 16 channels, an 8-bit sliding window).  Quantisers therefore round the
- * exact quotient once: they divide in fp64, and a short argument (kept with
- * the design notes) shows that an fp64 quotient of fp32 operands never lands
- * on a rounding midpoint unless the exact quotient is one.  Indexer scores are
+ * exact quotient once.  They divide in fp64, and that is enough.  Take a
+ * rounding midpoint m of E2M1 or E4M3 (at most 5 significant bits) and fp32
+ * operands a, b (24 bits).  If a != b*m, then a - b*m is a nonzero multiple of
+ * the smaller of a's lowest significand bit and the product of b's and m's.
+ * That step is at least about 2^-29 |b*m|, so |a/b - m| is at least about
+ * 2^-29 |m|, while the fp64 quotient errs by at most 2^-53 |a/b|.  The fp64
+ * quotient therefore lies on the same side of every midpoint as the exact
+ * one, and equals a midpoint only when the exact quotient does.  Indexer scores are
  * fp32 in one fixed summation order, because an integer decision (the top-K
  * set) hangs on them and both sides must take it in the same precision.
  * Attention is computed in fp64.
