@@ -2,8 +2,8 @@
  * CSA2 reference oracle -- TEST INFRASTRUCTURE ONLY.
  *
  * A plain, slow, obviously-correct CPU restatement of what the CSA2 hot path
- * computes.  Only the test-suite, the smoke check and the CPU-baseline leg of
- * the benchmark may load it.  It shares no code, header, table or constant
+ * computes.  Only the test-suite, the smoke check and the CPU-baseline and
+ * reference legs of the benchmark may load it.  It shares no code, header, table or constant
  * generator with the CUDA library, and the library never calls it.
  *
  * Sources (web pages about the DeepSeek V4.1 Flash report):
