@@ -59,7 +59,7 @@ typedef enum csa2_status {
 #define CSA2_MODE_REINDEX 1
 #define CSA2_MODE_REUSE   2
 
-/* Limits of this build. */
+/* Limits of this library. */
 #define CSA2_LATENT_DIM   512     /* main-KV latent width (attention)            */
 #define CSA2_INDEX_DIM    64      /* indexer key / query width                   */
 #define CSA2_MAX_INDEX_HEADS 16
