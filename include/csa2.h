@@ -12,7 +12,11 @@
  *    caller's `workspace`, sized by the matching *_workspace_size call).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
  *    call only enqueues work on it: nothing synchronises the host, so results are valid
- *    once the caller synchronises the stream.  Calls are stateless and thread-safe.
+ *    once the caller synchronises the stream.  Calls keep no data between calls.  The
+ *    library sets up, on its first calls, per-process launch settings (kernels' shared-
+ *    memory limits, the SM count, the layer group's side stream per thread).  Make the
+ *    first call of each kind from one thread, and drive one GPU per process; after that,
+ *    calls from several threads on their own streams are safe.
  *  - Arguments are validated before anything is launched; a call that returns an error
  *    has enqueued nothing.  Faults that happen on the device surface at the caller's
  *    next synchronisation, as for any CUDA kernel.
