@@ -19,7 +19,7 @@ __all__ = [
     "csa2_quantize_kv", "csa2_compress_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
     "csa2_index_topk_scored", "csa2_topk_merge_shards", "csa2_topk_merge_shards_workspace_size",
     "csa2_attn_merge_shards", "csa2_sparse_attn_shard",
-    "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_noalloc",
+    "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_plan", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error", "csa2_selftest_bounded_wait",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
     "FMT_FP4", "FMT_FP8_TOKEN", "DTYPE_F32", "DTYPE_BF16", "MODE_FULL", "MODE_REINDEX",
@@ -112,6 +112,9 @@ def lib():
     L.csa2_index_topk.argtypes = [_i32, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _vp, _i64,
                                   _vp, _vp, _i64, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _vp,
                                   _vp, _vp, _sz, _vp]
+    L.csa2_sparse_attn_plan.restype = _i32
+    L.csa2_sparse_attn_plan.argtypes = [_i32, _i32, _i32, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
+                                        ctypes.POINTER(_i32)]
     L.csa2_sparse_attn_workspace_size.restype = _i32
     L.csa2_sparse_attn_workspace_size.argtypes = [_i32, _i32, _i32, ctypes.POINTER(_sz)]
     L.csa2_sparse_attn.restype = _i32
@@ -242,6 +245,13 @@ def csa2_index_topk(mode, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_strid
                                  _ptr(pool_len), P_in, K, _ptr(out_idx), _ptr(out_cnt), P,
                                  _ptr(out_pool), _ptr(out_pool_len), _ptr(workspace), ws_bytes,
                                  _stream(stream)))
+
+
+def csa2_sparse_attn_plan(rows, H, K):
+    """(hgroups, splits, keys_per_split) of a csa2_sparse_attn launch on the current device."""
+    hg, sp, kps = _i32(0), _i32(0), _i32(0)
+    _check(lib().csa2_sparse_attn_plan(rows, H, K, ctypes.byref(hg), ctypes.byref(sp), ctypes.byref(kps)))
+    return hg.value, sp.value, kps.value
 
 
 def csa2_sparse_attn_workspace_size(rows, H, K) -> int:

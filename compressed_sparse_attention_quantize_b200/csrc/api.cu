@@ -272,6 +272,13 @@ csa2_status csa2_attn_merge_shards(const float *outs, const float *lses, int G, 
     return cuda_status(launch_attn_merge_shards(outs, lses, G, rows, H, D, out, out_dtype, lse, as_stream(stream)));
 }
 
+csa2_status csa2_sparse_attn_plan(int rows, int H, int K, int *hgroups, int *splits, int *keys_per_split) {
+    if (!hgroups || !splits || !keys_per_split) return CSA2_ERR_INVALID_ARG;
+    if (rows <= 0 || H <= 0 || K <= 0) return CSA2_ERR_SHAPE;
+    attn_plan(rows, H, K, *hgroups, *splits, *keys_per_split);
+    return CSA2_OK;
+}
+
 csa2_status csa2_sparse_attn_workspace_size(int rows, int H, int K, size_t *bytes) {
     if (!bytes) return CSA2_ERR_INVALID_ARG;
     if (rows <= 0 || H <= 0 || K <= 0) return CSA2_ERR_SHAPE;

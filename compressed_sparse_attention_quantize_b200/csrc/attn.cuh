@@ -36,9 +36,11 @@ cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st);
 cudaError_t launch_attn_tc_side_merge(AttnArgs a, cudaStream_t st, cudaStream_t side, cudaEvent_t attn_done,
                                       bool *merged);
 size_t tc_workspace_bytes(int rows, int H, int K);
+void tc_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_split);
 
 // Dispatch used by the C ABI.
 size_t attn_workspace_bytes(int rows, int H, int K);
+void attn_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_split);
 cudaError_t launch_attn(AttnArgs a, cudaStream_t st);
 
 }  // namespace csa2

@@ -216,6 +216,21 @@ CSA2_API csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uin
  * ---------------------------------------------------------------------------------- */
 CSA2_API csa2_status csa2_sparse_attn_workspace_size(int rows, int H, int K, size_t *bytes);
 
+/* ------------------------------------------------------------------------------------
+ * csa2_sparse_attn_plan -- how csa2_sparse_attn splits a launch of `rows` query rows,
+ * H heads and top-K on the current device (read-only; launches nothing).
+ *   hgroups: head groups of 64 (one CTA each per row and split);
+ *   splits: key splits per (row, head group), merged by log-sum-exp when > 1;
+ *   keys_per_split: keys per split, a multiple of 128; the last split takes the rest of
+ *     the K + CSA2_SWA_WINDOW keys.
+ * The plan minimises an estimated finish time over the device's SMs (148 assumed when no
+ * device is visible).  The workspace holds one partial of 131,584 bytes per (row, head
+ * group, split) when splits > 1.
+ * Errors: INVALID_ARG (NULL outputs), SHAPE (rows, H or K <= 0).
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_sparse_attn_plan(int rows, int H, int K, int *hgroups, int *splits,
+                                           int *keys_per_split);
+
 CSA2_API csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D,
                              const uint8_t *kv, int64_t kv_row_stride, const int64_t *seq_start,
                              const int32_t *idx, const int32_t *cnt, int K,

@@ -147,3 +147,29 @@ def test_layer_group_mode_table_validation(L):
     g, layers = _group([F, U])
     arr = (csa2.LayerDesc * 2)(*layers)
     assert L.csa2_layer_group(ctypes.byref(g), arr, 2, 16, 8, None) == WS
+
+
+def test_attention_plan_invariants():
+    """The split plan covers the K + window keys with no empty split, in whole 128-key tiles,
+    and the workspace query holds exactly one partial per (row, head group, split)."""
+    part = (2 * 64 + 64 * 512) * 4
+    for rows in (1, 3, 32, 148, 149, 1000, 4096):
+        for H in (16, 32, 64, 128):
+            for K in (1, 64, 2048, 4096):
+                hg, sp, kps = csa2.csa2_sparse_attn_plan(rows, H, K)
+                keys = K + 128
+                assert hg == -(-H // 64)
+                assert kps > 0 and kps % 128 == 0 and sp >= 1
+                assert sp * kps >= keys and (sp - 1) * kps < keys, (rows, H, K, sp, kps)
+                ws = csa2.csa2_sparse_attn_workspace_size(rows, H, K)
+                assert ws == (256 if sp == 1 else rows * hg * sp * part + 256), (rows, H, K)
+    # few rows split the keys finely; enough rows to fill the SMs take one split
+    assert csa2.csa2_sparse_attn_plan(1, 64, 2048)[1] > csa2.csa2_sparse_attn_plan(64, 64, 2048)[1]
+    assert csa2.csa2_sparse_attn_plan(4096, 64, 2048)[1] == 1
+
+
+def test_attention_plan_validation():
+    with pytest.raises(csa2.CSA2Error):
+        csa2.csa2_sparse_attn_plan(0, 64, 2048)
+    with pytest.raises(csa2.CSA2Error):
+        csa2.csa2_sparse_attn_plan(32, 64, 0)
