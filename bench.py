@@ -534,6 +534,9 @@ def run_csa2(args, wl):
         t_ms = statistics.mean(bd["index_topk"])
         kernels["index_topk"] = {"launches_per_step": 1, "avg_ms": t_ms, "algorithmic_bytes": ib,
                                  "achieved_gbs": ib / (t_ms * 1e-3) / 1e9}
+    for k in kernels.values():
+        k["hbm_frac"] = k["achieved_gbs"] / hbm_peak
+        k["hbm_frac_of_nominal_8tbs"] = k["achieved_gbs"] / 8000.0
     tot = sum(k["avg_ms"] * k["launches_per_step"] for k in kernels.values())
     for k in kernels.values():
         k["share"] = k["avg_ms"] * k["launches_per_step"] / tot if tot else None
