@@ -31,3 +31,18 @@ def test_prefill_workload_ends():
     n = wl.n_entries[0]
     assert oracle.visible_entries(int(qp[0]), n) == 32768        # the chunk's first token
     assert oracle.visible_entries(int(qp[-1]), n) == 33792       # all 1024 new entries complete
+
+
+def test_bench_accounting_matches_the_oracle():
+    """bench.py counts algorithmic bytes with its own copy of the rule; it must agree."""
+    import bench
+    for i in range(5):
+        wl = synth.workload(i)
+        for b in range(wl.B):
+            got = bench.visible_counts(wl, b)
+            if wl.prefill_start is None:
+                assert got.tolist() == [oracle.visible_entries(None, wl.n_entries[b])]
+            else:
+                qp = wl.q_pos(b)
+                for t in (0, 1, 2, 3, len(qp) // 2, len(qp) - 1):
+                    assert int(got[t]) == oracle.visible_entries(int(qp[t]), wl.n_entries[b])
