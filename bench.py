@@ -67,6 +67,32 @@ def visible_counts(wl, b):
     return np.minimum((wl.q_pos(b) + 1) // 4, wl.n_entries[b])
 
 
+STEP_WRITES = ("quantise-on-write inside the step: the newest compressed entry (FP4) and its indexer "
+               "key (FP4) of every sequence, every Full/Reindex layer's indexer query (FP4), every "
+               "layer's window entry of the step token (E4M3); an entry is written every step, an "
+               "upper bound on the one completed every 4th token")
+
+
+def write_calls(runner):
+    """Library calls of one write_step()."""
+    n = (2 if runner.step_rows is not None else 0) + (1 if runner.step_win_rows is not None else 0)
+    return n + sum(1 for ld in runner.layer_data if "iq_f32" in ld)
+
+
+def write_work(runner):
+    """Bytes of one write_step(): float rows and destination rows read, quantised rows written."""
+    byts = 0
+    if runner.step_rows is not None:
+        m = runner.step_rows.numel()
+        byts += m * (512 * 4 + 288 + 8) + m * (64 * 4 + 36 + 8)
+    if runner.step_win_rows is not None:
+        byts += runner.step_win_rows.numel() * (512 * 4 + 516 + 8)
+    for ld in runner.layer_data:
+        if "iq_f32" in ld:
+            byts += ld["iq_f32"].shape[0] * (64 * 4 + 36)
+    return byts
+
+
 def attn_work(wl, out_bytes):
     """Bytes and flops of one csa2_sparse_attn call over the workload."""
     from compressed_sparse_attention_quantize_b200 import synth
@@ -246,8 +272,9 @@ def time_steps(torch, step, steps, flush):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-def breakdown(torch, csa2, runner, steps, flush):
-    """Per-call device times of the decomposed group: csa2_index_topk + csa2_sparse_attn per layer."""
+def breakdown(torch, csa2, runner, steps, flush, writes=False):
+    """Per-call device times of the decomposed step: the step's writes (one mark around all of
+    them), then csa2_index_topk + csa2_sparse_attn per layer."""
     wl = runner.wl
     g = runner.g
     dev = runner.workspace.device
@@ -263,7 +290,7 @@ def breakdown(torch, csa2, runner, steps, flush):
     aws_bytes = csa2.csa2_sparse_attn_workspace_size(rows, wl.H, wl.K)
     aws = torch.empty((aws_bytes,), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
-    times = {"index_topk": [], "reindex_topk": [], "sparse_attn": []}
+    times = {"step_writes": [], "index_topk": [], "reindex_topk": [], "sparse_attn": []}
     for _ in range(steps):
         flush()
         marks = []
@@ -271,6 +298,10 @@ def breakdown(torch, csa2, runner, steps, flush):
             e = torch.cuda.Event(enable_timing=True)
             e.record(st)
             return e
+        if writes:
+            e0 = ev()
+            runner.write_step()
+            marks.append(("step_writes", e0, ev()))
         for l, m in enumerate(runner.modes):
             ld = runner.layer_data[l]
             if m != "U":
@@ -371,10 +402,11 @@ def topk_side_reference(torch, csa2, wl, flush, reps=10):
             "note": "csa2_topk_merge_shards (one shard) vs torch.topk(sorted=False); L2 flushed before each call"}
 
 
-def e2e_measure(torch, csa2, runner, steps, warmup, flush):
+def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     """The metric through csa2_layer_group with host buffers.  Per step: every layer's main query
     (bf16) and indexer query/weights (fp32) are copied from pinned host memory on a copy stream,
-    layer by layer (the indexer queries are quantised there too), and each layer of the group
+    layer by layer (the indexer queries are quantised there too; with ``writes`` the step's new
+    entry and window latents are copied and quantised there as well), and each layer of the group
     waits only for its own inputs (the group's per-layer ready events), so the copies of later
     layers overlap the work of earlier ones; the last layer's output is read back at the end.
     Steps do not overlap: the copy stream starts a step after the previous step's work."""
@@ -389,7 +421,16 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
 
     host = []
     h2d = 0
+    step_host = None
     with gpu_local_cpus(torch) as local:
+        if writes:
+            step_host = {}
+            if runner.step_rows is not None:
+                step_host["kv"] = pinned_copy(runner.step_kv.cpu())
+                step_host["ik"] = pinned_copy(runner.step_ik.cpu())
+            if runner.step_win_rows is not None:
+                step_host["win"] = pinned_copy(runner.step_win_lat.cpu())
+            h2d += sum(t.numel() * 4 for t in step_host.values())
         for l, m in enumerate(runner.modes):
             ld = runner.layer_data[l]
             hq = pinned_copy(ld["q"].cpu())
@@ -416,6 +457,14 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush):
     def body(main):
         copy_stream.wait_stream(main)
         with torch.cuda.stream(copy_stream):
+            if step_host is not None:                 # the step's new entries and window tokens
+                if "kv" in step_host:
+                    runner.step_kv.copy_(step_host["kv"], non_blocking=True)
+                    runner.step_ik.copy_(step_host["ik"], non_blocking=True)
+                if "win" in step_host:
+                    runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
+                runner.write_entries(stream=copy_stream)
+                runner.write_windows(stream=copy_stream)
             for l, m in enumerate(runner.modes):
                 ld, e = runner.layer_data[l], host[l]
                 ld["q"].copy_(e["q"], non_blocking=True)
@@ -482,11 +531,22 @@ def run_csa2(args, wl):
     def flush():
         flush_buf.fill_(1)
 
-    # the timed step replays the whole layer group as one CUDA graph (--eager: one C call per step)
-    step_fn = runner.run
+    # the timed step: the step's quantise-on-write (newest entry and indexer key per sequence,
+    # indexer queries, window entries of the step token), then the layer group; replayed as one
+    # CUDA graph (--eager: one call each per step).  If the writes fail on their first run (an
+    # argument the library rejects), the step falls back to the group alone and says so.
+    writes = True
+    writes_note = STEP_WRITES
+    try:
+        runner.write_step()
+        torch.cuda.synchronize()
+    except Exception as exc:
+        writes = False
+        writes_note = f"not run: {type(exc).__name__}: {exc}"[:300]
+    step_fn = runner.step if writes else runner.run
     graph_kernels = 0
     if not args.eager:
-        graph_kernels = runner.capture()
+        graph_kernels = runner.capture(with_writes=writes)
         step_fn = runner.replay
     for _ in range(args.warmup):
         flush()
@@ -520,7 +580,7 @@ def run_csa2(args, wl):
         return
 
     # per-call breakdown and roofline of the dominant kernel
-    bd = breakdown(torch, csa2, runner, max(3, min(args.steps, 10)), flush)
+    bd = breakdown(torch, csa2, runner, max(3, min(args.steps, 10)), flush, writes)
     ab, af = attn_work(wl, 2 if runner.out_dtype == csa2.DTYPE_BF16 else 4)
     ib = index_work(wl)
     kernels = {}
@@ -530,6 +590,11 @@ def run_csa2(args, wl):
                                   "share": None, "algorithmic_bytes": ab, "algorithmic_flops": af,
                                   "achieved_gbs": ab / (t_ms * 1e-3) / 1e9,
                                   "achieved_tflops": af / (t_ms * 1e-3) / 1e12}
+    if "step_writes" in bd:
+        t_ms = statistics.mean(bd["step_writes"])
+        wb = write_work(runner)
+        kernels["step_writes"] = {"launches_per_step": 1, "calls": write_calls(runner), "avg_ms": t_ms,
+                                  "algorithmic_bytes": wb, "achieved_gbs": wb / (t_ms * 1e-3) / 1e9}
     if "index_topk" in bd:
         t_ms = statistics.mean(bd["index_topk"])
         kernels["index_topk"] = {"launches_per_step": 1, "avg_ms": t_ms, "algorithmic_bytes": ib,
@@ -555,7 +620,7 @@ def run_csa2(args, wl):
                 "peak": hbm_peak, "unit": "GB/s", "frac": k["achieved_gbs"] / hbm_peak,
                 "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
 
-    e2e = e2e_measure(torch, csa2, runner, max(3, min(args.steps, 10)), 2, flush)
+    e2e = e2e_measure(torch, csa2, runner, max(3, min(args.steps, 10)), 2, flush, writes)
     if world > 1:
         t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -580,6 +645,7 @@ def run_csa2(args, wl):
                            "entries_per_seq": wl.n_entries[0], "layers": ",".join(wl.modes),
                            "heads": wl.H, "index_heads": wl.HI, "topk": wl.K, "pool": wl.P,
                            "swa": 128, "out": "bf16", "step": "eager" if args.eager else "cuda graph",
+                           "step_writes": writes_note,
                            "parallelism": f"replicas x{world} (independent sequences)",
                            "l2": "flushed between steps (256 MB write, outside the events)"},
                 "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,

@@ -63,15 +63,27 @@ class GroupRunner:
         self.kv = torch.empty((max(total, 1), KV_ROW), dtype=torch.uint8, device=d)
         self.k_codes = torch.empty((max(total, 1), 32), dtype=torch.uint8, device=d)
         self.k_scales = torch.empty((max(total, 1), 4), dtype=torch.uint8, device=d)
-        # caches: quantise-on-write, one sequence at a time (bounds host memory)
+        # caches: quantise-on-write, one sequence at a time (bounds host memory); the newest
+        # entry of each sequence is kept in float for the per-step write (write_step)
+        step_kv, step_ik, step_rows = [], [], []
         for b in range(B):
             s0 = int(starts[b])
             lat = torch.from_numpy(synth.kv_latent(wl, b)).to(d)
             quantize_fp4_rows(lat, self.kv[s0:], self.kv[s0:, 256:], KV_ROW, KV_ROW)
+            if n[b] > 0:
+                step_kv.append(lat[n[b] - 1:n[b]].clone())
+                step_rows.append(s0 + n[b] - 1)
             del lat
             ik = torch.from_numpy(synth.index_keys(wl, b)).to(d)
             quantize_fp4_rows(ik, self.k_codes[s0:], self.k_scales[s0:], 32, 4)
+            if n[b] > 0:
+                step_ik.append(ik[n[b] - 1:n[b]].clone())
             del ik
+        self.step_kv = torch.cat(step_kv) if step_kv else None
+        self.step_ik = torch.cat(step_ik) if step_ik else None
+        self.step_rows = torch.tensor(step_rows, dtype=torch.int64, device=d) if step_rows else None
+        if step_rows:
+            assert max(step_rows) < self.kv.shape[0] and min(step_rows) >= 0
         # query positions (prefill) and window slots
         if wl.prefill_start is not None:
             qp = np.concatenate([wl.q_pos(b) for b in range(B)]).astype(np.int32)
@@ -82,6 +94,14 @@ class GroupRunner:
         self.swa_start = torch.from_numpy(np.concatenate(st).astype(np.int32)).to(d)
         self.swa_len = torch.from_numpy(np.concatenate(ln).astype(np.int32)).to(d)
         self.swa_cap = wl.swa_tokens()
+        # every layer's window in one buffer (layer l holds rows l*B*swa_cap ..), so that one
+        # scatter call writes all layers' window entries of a step
+        win_rows = B * self.swa_cap
+        self.swa_codes_all = torch.empty((len(modes) * win_rows, 512), dtype=torch.uint8, device=d)
+        self.swa_scale_all = torch.empty((len(modes) * win_rows,), dtype=torch.float32, device=d)
+        win_slots = self._step_window_slots()
+        assert all(0 <= x < win_rows for x in win_slots)
+        step_win_lat, step_win_rows = [], []
         # per layer
         self.layer_data = []
         odt = torch.float32 if out_dtype == DTYPE_F32 else torch.bfloat16
@@ -94,22 +114,48 @@ class GroupRunner:
                 ld["iq_codes"] = torch.empty((self.rows * HI, 32), dtype=torch.uint8, device=d)
                 ld["iq_scales"] = torch.empty((self.rows * HI, 4), dtype=torch.uint8, device=d)
                 quantize_fp4_rows(iqt, ld["iq_codes"], ld["iq_scales"], 32, 4)
+                ld["iq_f32"] = iqt
                 w = np.stack([synth.head_weights(wl, l, b) for b in range(B)]).reshape(self.rows, HI)
                 ld["iw"] = torch.from_numpy(np.ascontiguousarray(w)).to(d)
             sw = np.stack([synth.swa_latent(wl, l, b) for b in range(B)]).reshape(B * self.swa_cap, 512)
             swt = torch.from_numpy(sw).to(d)
-            ld["swa_codes"] = torch.empty((B * self.swa_cap, 512), dtype=torch.uint8, device=d)
-            ld["swa_scale"] = torch.empty((B * self.swa_cap,), dtype=torch.float32, device=d)
+            ld["swa_codes"] = self.swa_codes_all[l * win_rows:(l + 1) * win_rows]
+            ld["swa_scale"] = self.swa_scale_all[l * win_rows:(l + 1) * win_rows]
             quantize_fp8_rows(swt, ld["swa_codes"], ld["swa_scale"])
+            # the window entries of this step's tokens, for the per-step write
+            if win_slots:
+                step_win_lat.append(swt.index_select(0, torch.tensor(win_slots, dtype=torch.int64, device=d)))
+                step_win_rows.extend(l * win_rows + x for x in win_slots)
+            del swt
             ld["out"] = torch.empty((self.rows, H, 512), dtype=odt, device=d)
             ld["lse"] = torch.empty((self.rows, H), dtype=torch.float32, device=d)
             ld["idx"] = torch.empty((self.rows, K), dtype=torch.int32, device=d)
             self.layer_data.append(ld)
+        self.step_win_lat = torch.cat(step_win_lat).contiguous() if step_win_lat else None
+        self.step_win_rows = (torch.tensor(step_win_rows, dtype=torch.int64, device=d)
+                              if step_win_rows else None)
+        if step_win_rows:
+            assert max(step_win_rows) < self.swa_codes_all.shape[0]
         self.g = self._group_desc()
         self.layer_descs = [self._layer_desc(l) for l in range(len(modes))]
         self.ws_bytes = csa2_layer_group_workspace_size(self.g, self.layer_descs)
         self.workspace = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=d)
         torch.cuda.synchronize()
+
+    def _step_window_slots(self) -> List[int]:
+        """Rows b * swa_cap + slot of the window entries this step's tokens write.  Decode: the
+        128-slot ring holds token p in slot p % 128, so the current token is slot (ctx - 1) % 128
+        (none for an empty context).  Prefill: the buffer holds the 127 tokens before the chunk
+        and then the chunk, so chunk token t is slot 127 + t."""
+        wl = self.wl
+        out = []
+        for b in range(wl.B):
+            if wl.prefill_start is None:
+                if wl.ctx_tokens[b] > 0:
+                    out.append(b * self.swa_cap + (wl.ctx_tokens[b] - 1) % synth.SWA_WINDOW)
+            else:
+                out.extend(b * self.swa_cap + (synth.SWA_WINDOW - 1) + t for t in range(wl.T))
+        return out
 
     def _group_desc(self) -> GroupDesc:
         wl = self.wl
@@ -145,22 +191,61 @@ class GroupRunner:
     def run(self, stream=None) -> None:
         csa2_layer_group(self.g, self.layer_descs, self.workspace, self.ws_bytes, stream)
 
-    def capture(self) -> int:
-        """Record one call of the layer group into a CUDA graph (after a warm-up call, so the
-        library's one-time attribute set-up happens outside the capture); ``replay()`` then
-        launches the whole group with one graph launch.  Returns the number of library kernels
-        the graph holds.  The graph reads the current contents of the runner's buffers."""
+    def write_step(self, stream=None) -> None:
+        """A decode step's quantise-on-write, from float inputs held on the device: the newest
+        compressed entry of every sequence and its indexer key (FP4, written at its cache row),
+        every Full/Reindex layer's indexer query (FP4), and every layer's window entries of the
+        step's tokens (E4M3 + fp32 scale, at their window slots; one call for all layers).  The
+        inputs are the ones the caches were built from, so the bytes written equal those already
+        there and a step that runs write_step() then run() reads the same caches as run() alone."""
+        self.write_entries(stream)
+        self.write_windows(stream)
+        self.write_queries(stream)
+
+    def write_entries(self, stream=None) -> None:
+        """The newest compressed entry of every non-empty sequence (main KV, FP4) and its
+        indexer key (FP4), each written at its cache row."""
+        if self.step_rows is not None:
+            quantize_fp4_rows(self.step_kv, self.kv, self.kv[:, 256:], KV_ROW, KV_ROW,
+                              dst_rows=self.step_rows, stream=stream)
+            quantize_fp4_rows(self.step_ik, self.k_codes, self.k_scales, 32, 4,
+                              dst_rows=self.step_rows, stream=stream)
+
+    def write_windows(self, stream=None) -> None:
+        """Every layer's window entries of the step's tokens, in one scatter call."""
+        if self.step_win_rows is not None:
+            quantize_fp8_rows(self.step_win_lat, self.swa_codes_all, self.swa_scale_all,
+                              dst_rows=self.step_win_rows, stream=stream)
+
+    def write_queries(self, stream=None) -> None:
+        """Every Full/Reindex layer's indexer query (FP4)."""
+        for ld in self.layer_data:
+            if "iq_f32" in ld:
+                quantize_fp4_rows(ld["iq_f32"], ld["iq_codes"], ld["iq_scales"], 32, 4, stream=stream)
+
+    def step(self, stream=None) -> None:
+        """One whole decode step: the step's writes, then the layer group."""
+        self.write_step(stream)
+        self.run(stream)
+
+    def capture(self, with_writes: bool = False) -> int:
+        """Record one call of the layer group (preceded by the step's writes when
+        ``with_writes``) into a CUDA graph, after a warm-up call so that the library's one-time
+        attribute set-up happens outside the capture; ``replay()`` then launches it with one
+        graph launch.  Returns the number of library kernels the graph holds.  The graph reads
+        the current contents of the runner's buffers."""
         from . import csa2_launch_count
+        fn = self.step if with_writes else self.run
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
-            self.run()
+            fn()
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         n0 = csa2_launch_count()
         with torch.cuda.graph(graph):
-            self.run()
+            fn()
         self.graph = graph
         self.graph_kernels = csa2_launch_count() - n0
         return self.graph_kernels

@@ -344,3 +344,35 @@ def test_topk_heavy_ties_full_pool_reindex():
         op, opl = o_pools[b]
         oi, oc = oracle.reindex(qc2[b], qs2[b], w2[b], kc[s0:s0 + n[b]], ks[s0:s0 + n[b]], op, opl, K)
         assert int(cnt2[b]) == oc and np.array_equal(idx2[b].cpu().numpy(), oi), f"reindex row {b}"
+
+
+@pytest.mark.parametrize("case", ["ragged_decode", "prefill"])
+def test_step_writes_rewrite_identical_bytes(case):
+    """A step's quantise-on-write (newest entry + indexer key per sequence, indexer queries, the
+    step tokens' window entries) rewrites exactly the bytes the caches already hold, eagerly and
+    inside a captured step, so the timed step reads the same caches and gives the same outputs."""
+    if case == "ragged_decode":
+        wl = synth.scaled(synth.workload(1), B=4, n=[1000, 0, 37, 4500], K=64, H=32, name="ragged_writes")
+        r = _run_group(wl, layers=3)
+    else:
+        wl = synth.scaled(synth.workload(4), n=2000, T=96, K=256, name="prefill_writes")
+        r = _run_group(wl)
+
+    def snapshot():
+        bufs = [r.kv, r.k_codes, r.k_scales, r.swa_codes_all, r.swa_scale_all.view(torch.int32)]
+        bufs += [ld["iq_codes"] for ld in r.layer_data if "iq_codes" in ld]
+        bufs += [ld["iq_scales"] for ld in r.layer_data if "iq_scales" in ld]
+        bufs += [ld["out"].view(torch.int32) for ld in r.layer_data]
+        bufs += [ld["idx"] for ld in r.layer_data]
+        return [b.clone() for b in bufs]
+
+    base = snapshot()
+    r.step()
+    torch.cuda.synchronize()
+    for a, b in zip(base, snapshot()):
+        assert torch.equal(a, b)
+    r.capture(with_writes=True)
+    r.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(base, snapshot()):
+        assert torch.equal(a, b)
