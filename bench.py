@@ -3,13 +3,16 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference] [--config C]
 
-One step = one decode token of every sequence of the workload through the whole layer group
-(indexer + top-K of the Full layer, then attention of all six layers), i.e. every hot-path
-step.  Default workload: decode at 128K context, batch 32, 1 Full + 5 Reuse layers.
+One step = one decode token of every sequence of the workload through the whole hot path: the
+step's quantise-on-write, then the layer group (indexer + top-K of the Full layer, Reindex
+re-scoring where the mode table has it, and attention of every layer).  Default workload:
+decode at 128K context, batch 32, 1 Full + 5 Reuse layers (the headline line).  The same line
+carries, under "workloads", the same measurement of the other timed workloads: decode at 1M
+context (batch 4), the Reindex group at 256K (batch 16) and the prefill chunk (4096 queries).
 
 Printed (rank 0, one JSON line): value = queries/s over all ranks (device time, CUDA events on
 the launch stream, L2 flushed by a 256 MB write between steps, max over ranks); e2e = the same
-metric through csa2_layer_group with host buffers (host->device copies of the step's queries and
+metric through csa2_layer_group with host buffers (host->device copies of the step's inputs and
 the device->host read of the last layer's output inside the timed region); roofline of the
 dominant kernel; cpu_baseline = the oracle on the host cores over a bounded sample.
 
@@ -51,11 +54,28 @@ def _peaks():
 # ------------------------------------------------------------------------------------------
 # algorithmic work per call (bytes that must move; flops of the contraction)
 # ------------------------------------------------------------------------------------------
-# DRAM bytes (read + write) of one attn_tc_kernel launch on this workload, from an ncu capture of
-# the current kernel (dram__bytes_read.sum + dram__bytes_write.sum); set to None whenever the
-# kernel changes until it is captured again.
-ATTN_TRAFFIC_BYTES = 29_462_272 + 256_256
-ATTN_TRAFFIC_SOURCE = "ncu --set full capture, profiles/attn_tc_decode128k_b32.md"
+# DRAM bytes (read + write) of one attn_tc_kernel launch on the 128K decode workload, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum), together with the SHA-256 of the kernel
+# source it was taken on: when the source has changed since, the figure is stale and the line
+# reports traffic null.
+ATTN_TRAFFIC = {"bytes": None, "source_sha256": None,
+                "capture": "ncu --set full --clock-control none -k regex:attn_tc -s 5 -c 2 python bench.py "
+                           "--config 1 --entries 16384 --steps 2 --warmup 3 --quick --no-cpu-baseline --eager"}
+ATTN_SOURCE = os.path.join(ROOT, "compressed_sparse_attention_quantize_b200", "csrc", "attn_tc.cu")
+
+
+def attn_traffic():
+    """(bytes or None, note): the captured DRAM traffic of one attention launch if it was taken
+    on the current kernel source."""
+    import hashlib
+    try:
+        with open(ATTN_SOURCE, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None, "kernel source not found"
+    if ATTN_TRAFFIC["bytes"] is None or ATTN_TRAFFIC["source_sha256"] != sha:
+        return None, "no capture of the current kernel source"
+    return ATTN_TRAFFIC["bytes"], ATTN_TRAFFIC["capture"]
 
 
 def visible_counts(wl, b):
@@ -74,9 +94,8 @@ STEP_WRITES = ("quantise-on-write inside the step: the newest compressed entry (
 
 
 def write_calls(runner):
-    """Library calls of one write_step()."""
-    n = (2 if runner.step_rows is not None else 0) + (1 if runner.step_win_rows is not None else 0)
-    return n + sum(1 for ld in runner.layer_data if "iq_f32" in ld)
+    """Library calls of one write_step(): one csa2_quantize_kv_batch launch."""
+    return 1 if (runner.entry_jobs or runner.window_jobs or runner.query_jobs) else 0
 
 
 def write_work(runner):
@@ -118,6 +137,18 @@ def index_work(wl):
             byts += int(nvis[t]) * 36 + wl.HI * 40 + wl.K * 4
             if wl.P:
                 byts += wl.P * 4
+    return byts
+
+
+def reindex_work(wl):
+    """Bytes of one Reindex csa2_index_topk call (pool ids and the gathered keys they name,
+    queries, selection written)."""
+    byts = 0
+    for b in range(wl.B):
+        nvis = visible_counts(wl, b)
+        for t in range(wl.T):
+            pool = min(wl.P, int(nvis[t]))
+            byts += pool * (4 + 36) + wl.HI * 40 + wl.K * 4
     return byts
 
 
@@ -273,10 +304,10 @@ def time_steps(torch, step, steps, flush):
 
 
 def breakdown(torch, csa2, runner, steps, flush, writes=False):
-    """Per-call device times of the decomposed step: the step's writes (one mark around all of
-    them), then csa2_index_topk + csa2_sparse_attn per layer."""
+    """Per-call device times of the decomposed step: the step's writes (one csa2_quantize_kv_batch
+    launch, replayed from a one-node CUDA graph so that host launch overhead is not counted),
+    then csa2_index_topk + csa2_sparse_attn per layer."""
     wl = runner.wl
-    g = runner.g
     dev = runner.workspace.device
     rows = runner.rows
     idx = torch.empty((rows, wl.K), dtype=torch.int32, device=dev)
@@ -290,6 +321,14 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
     aws_bytes = csa2.csa2_sparse_attn_workspace_size(rows, wl.H, wl.K)
     aws = torch.empty((aws_bytes,), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
+    write_graph = None
+    if writes:
+        runner.write_step()
+        torch.cuda.synchronize()
+        write_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(write_graph):
+            runner.write_step()
+        torch.cuda.synchronize()
     times = {"step_writes": [], "index_topk": [], "reindex_topk": [], "sparse_attn": []}
     for _ in range(steps):
         flush()
@@ -298,9 +337,9 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
             e = torch.cuda.Event(enable_timing=True)
             e.record(st)
             return e
-        if writes:
+        if write_graph is not None:
             e0 = ev()
-            runner.write_step()
+            write_graph.replay()
             marks.append(("step_writes", e0, ev()))
         for l, m in enumerate(runner.modes):
             ld = runner.layer_data[l]
@@ -320,7 +359,8 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
                                          wl.K, idx, cnt, 0, None, None, iws, iws_bytes)
                     marks.append(("reindex_topk", e0, ev()))
             e0 = ev()
-            csa2.csa2_sparse_attn(ld["q"], wl.B, wl.T, wl.H, 512, runner.kv, 288, runner.seq_start, idx, cnt,
+            csa2.csa2_sparse_attn(ld["q"], wl.B, wl.T, wl.H, 512, runner.kv, 288, runner.seq_start,
+                                  runner.n_entries, idx, cnt,
                                   wl.K, ld["swa_codes"], ld["swa_scale"], runner.swa_cap, runner.swa_start,
                                   runner.swa_len, runner.softmax_scale, ld["out"], runner.out_dtype, ld["lse"],
                                   aws, aws_bytes)
@@ -328,6 +368,7 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
         torch.cuda.synchronize()
         for name, a, b in marks:
             times[name].append(a.elapsed_time(b))
+    del write_graph
     return {k: v for k, v in times.items() if v}
 
 
@@ -370,9 +411,10 @@ def topk_side_reference(torch, csa2, wl, flush, reps=10):
     """torch.topk next to the library's top-K on the same fp32 score buffer (side reference only).
 
     Scores: [rows][n] uniform on [0, 1), seeded; K of n per row.  The library's side is
-    csa2_topk_merge_shards with one shard holding the whole row, which also returns the
-    selection in ascending index order.  Both selections are checked to have the same
-    K-th largest score per row."""
+    csa2_topk_merge_shards with one shard holding the whole row (it selects from the list in
+    place with the cluster top-K kernel, one launch), which also returns the selection in
+    ascending index order.  Both selections are checked to have the same K-th largest score
+    per row."""
     rows, n, K = wl.B * wl.T, int(max(wl.n_entries)), wl.K
     g = torch.Generator(device="cuda")
     g.manual_seed(int(wl.seed) + 77)
@@ -463,8 +505,9 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
                     runner.step_ik.copy_(step_host["ik"], non_blocking=True)
                 if "win" in step_host:
                     runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
-                runner.write_entries(stream=copy_stream)
-                runner.write_windows(stream=copy_stream)
+                jobs = runner.entry_jobs + runner.window_jobs
+                if jobs:
+                    csa2.csa2_quantize_kv_batch(jobs, stream=copy_stream)
             for l, m in enumerate(runner.modes):
                 ld, e = runner.layer_data[l], host[l]
                 ld["q"].copy_(e["q"], non_blocking=True)
@@ -477,8 +520,27 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
         runner.run()
         out_host.copy_(out_last, non_blocking=True)
 
+    def copies_only():
+        """The step's host->device and device->host copies alone (same buffers, same order)."""
+        if step_host is not None:
+            if "kv" in step_host:
+                runner.step_kv.copy_(step_host["kv"], non_blocking=True)
+                runner.step_ik.copy_(step_host["ik"], non_blocking=True)
+            if "win" in step_host:
+                runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
+        for l, m in enumerate(runner.modes):
+            ld, e = runner.layer_data[l], host[l]
+            ld["q"].copy_(e["q"], non_blocking=True)
+            if m != "U":
+                e["iq_dev"].copy_(e["iq"], non_blocking=True)
+                ld["iw"].copy_(e["iw"], non_blocking=True)
+        out_host.copy_(out_last, non_blocking=True)
+
     graph = None
     try:
+        copies_only()
+        torch.cuda.synchronize()
+        copy_ms = statistics.median(time_steps(torch, copies_only, max(3, steps), lambda: None))
         for _ in range(warmup):
             flush()
             body(cur)
@@ -504,37 +566,86 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": sum(ms) / steps, "overlap": "per-layer input copies on a second stream",
+            "copy_ms_per_step": copy_ms, "copy_gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
+            "copy_note": "the step's copies alone, back to back on one stream (no kernels)",
             "step": "cuda graph" if graph is not None else "eager",
             "host_buffers": "GPU-local NUMA node" if local.used else "default placement"}
 
 
-def run_csa2(args, wl):
-    import torch
+def kernel_table(wl, runner, bd, peaks, out_bytes):
+    """Per-call times, algorithmic bytes/flops and HBM fractions of the decomposed step."""
+    hbm_peak = peaks[0]
+    ab, af = attn_work(wl, out_bytes)
+    kernels = {}
+    if "sparse_attn" in bd:
+        t_ms = statistics.mean(bd["sparse_attn"])
+        kernels["sparse_attn"] = {"launches_per_step": len(runner.modes), "avg_ms": t_ms,
+                                  "algorithmic_bytes": ab, "algorithmic_flops": af,
+                                  "achieved_gbs": ab / (t_ms * 1e-3) / 1e9,
+                                  "achieved_tflops": af / (t_ms * 1e-3) / 1e12}
+    if "step_writes" in bd:
+        t_ms = statistics.mean(bd["step_writes"])
+        wb = write_work(runner)
+        kernels["step_writes"] = {"launches_per_step": 1, "calls": write_calls(runner), "avg_ms": t_ms,
+                                  "algorithmic_bytes": wb, "achieved_gbs": wb / (t_ms * 1e-3) / 1e9}
+    if "index_topk" in bd:
+        t_ms = statistics.mean(bd["index_topk"])
+        ib = index_work(wl)
+        kernels["index_topk"] = {"launches_per_step": 1, "avg_ms": t_ms, "algorithmic_bytes": ib,
+                                 "achieved_gbs": ib / (t_ms * 1e-3) / 1e9}
+    if "reindex_topk" in bd:
+        t_ms = statistics.mean(bd["reindex_topk"])
+        rb = reindex_work(wl)
+        kernels["reindex_topk"] = {"launches_per_step": sum(1 for m in runner.modes if m == "I"), "avg_ms": t_ms,
+                                   "algorithmic_bytes": rb, "achieved_gbs": rb / (t_ms * 1e-3) / 1e9}
+    for k in kernels.values():
+        k["hbm_frac"] = k["achieved_gbs"] / hbm_peak
+        k["hbm_frac_of_nominal_8tbs"] = k["achieved_gbs"] / 8000.0
+    tot = sum(k["avg_ms"] * k["launches_per_step"] for k in kernels.values())
+    for k in kernels.values():
+        k["share"] = k["avg_ms"] * k["launches_per_step"] / tot if tot else None
+    return kernels
+
+
+def roofline(wl, kernels, peaks):
+    """Roofline object of the kernel with the largest share of the step."""
+    hbm_peak, tc_peak, _, peak_src = peaks
+    if not kernels:
+        return None
+    dom = max(kernels, key=lambda k: kernels[k]["share"] or 0)
+    k = kernels[dom]
+    if dom == "sparse_attn":
+        traffic, note = attn_traffic()
+        if wl.name != "decode_128k_b32_F5U" and traffic is not None:
+            traffic, note = None, "captured on the 128K decode workload only"
+        roof = {"kernel": "csa2_sparse_attn", "bound": "tensor", "achieved": k["achieved_tflops"],
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": k["achieved_tflops"] / tc_peak,
+                "traffic": traffic, "traffic_source": note,
+                "peak_source": f"{peak_src} bf16_tflops (fp16 MMA runs at the same rate)",
+                "hbm_achieved_gbs": k["achieved_gbs"], "hbm_frac": k["achieved_gbs"] / hbm_peak,
+                "hbm_frac_of_nominal_8tbs": k["achieved_gbs"] / 8000.0}
+        if wl.prefill_start is not None:
+            roof["note"] = ("prefill: the selected rows are gathered from a cache that stays in L2, "
+                            "so the per-query bytes exceed what crosses HBM")
+        return roof
+    name = {"index_topk": "csa2_index_topk", "reindex_topk": "csa2_index_topk (Reindex)",
+            "step_writes": "csa2_quantize_kv_batch"}[dom]
+    return {"kernel": name, "bound": "hbm", "achieved": k["achieved_gbs"], "peak": hbm_peak, "unit": "GB/s",
+            "frac": k["achieved_gbs"] / hbm_peak, "traffic": None, "traffic_source": "no capture",
+            "peak_source": f"{peak_src} hbm_gbs"}
+
+
+def measure_workload(torch, csa2, args, wl, world, rank, local, peaks, flush, detail=True):
+    """Time the workload's step (graph replays, L2 flushed before each) and, with detail, the
+    per-call breakdown, roofline, e2e and the oracle's CPU baseline."""
     import torch.distributed as dist
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
-    import compressed_sparse_attention_quantize_b200 as csa2
-    from compressed_sparse_attention_quantize_b200 import build as csa2_build, runtime, synth
-    if not os.path.exists(csa2.library_path()):
-        csa2_build.build()
-    if rank > 0:
-        wl.seed = wl.seed + 1000 * rank          # independent sequences per rank
-    hbm_peak, tc_peak, tc_sus, peak_src = _peaks()
+    from compressed_sparse_attention_quantize_b200 import runtime
     runner = runtime.GroupRunner(wl, out_dtype=csa2.DTYPE_BF16)
-    flush_buf = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device="cuda")
-
-    def flush():
-        flush_buf.fill_(1)
-
     # the timed step: the step's quantise-on-write (newest entry and indexer key per sequence,
-    # indexer queries, window entries of the step token), then the layer group; replayed as one
-    # CUDA graph (--eager: one call each per step).  If the writes fail on their first run (an
-    # argument the library rejects), the step falls back to the group alone and says so.
+    # indexer queries, window entries of the step token) in one launch, then the layer group;
+    # replayed as one CUDA graph (--eager: one call each per step).  If the writes fail on their
+    # first run (an argument the library rejects), the step falls back to the group alone and
+    # says so.
     writes = True
     writes_note = STEP_WRITES
     try:
@@ -567,69 +678,94 @@ def run_csa2(args, wl):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
         dist.barrier()
-    value = wl.B * wl.T * world * args.steps / (total_ms / 1e3)
-
-    if args.quick:
-        if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-                              "steps": args.steps, "warmup": args.warmup,
-                              "ms_per_step": total_ms / args.steps, "config": {"workload": wl.name},
-                              "gpu_launches": int(launches), "clocks": clocks, "quick": True}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
-        return
-
-    # per-call breakdown and roofline of the dominant kernel
+    rows = wl.B * wl.T
+    res = {"value": rows * world * args.steps / (total_ms / 1e3), "unit": UNIT,
+           "ms_per_step": total_ms / args.steps, "steps": args.steps, "warmup": args.warmup,
+           "gpu_launches": int(launches), "clocks": clocks,
+           "config": {"workload": wl.name, "batch_per_gpu": wl.B, "queries_per_sequence": wl.T,
+                      "ctx_tokens": wl.ctx_tokens[0] if len(set(wl.ctx_tokens)) == 1 else wl.ctx_tokens,
+                      "entries_per_seq": wl.n_entries[0] if len(set(wl.n_entries)) == 1 else wl.n_entries,
+                      "layers": ",".join(wl.modes), "heads": wl.H, "index_heads": wl.HI, "topk": wl.K,
+                      "pool": wl.P, "swa": 128, "out": "bf16", "step": "eager" if args.eager else "cuda graph",
+                      "step_writes": writes_note,
+                      "parallelism": f"replicas x{world} (independent sequences)",
+                      "l2": "flushed between steps (256 MB write, outside the events)"}}
+    if not detail:
+        del runner
+        return res
     bd = breakdown(torch, csa2, runner, max(3, min(args.steps, 10)), flush, writes)
-    ab, af = attn_work(wl, 2 if runner.out_dtype == csa2.DTYPE_BF16 else 4)
-    ib = index_work(wl)
-    kernels = {}
-    if "sparse_attn" in bd:
-        t_ms = statistics.mean(bd["sparse_attn"])
-        kernels["sparse_attn"] = {"launches_per_step": len(runner.modes), "avg_ms": t_ms,
-                                  "share": None, "algorithmic_bytes": ab, "algorithmic_flops": af,
-                                  "achieved_gbs": ab / (t_ms * 1e-3) / 1e9,
-                                  "achieved_tflops": af / (t_ms * 1e-3) / 1e12}
-    if "step_writes" in bd:
-        t_ms = statistics.mean(bd["step_writes"])
-        wb = write_work(runner)
-        kernels["step_writes"] = {"launches_per_step": 1, "calls": write_calls(runner), "avg_ms": t_ms,
-                                  "algorithmic_bytes": wb, "achieved_gbs": wb / (t_ms * 1e-3) / 1e9}
-    if "index_topk" in bd:
-        t_ms = statistics.mean(bd["index_topk"])
-        kernels["index_topk"] = {"launches_per_step": 1, "avg_ms": t_ms, "algorithmic_bytes": ib,
-                                 "achieved_gbs": ib / (t_ms * 1e-3) / 1e9}
-    for k in kernels.values():
-        k["hbm_frac"] = k["achieved_gbs"] / hbm_peak
-        k["hbm_frac_of_nominal_8tbs"] = k["achieved_gbs"] / 8000.0
-    tot = sum(k["avg_ms"] * k["launches_per_step"] for k in kernels.values())
-    for k in kernels.values():
-        k["share"] = k["avg_ms"] * k["launches_per_step"] / tot if tot else None
-    dom = max(kernels, key=lambda k: kernels[k]["share"] or 0) if kernels else None
-    roof = None
-    if dom == "sparse_attn":
-        k = kernels[dom]
-        roof = {"kernel": "csa2_sparse_attn", "bound": "tensor", "achieved": k["achieved_tflops"],
-                "peak": tc_peak, "unit": "TFLOP/s", "frac": k["achieved_tflops"] / tc_peak,
-                "traffic": ATTN_TRAFFIC_BYTES, "traffic_source": ATTN_TRAFFIC_SOURCE, "peak_source": f"{peak_src} bf16_tflops (fp16 MMA runs at the same rate)",
-                "hbm_achieved_gbs": k["achieved_gbs"], "hbm_frac": k["achieved_gbs"] / hbm_peak,
-                "hbm_frac_of_nominal_8tbs": k["achieved_gbs"] / 8000.0}
-    elif dom == "index_topk":
-        k = kernels[dom]
-        roof = {"kernel": "csa2_index_topk", "bound": "hbm", "achieved": k["achieved_gbs"],
-                "peak": hbm_peak, "unit": "GB/s", "frac": k["achieved_gbs"] / hbm_peak,
-                "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
-
+    kernels = kernel_table(wl, runner, bd, peaks, 2)
+    res["kernels"] = kernels
+    res["roofline"] = roofline(wl, kernels, peaks)
     e2e = e2e_measure(torch, csa2, runner, max(3, min(args.steps, 10)), 2, flush, writes)
     if world > 1:
         t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["value"] = wl.B * wl.T * world / (float(t.item()) / 1e3)
+        e2e["value"] = rows * world / (float(t.item()) / 1e3)
         e2e["ms_per_step"] = float(t.item())
-
-    cpu = None
+    res["e2e"] = e2e
+    softmax_scale = runner.softmax_scale
+    del runner
+    torch.cuda.empty_cache()
+    res["cpu_baseline"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, runner.softmax_scale)
+        res["cpu_baseline"] = cpu_baseline(wl, softmax_scale, budget_s=15.0 if args.config == wl.seed else 4.0)
+    return res
+
+
+def run_csa2(args, wl):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    import compressed_sparse_attention_quantize_b200 as csa2
+    from compressed_sparse_attention_quantize_b200 import build as csa2_build, synth
+    if not os.path.exists(csa2.library_path()):
+        csa2_build.build()
+
+    def replica(w):
+        if rank > 0:
+            w.seed = w.seed + 1000 * rank          # independent sequences per rank
+        return w
+
+    peaks = _peaks()
+    flush_buf = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1)
+
+    head = measure_workload(torch, csa2, args, replica(wl), world, rank, local, peaks, flush,
+                            detail=not args.quick)
+    if args.quick:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                              "config": {"workload": wl.name}, "gpu_launches": head["gpu_launches"],
+                              "clocks": head["clocks"], "quick": True}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    # the other timed workloads (decode at 1M context first: the metric's second context)
+    workloads = {}
+    if not args.no_workloads and not args.entries:
+        for c in (3, 2, 4):
+            if c == args.config:
+                continue
+            w = replica(synth.workload(c))
+            try:
+                r = measure_workload(torch, csa2, args, w, world, rank, local, peaks, flush)
+            except Exception as exc:              # one workload never costs the headline line
+                torch.cuda.synchronize()
+                r = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            r.pop("steps", None)
+            r.pop("warmup", None)
+            workloads[w.name] = r
 
     try:
         side = topk_side_reference(torch, csa2, wl, flush)
@@ -637,21 +773,15 @@ def run_csa2(args, wl):
         side = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f16 MMA (attention), fp4 MMA (indexer), f32 accumulate",
+        line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None,
+                "dtype": "f16 MMA (attention), fp4 MMA (indexer), f32 accumulate",
                 "data": "synthetic (seeded; shapes and distributions of the workload)",
-                "config": {"workload": wl.name, "batch_per_gpu": wl.B, "ctx_tokens": wl.ctx_tokens[0],
-                           "entries_per_seq": wl.n_entries[0], "layers": ",".join(wl.modes),
-                           "heads": wl.H, "index_heads": wl.HI, "topk": wl.K, "pool": wl.P,
-                           "swa": 128, "out": "bf16", "step": "eager" if args.eager else "cuda graph",
-                           "step_writes": writes_note,
-                           "parallelism": f"replicas x{world} (independent sequences)",
-                           "l2": "flushed between steps (256 MB write, outside the events)"},
-                "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": int(launches), "clocks": clocks, "topk_side_reference": side}
+                "config": head["config"], "roofline": head["roofline"], "kernels": head["kernels"],
+                "cpu_baseline": head["cpu_baseline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+                "clocks": head["clocks"], "workloads": workloads, "topk_side_reference": side}
         print(json.dumps(line), flush=True)
-    del runner
     if world > 1:
         dist.destroy_process_group()
 
@@ -664,6 +794,8 @@ def main():
     ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time the --config workload only (no 'workloads' object)")
     ap.add_argument("--eager", action="store_true", help="time one csa2_layer_group call per step "
                     "instead of replaying it as a CUDA graph")
     ap.add_argument("--quick", action="store_true",

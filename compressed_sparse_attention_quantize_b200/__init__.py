@@ -16,15 +16,20 @@ from typing import Optional, Sequence
 
 __all__ = [
     "CSA2Error", "lib", "library_path",
-    "csa2_quantize_kv", "csa2_compress_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
+    "csa2_quantize_kv", "csa2_quantize_kv_batch", "quant_job", "QuantJob", "csa2_compress_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
     "csa2_index_topk_scored", "csa2_topk_merge_shards", "csa2_topk_merge_shards_workspace_size",
     "csa2_attn_merge_shards", "csa2_sparse_attn_shard",
     "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_plan", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error", "csa2_selftest_bounded_wait",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
     "FMT_FP4", "FMT_FP8_TOKEN", "DTYPE_F32", "DTYPE_BF16", "MODE_FULL", "MODE_REINDEX",
-    "MODE_REUSE",
+    "MODE_REUSE", "CSA2_OK", "CSA2_ERR_INVALID_ARG", "CSA2_ERR_SHAPE", "CSA2_ERR_TIMEOUT",
 ]
+
+CSA2_OK = 0
+CSA2_ERR_INVALID_ARG = 1
+CSA2_ERR_SHAPE = 2
+CSA2_ERR_TIMEOUT = 6
 
 FMT_FP4 = 0
 FMT_FP8_TOKEN = 1
@@ -47,6 +52,14 @@ _sz = ctypes.c_size_t
 
 class CSA2Error(RuntimeError):
     pass
+
+
+class QuantJob(ctypes.Structure):
+    """Mirror of ``csa2_quant_job``."""
+    _fields_ = [
+        ("fmt", _i32), ("x_dtype", _i32), ("x", _vp), ("rows", _i64), ("dim", _i32), ("x_stride", _i64),
+        ("codes", _vp), ("code_stride", _i64), ("scales", _vp), ("scale_stride", _i64), ("dst_rows", _vp),
+    ]
 
 
 class GroupDesc(ctypes.Structure):
@@ -91,6 +104,8 @@ def lib():
     L.csa2_version.argtypes = []
     L.csa2_quantize_kv.restype = _i32
     L.csa2_quantize_kv.argtypes = [_i32, _vp, _i32, _i64, _i32, _i64, _vp, _i64, _vp, _i64, _vp, _vp]
+    L.csa2_quantize_kv_batch.restype = _i32
+    L.csa2_quantize_kv_batch.argtypes = [ctypes.POINTER(QuantJob), _i32, _vp]
     L.csa2_compress_quantize_kv.restype = _i32
     L.csa2_compress_quantize_kv.argtypes = [_vp, _i32, _i64, _i32, _i32, _i64, _vp, _i64, _vp, _i64,
                                             _vp, _i64, _vp, _vp]
@@ -118,10 +133,10 @@ def lib():
     L.csa2_sparse_attn_workspace_size.restype = _i32
     L.csa2_sparse_attn_workspace_size.argtypes = [_i32, _i32, _i32, ctypes.POINTER(_sz)]
     L.csa2_sparse_attn.restype = _i32
-    L.csa2_sparse_attn.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _i32,
+    L.csa2_sparse_attn.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _i32,
                                    _vp, _vp, _i32, _vp, _vp, _f32, _vp, _i32, _vp, _vp, _sz, _vp]
     L.csa2_sparse_attn_noalloc.restype = _i32
-    L.csa2_sparse_attn_noalloc.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _i32,
+    L.csa2_sparse_attn_noalloc.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _i32,
                                            _vp, _vp, _i32, _vp, _vp, _f32, _vp, _i32, _vp, _vp]
     L.csa2_layer_group_workspace_size.restype = _i32
     L.csa2_layer_group_workspace_size.argtypes = [ctypes.POINTER(GroupDesc), ctypes.POINTER(LayerDesc),
@@ -183,6 +198,21 @@ def csa2_quantize_kv(fmt, x, x_dtype, rows, dim, x_stride, codes, code_stride, s
                      dst_rows=None, stream=None) -> None:
     _check(lib().csa2_quantize_kv(fmt, _ptr(x), x_dtype, rows, dim, x_stride, _ptr(codes), code_stride,
                                   _ptr(scales), scale_stride, _ptr(dst_rows), _stream(stream)))
+
+
+def quant_job(fmt, x, x_dtype, rows, dim, x_stride, codes, code_stride, scales, scale_stride,
+              dst_rows=None) -> QuantJob:
+    """One job of csa2_quantize_kv_batch (the arguments of csa2_quantize_kv)."""
+    j = QuantJob()
+    j.fmt, j.x_dtype, j.x, j.rows, j.dim, j.x_stride = fmt, x_dtype, _ptr(x), rows, dim, x_stride
+    j.codes, j.code_stride, j.scales, j.scale_stride = _ptr(codes), code_stride, _ptr(scales), scale_stride
+    j.dst_rows = _ptr(dst_rows)
+    return j
+
+
+def csa2_quantize_kv_batch(jobs: Sequence[QuantJob], stream=None) -> None:
+    arr = (QuantJob * max(len(jobs), 1))(*jobs)
+    _check(lib().csa2_quantize_kv_batch(arr, len(jobs), _stream(stream)))
 
 
 def csa2_compress_quantize_kv(x, x_dtype, entries, ratio, dim, x_stride, w, w_stride, codes,
@@ -260,22 +290,22 @@ def csa2_sparse_attn_workspace_size(rows, H, K) -> int:
     return out.value
 
 
-def csa2_sparse_attn(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, cnt, K, swa_codes, swa_scale,
-                     swa_cap, swa_start, swa_len, softmax_scale, out, out_dtype, lse, workspace,
+def csa2_sparse_attn(q, B, T, H, D, kv, kv_row_stride, seq_start, n_entries, idx, cnt, K, swa_codes,
+                     swa_scale, swa_cap, swa_start, swa_len, softmax_scale, out, out_dtype, lse, workspace,
                      ws_bytes, stream=None) -> None:
     _check(lib().csa2_sparse_attn(_ptr(q), B, T, H, D, _ptr(kv), kv_row_stride, _ptr(seq_start),
-                                  _ptr(idx), _ptr(cnt), K, _ptr(swa_codes), _ptr(swa_scale), swa_cap,
+                                  _ptr(n_entries), _ptr(idx), _ptr(cnt), K, _ptr(swa_codes), _ptr(swa_scale), swa_cap,
                                   _ptr(swa_start), _ptr(swa_len), float(softmax_scale), _ptr(out),
                                   out_dtype, _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
-def csa2_sparse_attn_noalloc(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, cnt, K, swa_codes,
-                             swa_scale, swa_cap, swa_start, swa_len, softmax_scale, out, out_dtype, lse,
-                             stream=None) -> None:
+def csa2_sparse_attn_noalloc(q, B, T, H, D, kv, kv_row_stride, seq_start, n_entries, idx, cnt, K,
+                             swa_codes, swa_scale, swa_cap, swa_start, swa_len, softmax_scale, out,
+                             out_dtype, lse, stream=None) -> None:
     """csa2_sparse_attn without a workspace argument, for callers that cannot allocate device
     memory: the scratch lives in a fixed array inside the library (see include/csa2.h)."""
     _check(lib().csa2_sparse_attn_noalloc(_ptr(q), B, T, H, D, _ptr(kv), kv_row_stride, _ptr(seq_start),
-                                          _ptr(idx), _ptr(cnt), K, _ptr(swa_codes), _ptr(swa_scale),
+                                          _ptr(n_entries), _ptr(idx), _ptr(cnt), K, _ptr(swa_codes), _ptr(swa_scale),
                                           swa_cap, _ptr(swa_start), _ptr(swa_len), float(softmax_scale),
                                           _ptr(out), out_dtype, _ptr(lse), _stream(stream)))
 

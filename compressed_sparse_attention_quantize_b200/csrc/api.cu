@@ -22,6 +22,7 @@ cudaError_t launch_quant_fp4(const void *, int, int64_t, int, int64_t, uint8_t *
                              uint8_t *, int64_t, const int64_t *, cudaStream_t);
 cudaError_t launch_quant_fp8_token(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
                                    uint8_t *, int64_t, const int64_t *, cudaStream_t);
+cudaError_t launch_quant_batch(const csa2_quant_job *, int, cudaStream_t);
 }  // namespace csa2
 
 #include "index_api.cuh"
@@ -133,16 +134,15 @@ const char *csa2_status_string(csa2_status s) {
     return "CSA2: unknown status";
 }
 
-int csa2_version(void) { return 2; }
+int csa2_version(void) { return 3; }
 
 const char *csa2_last_error_string(void) { return t_last_error; }
 
 uint64_t csa2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
-                             int64_t x_stride, uint8_t *codes, int64_t code_stride, void *scales,
-                             int64_t scale_stride, const int64_t *dst_rows, void *stream) {
-    const Range range("csa2_quantize_kv");
+static csa2_status check_quant_args(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
+                                    int64_t x_stride, const uint8_t *codes, int64_t code_stride,
+                                    const void *scales, int64_t scale_stride) {
     if (fmt != CSA2_FMT_FP4_E2M1_E4M3S16 && fmt != CSA2_FMT_FP8_E4M3_TOKEN) return CSA2_ERR_INVALID_ARG;
     if (x_dtype != CSA2_DTYPE_F32 && x_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_INVALID_ARG;
     if (rows == 0) return CSA2_OK;                               // no-op, whatever the strides
@@ -150,15 +150,41 @@ csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, 
     if (!x || !codes || !scales) return CSA2_ERR_INVALID_ARG;
     if (fmt == CSA2_FMT_FP4_E2M1_E4M3S16) {
         if (code_stride < dim / 2 || scale_stride < dim / 16) return CSA2_ERR_SHAPE;
-        return cuda_status(launch_quant_fp4(x, x_dtype, rows, dim, x_stride, codes, code_stride,
-                                            (uint8_t *)scales, scale_stride, dst_rows,
-                                            as_stream(stream)));
+        return CSA2_OK;
     }
     if (code_stride < dim || scale_stride < 4) return CSA2_ERR_SHAPE;
     if ((((uintptr_t)scales) & 3u) || (scale_stride & 3)) return CSA2_ERR_ALIGN;
+    return CSA2_OK;
+}
+
+csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64_t rows, int dim,
+                             int64_t x_stride, uint8_t *codes, int64_t code_stride, void *scales,
+                             int64_t scale_stride, const int64_t *dst_rows, void *stream) {
+    const Range range("csa2_quantize_kv");
+    const csa2_status s = check_quant_args(fmt, x, x_dtype, rows, dim, x_stride, codes, code_stride, scales,
+                                           scale_stride);
+    if (s != CSA2_OK || rows == 0) return s;
+    if (fmt == CSA2_FMT_FP4_E2M1_E4M3S16)
+        return cuda_status(launch_quant_fp4(x, x_dtype, rows, dim, x_stride, codes, code_stride,
+                                            (uint8_t *)scales, scale_stride, dst_rows,
+                                            as_stream(stream)));
     return cuda_status(launch_quant_fp8_token(x, x_dtype, rows, dim, x_stride, codes, code_stride,
                                               (uint8_t *)scales, scale_stride, dst_rows,
                                               as_stream(stream)));
+}
+
+csa2_status csa2_quantize_kv_batch(const csa2_quant_job *jobs, int n_jobs, void *stream) {
+    const Range range("csa2_quantize_kv_batch");
+    if (n_jobs < 0 || n_jobs > CSA2_MAX_QUANT_JOBS) return CSA2_ERR_SHAPE;
+    if (n_jobs == 0) return CSA2_OK;
+    if (!jobs) return CSA2_ERR_INVALID_ARG;
+    for (int i = 0; i < n_jobs; ++i) {
+        const csa2_quant_job &j = jobs[i];
+        const csa2_status s = check_quant_args(j.fmt, j.x, j.x_dtype, j.rows, j.dim, j.x_stride, j.codes,
+                                               j.code_stride, j.scales, j.scale_stride);
+        if (s != CSA2_OK) return s;
+    }
+    return cuda_status(launch_quant_batch(jobs, n_jobs, as_stream(stream)));
 }
 
 csa2_status csa2_compress_quantize_kv(const void *x, int x_dtype, int64_t entries, int ratio, int dim,
@@ -287,7 +313,8 @@ csa2_status csa2_sparse_attn_workspace_size(int rows, int H, int K, size_t *byte
 }
 
 csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D, const uint8_t *kv,
-                             int64_t kv_row_stride, const int64_t *seq_start, const int32_t *idx,
+                             int64_t kv_row_stride, const int64_t *seq_start,
+                             const int32_t *n_entries, const int32_t *idx,
                              const int32_t *cnt, int K, const uint8_t *swa_codes,
                              const float *swa_scale, int swa_cap, const int32_t *swa_start,
                              const int32_t *swa_len, float softmax_scale, void *out,
@@ -301,7 +328,7 @@ csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D, cons
     if (!workspace || ws_bytes < attn_ws(rows, H, K)) return CSA2_ERR_WORKSPACE;
     AttnArgs a;
     a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
-    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start;
+    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start; a.n_entries = n_entries;
     a.shard_lo = nullptr; a.shard_n = nullptr;
     a.idx = idx; a.cnt = cnt;
     a.swa_codes = swa_codes; a.swa_scale = swa_scale; a.swa_cap = swa_cap;
@@ -327,7 +354,7 @@ csa2_status csa2_sparse_attn_shard(const uint16_t *q, int B, int T, int H, int D
     if (!workspace || ws_bytes < attn_ws(rows, H, K)) return CSA2_ERR_WORKSPACE;
     AttnArgs a;
     a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
-    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start;
+    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start; a.n_entries = nullptr;
     a.shard_lo = shard_lo; a.shard_n = shard_n;
     a.idx = idx; a.cnt = cnt;
     a.swa_codes = swa_codes; a.swa_scale = swa_scale; a.swa_cap = swa_cap;
@@ -488,6 +515,7 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
         AttnArgs a;
         a.q = L.q; a.rows = rows; a.T = g->T; a.H = g->H; a.K = g->K;
         a.kv = g->kv; a.kv_row_stride = g->kv_row_stride; a.seq_start = g->seq_start;
+        a.n_entries = g->n_entries;
         a.shard_lo = nullptr; a.shard_n = nullptr;
         a.idx = idx; a.cnt = cnt;
         a.swa_codes = L.swa_codes; a.swa_scale = L.swa_scale; a.swa_cap = g->swa_cap;
@@ -496,7 +524,7 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
         a.partials = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(aws) + slot * aws_one);
         a.splits = 1;
         bool merged = false;
-        cudaError_t e = launch_attn_tc_side_merge(a, st, aux->side, aux->attn_done, &merged);
+        cudaError_t e = launch_attn_side_merge(a, st, aux->side, aux->attn_done, &merged);
         if (e != cudaSuccess) return cuda_status(e);
         if (merged) {
             e = cudaEventRecord(aux->merge_done[slot], aux->side);

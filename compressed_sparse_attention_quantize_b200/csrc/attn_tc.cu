@@ -91,21 +91,32 @@ struct KeySrc {
     float scale;             // window token scale (1 for main entries, 0 if invalid)
 };
 
-CSA2_D KeySrc source_of(const AttnArgs &a, int r, int b, int64_t seq_start, int32_t e) {
+// An id at or above its sequence's entry count (n_lim) or a window slot outside the window buffer
+// breaks the caller contract: the key is skipped and the device error word records
+// CSA2_ERR_INVALID_ARG, so nothing is read outside the caller's buffers.
+CSA2_D KeySrc source_of(const AttnArgs &a, int r, int b, int64_t seq_start, int64_t n_lim, int32_t e) {
     KeySrc k{false, false, nullptr, 0.0f};
     if (e == kNoKey) return k;
     if (e >= 0 && a.shard_lo) {                   // context shard: global entry -> this shard's row
         const int64_t le = (int64_t)e - a.shard_lo[b];
         if (le < 0 || le >= a.shard_n[b]) return k;
         e = (int32_t)le;
+    } else if (e >= n_lim) {
+        raise_device_error(CSA2_ERR_INVALID_ARG);
+        return k;
     }
-    k.valid = true;
     if (e >= 0) {
+        k.valid = true;
         k.ptr = a.kv + (seq_start + e) * a.kv_row_stride;
         k.scale = 1.0f;
     } else {
         const int slot = (a.swa_start ? a.swa_start[r] : 0) + (-1 - e);
+        if (slot < 0 || slot >= a.swa_cap) {
+            raise_device_error(CSA2_ERR_INVALID_ARG);
+            return k;
+        }
         const int64_t srow = (int64_t)b * a.swa_cap + slot;
+        k.valid = true;
         k.swa = true;
         k.ptr = a.swa_codes + srow * kLatent;
         k.scale = a.swa_scale[srow];
@@ -311,8 +322,16 @@ attn_tc_kernel(AttnArgs a) {
     const int b = r / a.T;
     const int h0 = hg * kHeads;
 
-    const int n_sel = a.cnt ? a.cnt[r] : a.K;
-    const int total = n_sel + a.swa_len[r];
+    // counts outside [0, K] and window lengths outside [0, CSA2_SWA_WINDOW] break the caller
+    // contract: they are clamped and the device error word records CSA2_ERR_SHAPE
+    int n_sel = a.cnt ? a.cnt[r] : a.K;
+    int wlen = a.swa_len[r];
+    if (n_sel < 0 || n_sel > a.K || wlen < 0 || wlen > CSA2_SWA_WINDOW) {
+        if (threadIdx.x == 0) raise_device_error(CSA2_ERR_SHAPE);
+        n_sel = min(max(n_sel, 0), a.K);
+        wlen = min(max(wlen, 0), CSA2_SWA_WINDOW);
+    }
+    const int total = n_sel + wlen;
     const int x_begin = split * a.keys_per_split;
     const int x_end = min(total, x_begin + a.keys_per_split);
     const int ntiles = x_end > x_begin ? (x_end - x_begin + kTile - 1) / kTile : 0;
@@ -323,11 +342,12 @@ attn_tc_kernel(AttnArgs a) {
     const int hsel = (warp - 1) >> 2;
     const int t = sub * 32 + lane;
     const int64_t seq_start = a.seq_start[b];
+    const int64_t n_lim = a.n_entries ? (int64_t)a.n_entries[b] : INT64_MAX;
     // the first tile's rows are requested before anything else
     KeySrc src{false, false, nullptr, 0.0f};
     RowPart rp;
     if (warp > 0) {
-        src = source_of(a, r, b, seq_start, entry_of(a, r, x_begin + t, x_end, n_sel));
+        src = source_of(a, r, b, seq_start, n_lim, entry_of(a, r, x_begin + t, x_end, n_sel));
         prefetch_part(src, hsel, rp);
     }
 
@@ -451,7 +471,7 @@ attn_tc_kernel(AttnArgs a) {
             // ---- the next tile's rows are requested now, while the tensor core is idle until P
             //      is ready (issued during P.V they slowed its operand reads); the softmax below
             //      works on 16 heads at a time so these registers stay live without spilling
-            src = source_of(a, r, b, seq_start, e_next);
+            src = source_of(a, r, b, seq_start, n_lim, e_next);
             prefetch_part(src, hsel, rp);
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             if (!ptx::mbar_wait(&S.s_full, ph, abort_flag)) bad = true;
@@ -727,36 +747,31 @@ __global__ void __launch_bounds__(128) attn_tc_merge_kernel(AttnArgs a) {
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
-static int g_num_sms = 0;
+static SmemLimit g_attn_smem;
 
-static int num_sms() {
-    if (g_num_sms == 0) {
-        int dev = 0, n = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-            g_num_sms = n;
-        else
-            g_num_sms = 148;
-    }
-    return g_num_sms;
+size_t attn_plan_workspace(int rows, int hgroups, int splits) {
+    if (splits <= 1) return 256;
+    return (size_t)rows * hgroups * splits * kPartialFloats * sizeof(float) + 256;
 }
 
 // Split plan (one CTA per SM).  Each CTA costs a fixed part (Q staging, first loads, epilogue:
 // about 1.8 tile times, measured) plus its tiles; splits add merge work (about 0.009 tile times
 // per row and split, plus the merge launch).  The remainder split is the slowest-varying grid
 // index, so its short CTAs are the ones that wait for an SM when the grid exceeds the SMs.
-// Pick the tiles per split with the smallest estimated finish time.
-void tc_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_split) {
+// Pick the tiles per split with the smallest estimated finish time among the plans whose
+// partials fit in max_ws bytes.
+void attn_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_split, size_t max_ws) {
     hgroups = (H + tc::kHeads - 1) / tc::kHeads;
     const int max_keys = K + CSA2_SWA_WINDOW;
     const int tiles = (max_keys + tc::kTile - 1) / tc::kTile;
     const int per_split = rows * hgroups;                     // CTAs of one split index
-    const int nsm = num_sms();
+    const int nsm = device_sm_count();
     const double fixed = 1.8, merge_per = 0.009, merge_launch = 0.3;
     double best = 1e30;
     int best_tp = tiles;
     for (int tp = 1; tp <= tiles; ++tp) {
         const int sp = (tiles + tp - 1) / tp;
+        if (attn_plan_workspace(rows, hgroups, sp) > max_ws) continue;
         const int last = tiles - (sp - 1) * tp;
         const long long ctas = (long long)per_split * sp;
         double t;
@@ -776,60 +791,53 @@ void tc_plan(int rows, int H, int K, int &hgroups, int &splits, int &keys_per_sp
     keys_per_split = best_tp * tc::kTile;
 }
 
-size_t tc_workspace_bytes(int rows, int H, int K) {
+size_t attn_workspace_bytes(int rows, int H, int K) {
     int hg, sp, kps;
-    tc_plan(rows, H, K, hg, sp, kps);
-    if (sp == 1) return 256;
-    return (size_t)rows * hg * sp * kPartialFloats * sizeof(float) + 256;
+    attn_plan(rows, H, K, hg, sp, kps);
+    return attn_plan_workspace(rows, hg, sp);
 }
 
-// As launch_attn_tc, but the split merge runs on `side` once the attention kernel has finished
-// (`attn_done` is recorded on `st` and waited on `side`); returns in *merged whether a merge was
-// queued on `side`.
-cudaError_t launch_attn_tc_side_merge(AttnArgs a, cudaStream_t st, cudaStream_t side, cudaEvent_t attn_done,
-                                      bool *merged) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             tc::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    tc_plan(a.rows, a.H, a.K, a.hgroups, a.splits, a.keys_per_split);
-    dim3 grid(a.rows, a.hgroups, a.splits);
-    tc::attn_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a);
-    int n = 1;
+// The attention kernel with the plan in `a`; the split merge (splits > 1) goes to `side` after
+// `attn_done` when a side stream is given, else it follows on `st`.
+static cudaError_t launch_with_plan(const AttnArgs &a, cudaStream_t st, cudaStream_t side, cudaEvent_t attn_done,
+                                   bool *merged) {
     *merged = false;
+    cudaError_t e = ensure_smem_limit(g_attn_smem, tc::attn_tc_kernel, tc::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.rows, a.hgroups, a.splits);
+    tc::attn_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a);
+    int n = 1;
     if (a.splits > 1) {
-        cudaError_t e = cudaEventRecord(attn_done, st);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, attn_done, 0);
-        if (e != cudaSuccess) return e;
-        tc::attn_tc_merge_kernel<<<dim3(a.rows, a.H), 128, 0, side>>>(a);
+        cudaStream_t ms = st;
+        if (side) {
+            e = cudaEventRecord(attn_done, st);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(side, attn_done, 0);
+            if (e != cudaSuccess) return e;
+            ms = side;
+            *merged = true;
+        }
+        tc::attn_tc_merge_kernel<<<dim3(a.rows, a.H), 128, 0, ms>>>(a);
         ++n;
-        *merged = true;
     }
     note_launches(n);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attn_tc(AttnArgs a, cudaStream_t st) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             tc::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    tc_plan(a.rows, a.H, a.K, a.hgroups, a.splits, a.keys_per_split);
-    dim3 grid(a.rows, a.hgroups, a.splits);
-    tc::attn_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, st>>>(a);
-    int n = 1;
-    if (a.splits > 1) {
-        tc::attn_tc_merge_kernel<<<dim3(a.rows, a.H), 128, 0, st>>>(a);
-        ++n;
-    }
-    note_launches(n);
-    return cudaGetLastError();
+cudaError_t launch_attn_planned(const AttnArgs &a, cudaStream_t st) {
+    bool merged;
+    return launch_with_plan(a, st, nullptr, nullptr, &merged);
+}
+
+cudaError_t launch_attn(AttnArgs a, cudaStream_t st) {
+    attn_plan(a.rows, a.H, a.K, a.hgroups, a.splits, a.keys_per_split);
+    bool merged;
+    return launch_with_plan(a, st, nullptr, nullptr, &merged);
+}
+
+cudaError_t launch_attn_side_merge(AttnArgs a, cudaStream_t st, cudaStream_t side, cudaEvent_t attn_done,
+                                   bool *merged) {
+    attn_plan(a.rows, a.H, a.K, a.hgroups, a.splits, a.keys_per_split);
+    return launch_with_plan(a, st, side, attn_done, merged);
 }
 
 }  // namespace csa2

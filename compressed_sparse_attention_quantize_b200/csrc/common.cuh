@@ -10,6 +10,9 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/csa2.h"
 
 #define CSA2_HD __host__ __device__ __forceinline__
@@ -93,8 +96,65 @@ CSA2_HD uint32_t float_key(float f) {
 
 CSA2_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Device-side error word: a bounded wait that expires stores a csa2_status here.
+// Device-side error word: a bounded wait that expires, or a kernel that meets an argument
+// outside the caller contract, stores a csa2_status here (the first one sticks).
 __device__ int g_device_error = 0;
+
+CSA2_D void raise_device_error(int status) { atomicCAS(&g_device_error, 0, status); }
+
+// ---------------------------------------------------------------------------------------
+// Per-device launch settings
+// ---------------------------------------------------------------------------------------
+// A kernel's dynamic shared-memory limit is a per-device setting (cudaFuncSetAttribute acts on
+// the current device) and launch plans depend on the device's SM count.  Launchers keep such
+// settings in tables indexed by device; a table entry is filled once per device under one
+// mutex, so first calls may come from several host threads and several devices at once.
+constexpr int kMaxDevices = 64;
+
+inline std::mutex &settings_mutex() {
+    static std::mutex m;
+    return m;
+}
+
+// The calling thread's current device, or -1 when there is none (or its number is too large).
+inline int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
+}
+
+// SM count of the current device; 148 (a B200) when no device can be queried, so that plans
+// can still be inspected on a host without a GPU.
+inline int device_sm_count() {
+    static std::atomic<int> cache[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return 148;
+    int n = cache[dev].load(std::memory_order_acquire);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_release);
+    return n;
+}
+
+// Dynamic shared-memory limit of one kernel on every device it has been raised on.
+struct SmemLimit {
+    std::atomic<int> bytes[kMaxDevices];
+};
+
+// Raises `kernel`'s dynamic shared-memory limit on the current device to at least `bytes`
+// (the limit only grows; a launch asks for its own size).
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(SmemLimit &lim, Kernel kernel, int bytes) {
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (lim.bytes[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(settings_mutex());
+    if (lim.bytes[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    lim.bytes[dev].store(bytes, std::memory_order_release);
+    return cudaSuccess;
+}
 
 // Host-side count of kernel launches (csa2_launch_count); every launcher adds its launches.
 void note_launches(int n);

@@ -111,6 +111,9 @@ size_t topk_merge_workspace_bytes(int G, int rows, int K_in) {
 cudaError_t launch_topk_merge_shards(const float *scores, const int32_t *ids, const int64_t *id_offset,
                                      const int32_t *cnt, int G, int rows, int K_in, int K, int32_t *out_idx,
                                      int32_t *out_cnt, void *workspace, cudaStream_t st) {
+    if (G == 1 && id_offset == nullptr)         // one list already in place: select from it directly
+        return launch_topk_cluster(scores, K_in, ids, K_in, nullptr, nullptr, cnt, 1, 0, rows, K, out_idx, out_cnt, 0,
+                                   nullptr, nullptr, K_in, st);
     const int64_t stride = (int64_t)G * K_in;
     float *c_scores = reinterpret_cast<float *>(workspace);
     int32_t *c_ids = reinterpret_cast<int32_t *>(c_scores + (size_t)rows * stride);

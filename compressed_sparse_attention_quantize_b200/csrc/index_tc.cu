@@ -315,6 +315,41 @@ index_score_tc_kernel(Args a) {
 
 }  // namespace itc
 
+static SmemLimit g_index_smem;
+
+// Resident CTAs of the score kernel on the current device for a dynamic shared-memory size:
+// the minimum of the TMEM-column limit (per_sm), shared memory (1 KB reserved per CTA) and
+// registers (the occupancy query does not account for the TMEM limit).  Cached per device and
+// TMEM width (per_sm is 512 / columns: 1, 2, 4, 8 or 16).
+static int index_resident_ctas(int per_sm, int dyn) {
+    static std::atomic<int> cache[kMaxDevices][5];
+    const int dev = current_device();
+    int slot = 0;
+    while ((1 << slot) < per_sm && slot < 4) ++slot;
+    if (dev >= 0) {
+        const int v = cache[dev][slot].load(std::memory_order_acquire);
+        if (v > 0) return v;
+    }
+    int nsm = 148, smem_sm = 228 * 1024;
+    if (dev >= 0) {
+        nsm = device_sm_count();
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    }
+    cudaFuncAttributes fa;
+    int regs = 72;
+    size_t stat = sizeof(itc::Smem);
+    if (cudaFuncGetAttributes(&fa, itc::index_score_tc_kernel) == cudaSuccess) {
+        regs = fa.numRegs > 0 ? fa.numRegs : regs;
+        stat = fa.sharedSizeBytes;
+    }
+    int blocks = per_sm;
+    blocks = min(blocks, smem_sm / (int)(stat + (size_t)dyn + 1024));
+    blocks = min(blocks, 65536 / (regs * itc::kThreads));
+    const int resident = max(blocks, 1) * nsm;
+    if (dev >= 0) cache[dev][slot].store(resident, std::memory_order_release);
+    return resident;
+}
+
 cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, float *scores,
                                   int64_t score_stride, cudaStream_t st) {
     itc::Args a;
@@ -340,32 +375,9 @@ cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, flo
     const int per_sm = 512 / (int)cols;
     const int smem_total = (227 * 1024) / per_sm - 1024;
     const int dyn = max(smem_total - (int)sizeof(itc::Smem), itc::kRingBytes);
-    static int attr_dyn = -1;
-    static int resident = 0;
-    if (attr_dyn != dyn) {
-        cudaError_t e = cudaFuncSetAttribute(itc::index_score_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-        if (e != cudaSuccess) return e;
-        attr_dyn = dyn;
-        // resident CTAs per SM, from TMEM columns, shared memory (1 KB reserved per CTA) and
-        // registers (the occupancy query does not account for this kernel's limits)
-        int dev = 0, nsm = 148, smem_sm = 228 * 1024;
-        if (cudaGetDevice(&dev) == cudaSuccess) {
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-            cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-        }
-        cudaFuncAttributes fa;
-        int regs = 72;
-        size_t stat = sizeof(itc::Smem);
-        if (cudaFuncGetAttributes(&fa, itc::index_score_tc_kernel) == cudaSuccess) {
-            regs = fa.numRegs > 0 ? fa.numRegs : regs;
-            stat = fa.sharedSizeBytes;
-        }
-        int blocks = per_sm;
-        blocks = min(blocks, smem_sm / (int)(stat + (size_t)dyn + 1024));
-        blocks = min(blocks, 65536 / (regs * itc::kThreads));
-        resident = max(blocks, 1) * nsm;
-    }
+    cudaError_t e = ensure_smem_limit(g_index_smem, itc::index_score_tc_kernel, dyn);
+    if (e != cudaSuccess) return e;
+    const int resident = index_resident_ctas(per_sm, dyn);
     // tiles per CTA: the fewest that fit every row's tiles into one wave of resident CTAs (a
     // partial second wave would cost a whole CTA time); with more rows than resident CTAs, 8
     const int64_t tiles_row = ceil_div(score_stride, (int64_t)itc::kTile);

@@ -10,8 +10,10 @@
 // The scratch is a file-scope __device__ array (kNoAllocScratchBytes); every device that loads
 // the library holds it until the process exits.  On first use on a device the call looks up
 // the array's device address with cudaGetSymbolAddress while that device is current and keeps
-// it; that first call should therefore happen before any stream capture.  All calls share the
-// one array and each call overwrites it completely before reading it (every split writes its
+// it; that first call should therefore happen before any stream capture.  The split plan is
+// the best one whose partials fit in the array (csa2_sparse_attn may pick more splits when its
+// workspace allows); one split per row needs no partials, so a fitting plan always exists.
+// All calls share the one array and each call overwrites what it reads (every split writes its
 // full partial before the merge reads it), so nothing needs clearing; calls whose kernels
 // overlap on the GPU (two streams, or two host threads) race on it.
 #include <mutex>
@@ -23,7 +25,6 @@ constexpr size_t kNoAllocScratchBytes = (size_t)20 << 20;    // 20 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kMaxDevices] = {nullptr};
 
@@ -49,31 +50,32 @@ csa2_status noalloc_scratch(void **out) {
 
 extern "C" csa2_status csa2_sparse_attn_noalloc(const uint16_t *q, int B, int T, int H, int D,
                                                 const uint8_t *kv, int64_t kv_row_stride,
-                                                const int64_t *seq_start, const int32_t *idx,
-                                                const int32_t *cnt, int K, const uint8_t *swa_codes,
-                                                const float *swa_scale, int swa_cap,
-                                                const int32_t *swa_start, const int32_t *swa_len,
-                                                float softmax_scale, void *out, int out_dtype,
-                                                float *lse, void *stream) {
+                                                const int64_t *seq_start, const int32_t *n_entries,
+                                                const int32_t *idx, const int32_t *cnt, int K,
+                                                const uint8_t *swa_codes, const float *swa_scale,
+                                                int swa_cap, const int32_t *swa_start,
+                                                const int32_t *swa_len, float softmax_scale, void *out,
+                                                int out_dtype, float *lse, void *stream) {
     using namespace csa2;
+    const Range range("csa2_sparse_attn_noalloc");
     csa2_status s = check_attn_args(q, B, T, H, D, kv, kv_row_stride, seq_start, idx, K, swa_codes,
                                     swa_scale, swa_cap, swa_len, out, out_dtype);
     if (s != CSA2_OK) return s;
-    const int rows = B * T;
-    if (tc_workspace_bytes(rows, H, K) > kNoAllocScratchBytes) return CSA2_ERR_WORKSPACE;
+    AttnArgs a;
+    a.rows = B * T;
+    attn_plan(a.rows, H, K, a.hgroups, a.splits, a.keys_per_split, kNoAllocScratchBytes);
+    if (attn_plan_workspace(a.rows, a.hgroups, a.splits) > kNoAllocScratchBytes) return CSA2_ERR_WORKSPACE;
     void *scratch = nullptr;
     s = noalloc_scratch(&scratch);
     if (s != CSA2_OK) return s;
-    AttnArgs a;
-    a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
-    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start;
+    a.q = q; a.T = T; a.H = H; a.K = K;
+    a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start; a.n_entries = n_entries;
     a.idx = idx; a.cnt = cnt;
     a.swa_codes = swa_codes; a.swa_scale = swa_scale; a.swa_cap = swa_cap;
     a.swa_start = swa_start; a.swa_len = swa_len;
     a.softmax_scale = softmax_scale; a.out = out; a.out_dtype = out_dtype; a.lse = lse;
     a.partials = reinterpret_cast<float *>(scratch);
-    a.splits = 1;
     a.shard_lo = nullptr;
     a.shard_n = nullptr;
-    return cuda_status(launch_attn_tc(a, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_attn_planned(a, reinterpret_cast<cudaStream_t>(stream)));
 }

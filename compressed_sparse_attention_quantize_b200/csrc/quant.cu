@@ -148,6 +148,101 @@ __global__ void quant_fp8_token_kernel(const T *__restrict__ x, int64_t rows, in
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Several quantise-on-write jobs in one launch (a decode step writes a main-KV entry, its
+// indexer key, window tokens and indexer queries: one launch instead of one per buffer).
+// Block b belongs to the job whose block range holds it; FP4 jobs take one thread per
+// 16-channel block, FP8 jobs one warp per row, as the single-job kernels do.
+// ---------------------------------------------------------------------------------------
+struct QuantJob {
+    int fmt, x_dtype, dim;
+    const void *x;
+    int64_t rows, x_stride;
+    uint8_t *codes;
+    int64_t code_stride;
+    uint8_t *scales;
+    int64_t scale_stride;
+    const int64_t *dst_rows;
+};
+
+constexpr int kMaxQuantJobs = 16;
+static_assert(kMaxQuantJobs == CSA2_MAX_QUANT_JOBS, "one job table size");
+constexpr int kQuantThreads = 256;
+
+struct QuantJobs {
+    QuantJob job[kMaxQuantJobs];
+    int64_t block_start[kMaxQuantJobs + 1];
+    int n;
+};
+
+CSA2_D float load_elem(const void *x, int dtype, int64_t i) {
+    return dtype == CSA2_DTYPE_F32 ? __ldg(reinterpret_cast<const float *>(x) + i)
+                                   : bf16_bits_to_f32(__ldg(reinterpret_cast<const uint16_t *>(x) + i));
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quant_batch_kernel(const __grid_constant__ QuantJobs J) {
+    int j = 0;
+    while (j + 1 < J.n && (int64_t)blockIdx.x >= J.block_start[j + 1]) ++j;
+    const QuantJob &q = J.job[j];
+    const int64_t lb = (int64_t)blockIdx.x - J.block_start[j];
+    if (q.fmt == CSA2_FMT_FP4_E2M1_E4M3S16) {
+        const int nblk = q.dim >> 4;
+        const int64_t t = lb * kQuantThreads + threadIdx.x;
+        if (t >= q.rows * nblk) return;
+        const int64_t r = t / nblk;
+        const int b = (int)(t - r * nblk);
+        const int64_t base = r * q.x_stride + b * 16;
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = load_elem(q.x, q.x_dtype, base + i);
+        const int64_t d = q.dst_rows ? q.dst_rows[r] : r;
+        quantize_block16(v, q.codes + d * q.code_stride + b * 8, q.scales + d * q.scale_stride + b);
+    } else {
+        const int lane = threadIdx.x & 31;
+        const int64_t r = lb * (kQuantThreads / 32) + (threadIdx.x >> 5);
+        if (r >= q.rows) return;                                   // uniform per warp
+        const int64_t base = r * q.x_stride;
+        float amax = 0.0f;
+        for (int i = lane; i < q.dim; i += 32) amax = fmaxf(amax, fabsf(load_elem(q.x, q.x_dtype, base + i)));
+        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+        const float sc = __fdiv_rn(amax, 448.0f);
+        const int64_t d = q.dst_rows ? q.dst_rows[r] : r;
+        uint8_t *cd = q.codes + d * q.code_stride;
+        for (int i = lane; i < q.dim; i += 32) {
+            const float v = load_elem(q.x, q.x_dtype, base + i);
+            uint32_t c = 0u;
+            if (sc != 0.0f) c = e4m3_code_of_quotient(fabsf(v), sc) | (signbit(v) ? 0x80u : 0u);
+            cd[i] = (uint8_t)c;
+        }
+        if (lane == 0) *reinterpret_cast<float *>(q.scales + d * q.scale_stride) = sc;
+    }
+}
+
+cudaError_t launch_quant_batch(const csa2_quant_job *jobs, int n, cudaStream_t st) {
+    QuantJobs J;
+    J.n = 0;
+    int64_t blocks = 0;
+    for (int i = 0; i < n; ++i) {
+        const csa2_quant_job &s = jobs[i];
+        if (s.rows == 0) continue;
+        QuantJob &q = J.job[J.n];
+        q.fmt = s.fmt; q.x_dtype = s.x_dtype; q.dim = s.dim; q.x = s.x; q.rows = s.rows;
+        q.x_stride = s.x_stride; q.codes = s.codes; q.code_stride = s.code_stride;
+        q.scales = reinterpret_cast<uint8_t *>(s.scales); q.scale_stride = s.scale_stride;
+        q.dst_rows = s.dst_rows;
+        J.block_start[J.n] = blocks;
+        blocks += s.fmt == CSA2_FMT_FP4_E2M1_E4M3S16 ? ceil_div(s.rows * (s.dim / 16), kQuantThreads)
+                                                     : ceil_div(s.rows, kQuantThreads / 32);
+        ++J.n;
+    }
+    J.block_start[J.n] = blocks;
+    if (J.n == 0) return cudaSuccess;
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    quant_batch_kernel<<<(unsigned)blocks, kQuantThreads, 0, st>>>(J);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_fp4(const void *x, int x_dtype, int64_t rows, int dim, int64_t x_stride,
                              uint8_t *codes, int64_t code_stride, uint8_t *scales,
                              int64_t scale_stride, const int64_t *dst_rows, cudaStream_t st) {

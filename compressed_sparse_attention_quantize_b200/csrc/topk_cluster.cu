@@ -46,7 +46,7 @@ struct Args {
 };
 
 CSA2_D int64_t row_n(const Args &a, int r) {
-    if (a.cand) return a.pool_len[r];
+    if (a.cand) return max(a.pool_len[r], 0);
     const int b = r / a.T;
     int64_t n = a.n_entries[b];
     if (a.q_pos) {
@@ -260,6 +260,8 @@ topk_cluster_kernel(Args a) {
 
 int64_t topk_cluster_max_n() { return (int64_t)tkc::kCluster * tkc::kMaxChunk; }
 
+static SmemLimit g_topk_smem;
+
 // Selection for rows [row0, row0+nrows) from scores in global memory (max_n <= topk_cluster_max_n()).
 cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const int32_t *cand,
                                 int cand_stride, const int32_t *n_entries, const int32_t *q_pos,
@@ -274,13 +276,8 @@ cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const
     a.P = P; a.out_pool = out_pool; a.out_pool_len = out_pool_len;
     const int chunk = (int)((max_n + tkc::kCluster - 1) / tkc::kCluster);
     const size_t smem = (size_t)(chunk > 0 ? chunk : 1) * sizeof(uint32_t);
-    static size_t attr_smem = 0;
-    if (smem > attr_smem) {
-        cudaError_t e = cudaFuncSetAttribute(tkc::topk_cluster_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_smem = smem;
-    }
+    cudaError_t e = ensure_smem_limit(g_topk_smem, tkc::topk_cluster_kernel, (int)smem);
+    if (e != cudaSuccess) return e;
     tkc::topk_cluster_kernel<<<nrows * tkc::kCluster, tkc::kThreads, smem, st>>>(a);
     note_launches(1);
     return cudaGetLastError();

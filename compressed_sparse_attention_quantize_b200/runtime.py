@@ -15,7 +15,7 @@ import torch
 
 from . import (DTYPE_BF16, DTYPE_F32, FMT_FP4, FMT_FP8_TOKEN, MODE_FULL, MODE_REINDEX, MODE_REUSE,
                GroupDesc, LayerDesc, csa2_layer_group, csa2_layer_group_workspace_size,
-               csa2_quantize_kv)
+               csa2_quantize_kv, csa2_quantize_kv_batch, quant_job)
 from . import synth
 
 KV_ROW = 288
@@ -136,6 +136,7 @@ class GroupRunner:
                               if step_win_rows else None)
         if step_win_rows:
             assert max(step_win_rows) < self.swa_codes_all.shape[0]
+        self.entry_jobs, self.window_jobs, self.query_jobs = self._write_jobs()
         self.g = self._group_desc()
         self.layer_descs = [self._layer_desc(l) for l in range(len(modes))]
         self.ws_bytes = csa2_layer_group_workspace_size(self.g, self.layer_descs)
@@ -156,6 +157,25 @@ class GroupRunner:
             else:
                 out.extend(b * self.swa_cap + (synth.SWA_WINDOW - 1) + t for t in range(wl.T))
         return out
+
+    def _write_jobs(self):
+        """csa2_quantize_kv_batch jobs of a step's writes: (entry jobs, window jobs, query jobs)."""
+        def fp4(x, codes, scales, cs, ss, dst=None):
+            dt = DTYPE_F32 if x.dtype == torch.float32 else DTYPE_BF16
+            return quant_job(FMT_FP4, x, dt, x.shape[0], x.shape[1], x.stride(0), codes, cs, scales, ss, dst)
+        entries, windows, queries = [], [], []
+        if self.step_rows is not None:
+            entries.append(fp4(self.step_kv, self.kv, self.kv[:, 256:], KV_ROW, KV_ROW, self.step_rows))
+            entries.append(fp4(self.step_ik, self.k_codes, self.k_scales, 32, 4, self.step_rows))
+        if self.step_win_rows is not None:
+            x = self.step_win_lat
+            windows.append(quant_job(FMT_FP8_TOKEN, x, DTYPE_F32, x.shape[0], x.shape[1], x.stride(0),
+                                     self.swa_codes_all, self.swa_codes_all.stride(0), self.swa_scale_all, 4,
+                                     self.step_win_rows))
+        for ld in self.layer_data:
+            if "iq_f32" in ld:
+                queries.append(fp4(ld["iq_f32"], ld["iq_codes"], ld["iq_scales"], 32, 4))
+        return entries, windows, queries
 
     def _group_desc(self) -> GroupDesc:
         wl = self.wl
@@ -197,10 +217,11 @@ class GroupRunner:
         every Full/Reindex layer's indexer query (FP4), and every layer's window entries of the
         step's tokens (E4M3 + fp32 scale, at their window slots; one call for all layers).  The
         inputs are the ones the caches were built from, so the bytes written equal those already
-        there and a step that runs write_step() then run() reads the same caches as run() alone."""
-        self.write_entries(stream)
-        self.write_windows(stream)
-        self.write_queries(stream)
+        there and a step that runs write_step() then run() reads the same caches as run() alone.
+        All of it is one csa2_quantize_kv_batch launch."""
+        jobs = self.entry_jobs + self.window_jobs + self.query_jobs
+        if jobs:
+            csa2_quantize_kv_batch(jobs, stream)
 
     def write_entries(self, stream=None) -> None:
         """The newest compressed entry of every non-empty sequence (main KV, FP4) and its

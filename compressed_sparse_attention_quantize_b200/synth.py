@@ -97,7 +97,8 @@ def workload(i: int) -> Workload:
     raise ValueError(i)
 
 
-def scaled(wl: Workload, *, B=None, n=None, T=None, K=None, P=None, H=None, name=None) -> Workload:
+def scaled(wl: Workload, *, B=None, n=None, T=None, K=None, P=None, H=None, HI=None, modes=None,
+           name=None) -> Workload:
     """A smaller copy of a workload with the same structure (for tests the oracle runs fully)."""
     B = wl.B if B is None else B
     n_entries = list(wl.n_entries[:B]) if n is None else ([n] * B if isinstance(n, int) else list(n))
@@ -107,8 +108,9 @@ def scaled(wl: Workload, *, B=None, n=None, T=None, K=None, P=None, H=None, name
     if wl.prefill_start is not None:
         pstart = ctx[0] - T
     return Workload(name or (wl.name + "_scaled"), wl.seed, B=B, T=T, n_entries=n_entries,
-                    H=wl.H if H is None else H, HI=wl.HI, K=wl.K if K is None else K,
-                    P=wl.P if P is None else P, modes=wl.modes, ctx_tokens=ctx,
+                    H=wl.H if H is None else H, HI=wl.HI if HI is None else HI,
+                    K=wl.K if K is None else K, P=wl.P if P is None else P,
+                    modes=wl.modes if modes is None else tuple(modes), ctx_tokens=ctx,
                     prefill_start=pstart, new_entries=(min(wl.new_entries, n_entries[0])
                                                        if wl.new_entries else 0))
 
@@ -159,6 +161,17 @@ def head_weights(wl: Workload, layer: int, b: int) -> np.ndarray:
 def swa_latent(wl: Workload, layer: int, b: int) -> np.ndarray:
     """Sliding-window token latents of sequence b at a layer: float32 [swa_tokens, 512]."""
     return _latent(_rng(wl.seed, _S_SWA, layer, b), wl.swa_tokens(), outlier_channels(wl.seed))
+
+
+def window_slot(wl: Workload, b: int, token: int) -> int:
+    """Slot of the layer's window buffer that holds absolute token `token` of sequence b.
+
+    Decode keeps a ring of SWA_WINDOW slots, token u in slot u % SWA_WINDOW.  Prefill keeps the
+    SWA_WINDOW - 1 tokens before the chunk followed by the chunk, token u in slot
+    u - (prefill_start - SWA_WINDOW + 1)."""
+    if wl.prefill_start is None:
+        return int(token) % SWA_WINDOW
+    return int(token) - (wl.prefill_start - (SWA_WINDOW - 1))
 
 
 def swa_window(wl: Workload, b: int) -> Tuple[np.ndarray, np.ndarray]:

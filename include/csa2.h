@@ -13,10 +13,10 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
  *    call only enqueues work on it: nothing synchronises the host, so results are valid
  *    once the caller synchronises the stream.  Calls keep no data between calls.  The
- *    library sets up, on its first calls, per-process launch settings (kernels' shared-
- *    memory limits, the SM count, the layer group's side stream per thread).  Make the
- *    first call of each kind from one thread, and drive one GPU per process; after that,
- *    calls from several threads on their own streams are safe.
+ *    library keeps launch settings per device (kernels' shared-memory limits, the SM
+ *    count), set once per device under a lock, and the layer group keeps a side stream
+ *    per host thread and device; calls may come from several host threads, on their own
+ *    streams, for any of the process's devices (the current device at the call).
  *  - Arguments are validated before anything is launched; a call that returns an error
  *    has enqueued nothing.  Faults that happen on the device surface at the caller's
  *    next synchronisation, as for any CUDA kernel.
@@ -110,6 +110,37 @@ CSA2_API csa2_status csa2_quantize_kv(int fmt, const void *x, int x_dtype, int64
                              void *stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa2_quantize_kv_batch -- several csa2_quantize_kv jobs in one kernel launch.
+ *
+ * A decode step writes to several caches at once (the new compressed entry, its indexer key,
+ * the step token's window entry of every layer, the indexer queries); this call quantises all
+ * of them in one launch.  Each job has the arguments, meaning and result of csa2_quantize_kv
+ * ([B] section "FP4 量化 + Bounded Replay"; [A] section "压缩吸收注意力（二代）").  Jobs must
+ * not write overlapping bytes (they run concurrently).
+ * jobs: host array of n_jobs descriptors (read during the call only), 0 <= n_jobs <=
+ *   CSA2_MAX_QUANT_JOBS; jobs with rows == 0 are skipped.
+ * Errors: INVALID_ARG (jobs NULL with n_jobs > 0), SHAPE (n_jobs out of range), and any job's
+ *   csa2_quantize_kv error (nothing is launched then), CUDA.
+ * ---------------------------------------------------------------------------------- */
+#define CSA2_MAX_QUANT_JOBS 16
+
+typedef struct csa2_quant_job {
+    int fmt;                     /* CSA2_FMT_*                                          */
+    int x_dtype;                 /* CSA2_DTYPE_F32 or CSA2_DTYPE_BF16                   */
+    const void *x;               /* rows x dim elements, row r at x + r*x_stride         */
+    int64_t rows;
+    int dim;
+    int64_t x_stride;
+    uint8_t *codes;              /* as csa2_quantize_kv                                 */
+    int64_t code_stride;
+    void *scales;
+    int64_t scale_stride;
+    const int64_t *dst_rows;     /* NULL or int64 [rows] destination rows               */
+} csa2_quant_job;
+
+CSA2_API csa2_status csa2_quantize_kv_batch(const csa2_quant_job *jobs, int n_jobs, void *stream);
+
+/* ------------------------------------------------------------------------------------
  * csa2_compress_quantize_kv -- sequence compressor fused with the FP4 quantise-on-write.
  *
  * [B] section "CSA2：三层压缩一次吃满": along the sequence every m tokens are compressed into
@@ -199,16 +230,22 @@ CSA2_API csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uin
  *
  * Layouts: q bf16 [B*T][H][D]; main entry e at kv + e*kv_row_stride holds D/2 bytes of
  *   E2M1 codes followed by D/16 E4M3 scales (288 bytes for D = 512); entry ids are
- *   relative to seq_start[b]; idx int32 [B*T][K] (-1 = empty slot, ignored); cnt int32
- *   [B*T] or NULL (number of leading non-negative ids; NULL = scan all K);
+ *   relative to seq_start[b]; n_entries int32 [B] (entries of each sequence) or NULL;
+ *   idx int32 [B*T][K] (-1 = empty slot, ignored); cnt int32 [B*T] or NULL (number of
+ *   leading ids to read, 0 <= cnt <= K; NULL = scan all K);
  *   swa_codes u8 [B][swa_cap][D] (E4M3), swa_scale f32 [B][swa_cap]; row r uses slots
  *   swa_start[r] .. swa_start[r]+swa_len[r]-1 of its sequence (swa_start NULL = 0);
  *   out [B*T][H][D] of out_dtype (CSA2_DTYPE_F32 or CSA2_DTYPE_BF16); lse f32 [B*T][H]
  *   or NULL.
- * Caller contract (not checked on the device): every non-negative id in idx names an entry
- *   of its own sequence (id < that sequence's entry count, so the row lies inside kv), and
- *   swa_start[r] + swa_len[r] <= swa_cap.  csa2_index_topk's outputs always satisfy the
- *   first condition.
+ * Caller contract: every non-negative id in idx names an entry of its own sequence (id <
+ *   n_entries[b], so the row lies inside kv), 0 <= swa_len[r] <= CSA2_SWA_WINDOW and
+ *   0 <= swa_start[r], swa_start[r] + swa_len[r] <= swa_cap.  csa2_index_topk's outputs
+ *   always satisfy the first condition.  The kernel checks it as it reads: an id at or
+ *   above n_entries[b] (checked only when n_entries is given) or a window slot outside
+ *   [0, swa_cap) is skipped and the device error word becomes CSA2_ERR_INVALID_ARG; a cnt
+ *   outside [0, K] or a swa_len outside [0, CSA2_SWA_WINDOW] is clamped and the word
+ *   becomes CSA2_ERR_SHAPE (read and clear it with csa2_device_error).  The row of such a
+ *   call is not meaningful, but nothing outside the caller's buffers is read.
  * Limits: D == 512; H a multiple of 16, 16 <= H <= CSA2_MAX_HEADS; 1 <= K <=
  *   CSA2_MAX_TOPK; swa_len <= CSA2_SWA_WINDOW; kv and kv_row_stride 16-byte aligned.
  * Workspace: csa2_sparse_attn_workspace_size(B*T, H, K, &bytes).
@@ -233,7 +270,7 @@ CSA2_API csa2_status csa2_sparse_attn_plan(int rows, int H, int K, int *hgroups,
 
 CSA2_API csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D,
                              const uint8_t *kv, int64_t kv_row_stride, const int64_t *seq_start,
-                             const int32_t *idx, const int32_t *cnt, int K,
+                             const int32_t *n_entries, const int32_t *idx, const int32_t *cnt, int K,
                              const uint8_t *swa_codes, const float *swa_scale, int swa_cap,
                              const int32_t *swa_start, const int32_t *swa_len,
                              float softmax_scale, void *out, int out_dtype, float *lse,
@@ -250,15 +287,18 @@ CSA2_API csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, in
  * forbids device allocations after start-up -- use this call instead.
  *   - The first call on a device looks up the array's address (cudaGetSymbolAddress) with
  *     that device current; make that first call before any stream capture.
+ *   - The split plan is the best one whose partials (131,584 bytes each) fit in the array;
+ *     it may use fewer key splits than csa2_sparse_attn would.  One split per query row
+ *     needs no partials, so every valid shape runs; CSA2_ERR_WORKSPACE would mean a plan
+ *     that does not fit, which cannot happen for arguments that pass validation.
  *   - All calls share the array, and each call fully rewrites what it reads, so nothing needs
  *     clearing; calls whose kernels overlap on the GPU (other streams or host threads) race.
- *   - Returns CSA2_ERR_WORKSPACE when the launch needs more scratch than the array holds
- *     (never on a GPU with <= 159 SMs: the split plan makes at most one partial per SM, each
- *     131,584 bytes); otherwise the errors of csa2_sparse_attn.
+ *   - Otherwise the errors of csa2_sparse_attn.
  * ---------------------------------------------------------------------------------- */
 CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t *q, int B, int T, int H, int D,
                                               const uint8_t *kv, int64_t kv_row_stride,
-                                              const int64_t *seq_start, const int32_t *idx,
+                                              const int64_t *seq_start, const int32_t *n_entries,
+                                              const int32_t *idx,
                                               const int32_t *cnt, int K, const uint8_t *swa_codes,
                                               const float *swa_scale, int swa_cap,
                                               const int32_t *swa_start, const int32_t *swa_len,
@@ -394,8 +434,10 @@ CSA2_API csa2_status csa2_attn_merge_shards(const float *outs, const float *lses
 
 /* ------------------------------------------------------------------------------------
  * csa2_device_error -- reads (and clears) the library's device-side error word for the
- * current device: 0 when no bounded wait has expired since the last call, otherwise a
- * csa2_status code.  Synchronises `stream` first.
+ * current device: 0 when nothing was recorded since the last call, otherwise the first
+ * csa2_status code a kernel recorded: CSA2_ERR_TIMEOUT (a bounded wait expired),
+ * CSA2_ERR_INVALID_ARG or CSA2_ERR_SHAPE (csa2_sparse_attn met an id, window slot or count
+ * outside its caller contract).  Synchronises `stream` first.
  * ---------------------------------------------------------------------------------- */
 CSA2_API csa2_status csa2_device_error(void *stream);
 

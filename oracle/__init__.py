@@ -310,6 +310,27 @@ def visible_entries(q_pos: Optional[int], n_entries: int) -> int:
 
 
 # --------------------------------------------------------------------------
+# sliding window
+# --------------------------------------------------------------------------
+SWA_WINDOW = 128
+
+
+def window_tokens(q_pos: int, window: int = SWA_WINDOW) -> np.ndarray:
+    """Absolute positions of the tokens in the sliding window of the query at position q_pos.
+
+    [B: FP4 量化 + Bounded Replay]: the sliding window is cut down to the most recent 128
+    tokens.  Reading: the query at token p sees token u through the window exactly when u is
+    one of the `window` most recent tokens up to and including p, i.e. p - window < u <= p and
+    u >= 0.  Written out as that definition over the candidate tokens 0..p, ascending.
+    """
+    p = int(q_pos)
+    if p < 0:
+        return np.zeros(0, np.int64)
+    u = np.arange(p + 1, dtype=np.int64)
+    return u[(u > p - int(window)) & (u <= p)]
+
+
+# --------------------------------------------------------------------------
 # layer group (mode table)
 # --------------------------------------------------------------------------
 FULL, REINDEX, REUSE = "F", "I", "U"

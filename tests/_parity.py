@@ -55,11 +55,16 @@ class OracleSeq:
         return oracle.layer_group_indices(modes, inputs, self.k_codes, self.k_scales, n_vis, wl.K,
                                           wl.P)
 
+    def window_slots(self, t: int):
+        """Window-buffer slots of the tokens the oracle puts in query t's window."""
+        qp = int(self.wl.q_pos(self.b)[t])
+        return np.array([synth.window_slot(self.wl, self.b, u) for u in oracle.window_tokens(qp)],
+                        np.int64)
+
     def attention(self, l: int, t: int, idx, softmax_scale):
         L = self.layer(l)
-        st, ln = synth.swa_window(self.wl, self.b)
-        s0, n = int(st[t]), int(ln[t])
-        return oracle.attention(L["q"][t], self.kv_rows, idx, L["swc"][s0:s0 + n], L["sws"][s0:s0 + n],
+        slots = self.window_slots(t)
+        return oracle.attention(L["q"][t], self.kv_rows, idx, L["swc"][slots], L["sws"][slots],
                                 softmax_scale)
 
 

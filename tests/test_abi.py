@@ -83,13 +83,14 @@ def test_compress_validation(L):
 
 
 def _attn(L, **kw):
-    a = dict(q=16, B=1, T=1, H=64, D=512, kv=16, kv_row_stride=288, seq_start=16, idx=16, cnt=None,
+    a = dict(q=16, B=1, T=1, H=64, D=512, kv=16, kv_row_stride=288, seq_start=16, n_entries=None, idx=16, cnt=None,
              K=64, swa_codes=16, swa_scale=16, swa_cap=128, swa_start=None, swa_len=16,
              softmax_scale=1.0, out=16, out_dtype=0, lse=None, workspace=16, ws_bytes=1 << 40,
              stream=None)
     a.update(kw)
     return L.csa2_sparse_attn(a["q"], a["B"], a["T"], a["H"], a["D"], a["kv"], a["kv_row_stride"],
-                              a["seq_start"], a["idx"], a["cnt"], a["K"], a["swa_codes"], a["swa_scale"],
+                              a["seq_start"], a["n_entries"], a["idx"], a["cnt"], a["K"], a["swa_codes"],
+                              a["swa_scale"],
                               a["swa_cap"], a["swa_start"], a["swa_len"], ctypes.c_float(a["softmax_scale"]),
                               a["out"], a["out_dtype"], a["lse"], a["workspace"], a["ws_bytes"], a["stream"])
 
@@ -173,3 +174,43 @@ def test_attention_plan_validation():
         csa2.csa2_sparse_attn_plan(0, 64, 2048)
     with pytest.raises(csa2.CSA2Error):
         csa2.csa2_sparse_attn_plan(32, 64, 0)
+
+
+def test_default_plan_of_the_headline_decode_exceeds_the_noalloc_array():
+    """32 rows x 64 heads x top-2048 (the 128K decode workload): the default split plan's
+    partials need more than the 20 MiB array of csa2_sparse_attn_noalloc, so that call must
+    (and does, on the GPU: tests/test_zz_no_alloc.py) run a plan fitted to the array."""
+    hg, sp, kps = csa2.csa2_sparse_attn_plan(32, 64, 2048)
+    assert sp > 1
+    assert csa2.csa2_sparse_attn_workspace_size(32, 64, 2048) > (20 << 20)
+
+
+def test_noalloc_validation(L):
+    def call(**kw):
+        a = dict(q=16, B=1, T=1, H=64, D=512, kv=16, kv_row_stride=288, seq_start=16, n_entries=None,
+                 idx=16, cnt=None, K=64, swa_codes=16, swa_scale=16, swa_cap=128, swa_start=None,
+                 swa_len=16, softmax_scale=1.0, out=16, out_dtype=0, lse=None, stream=None)
+        a.update(kw)
+        return L.csa2_sparse_attn_noalloc(
+            a["q"], a["B"], a["T"], a["H"], a["D"], a["kv"], a["kv_row_stride"], a["seq_start"],
+            a["n_entries"], a["idx"], a["cnt"], a["K"], a["swa_codes"], a["swa_scale"], a["swa_cap"],
+            a["swa_start"], a["swa_len"], ctypes.c_float(a["softmax_scale"]), a["out"], a["out_dtype"],
+            a["lse"], a["stream"])
+    assert call(D=256) == UNSUP
+    assert call(H=24) == SHAPE
+    assert call(K=5000) == SHAPE
+    assert call(kv=24) == ALIGN
+    assert call(q=None) == INVALID
+
+
+def test_quantize_batch_validation(L):
+    J = csa2.QuantJob
+    ok = csa2.quant_job(0, 16, 0, 4, 512, 512, 16, 256, 16, 32)
+    bad = csa2.quant_job(0, 16, 0, 4, 500, 512, 16, 256, 16, 32)          # dim % 16
+    arr = (J * 2)(ok, bad)
+    assert L.csa2_quantize_kv_batch(arr, 2, None) == SHAPE               # nothing launched
+    assert L.csa2_quantize_kv_batch(arr, 17, None) == SHAPE              # too many jobs
+    assert L.csa2_quantize_kv_batch(None, 1, None) == INVALID
+    assert L.csa2_quantize_kv_batch(None, 0, None) == OK
+    empty = csa2.quant_job(0, None, 0, 0, 512, 512, None, 256, None, 32)
+    assert L.csa2_quantize_kv_batch((J * 1)(empty), 1, None) == OK        # rows == 0 only

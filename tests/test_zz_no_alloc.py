@@ -21,10 +21,12 @@ from tests._parity import check_attention
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
+@pytest.mark.parametrize("B,K", [(4, 256), (32, 2048)])
+def test_noalloc_matches_workspace_entry_point_twice(B, K):
     # 4 rows x 64 heads and top-256 + a 128-token window: 3 key splits per row, so the split
-    # partials (the scratch) are really used.
-    wl = synth.scaled(synth.workload(1), B=4, n=3000, K=256, name="noalloc")
+    # partials (the scratch) are really used.  32 rows x top-2048 is the 128K decode shape, whose
+    # default plan needs more partials than the array holds: the call runs a plan fitted to it.
+    wl = synth.scaled(synth.workload(1), B=B, n=3000, K=K, name="noalloc")
     r = runtime.GroupRunner(wl, layers=2)
     r.run()
     torch.cuda.synchronize()
@@ -34,7 +36,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda")
     for layer in (0, 1):
         ld = r.layer_data[layer]
-        args = (ld["q"], wl.B, wl.T, wl.H, 512, r.kv, 288, r.seq_start, idx, cnt, wl.K,
+        args = (ld["q"], wl.B, wl.T, wl.H, 512, r.kv, 288, r.seq_start, r.n_entries, idx, cnt, wl.K,
                 ld["swa_codes"], ld["swa_scale"], r.swa_cap, r.swa_start, r.swa_len, r.softmax_scale)
         out_ref = torch.empty((r.rows, wl.H, 512), dtype=torch.float32, device="cuda")
         lse_ref = torch.empty((r.rows, wl.H), dtype=torch.float32, device="cuda")
