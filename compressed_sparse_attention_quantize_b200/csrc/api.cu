@@ -113,7 +113,7 @@ size_t attn_ws(int rows, int H, int K) { return round_up(attn_workspace_bytes(ro
 
 size_t index_ws(int mode, int rows, int64_t max_n, int K, int P) {
     const int64_t n = mode == CSA2_MODE_REINDEX ? (int64_t)P : max_n;
-    return round_up(index_topk_workspace_bytes(rows, n, K));
+    return round_up(index_topk_workspace_bytes(rows, n, K, mode == CSA2_MODE_REINDEX ? 0 : P));
 }
 
 }  // namespace

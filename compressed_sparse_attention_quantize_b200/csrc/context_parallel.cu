@@ -103,18 +103,47 @@ cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const
                                 int32_t *out_idx, int32_t *out_cnt, int P, int32_t *out_pool,
                                 int32_t *out_pool_len, int64_t max_n, cudaStream_t st);
 
-size_t topk_merge_workspace_bytes(int G, int rows, int K_in) {
+int topk_row_chunks(int64_t max_n, int K, int P);
+size_t topk_row_scratch_bytes(int rows, int64_t max_n, int K, int P);
+cudaError_t launch_topk_row(const float *scores, int64_t score_stride, const int32_t *cand, int64_t cand_stride,
+                            const int32_t *n_entries, const int32_t *q_pos, const int32_t *pool_len, int T,
+                            int row0, int nrows, int K, int32_t *out_idx, int32_t *out_cnt, int P,
+                            int32_t *out_pool, int32_t *out_pool_len, int64_t max_n, void *scratch,
+                            cudaStream_t st);
+
+// The largest selection scratch any K <= CSA2_MAX_TOPK needs for lists of up to n candidates.
+static size_t merge_select_scratch(int rows, int64_t n) {
+    size_t best = 0;
+    for (int K = 1; K <= CSA2_MAX_TOPK; K *= 2) {
+        const size_t b = topk_row_scratch_bytes(rows, n, K, 0);
+        if (b > best) best = b;
+    }
+    const size_t b = topk_row_scratch_bytes(rows, n, CSA2_MAX_TOPK, 0);
+    return b > best ? b : best;
+}
+
+static size_t merge_list_bytes(int G, int rows, int K_in) {
     const size_t cands = (size_t)rows * G * K_in;
-    return cands * 8 + (size_t)rows * 4 + 256;
+    return (cands * 8 + (size_t)rows * 4 + 255) / 256 * 256;
+}
+
+size_t topk_merge_workspace_bytes(int G, int rows, int K_in) {
+    return merge_list_bytes(G, rows, K_in) + merge_select_scratch(rows, (int64_t)G * K_in) + 256;
 }
 
 cudaError_t launch_topk_merge_shards(const float *scores, const int32_t *ids, const int64_t *id_offset,
                                      const int32_t *cnt, int G, int rows, int K_in, int K, int32_t *out_idx,
                                      int32_t *out_cnt, void *workspace, cudaStream_t st) {
-    if (G == 1 && id_offset == nullptr)         // one list already in place: select from it directly
+    const int64_t stride = (int64_t)G * K_in;
+    void *sel_scratch = reinterpret_cast<uint8_t *>(workspace) + merge_list_bytes(G, rows, K_in);
+    const bool row_path = topk_row_chunks(stride, K, 0) > 0;
+    if (G == 1 && id_offset == nullptr) {       // one list already in place: select from it directly
+        if (row_path)
+            return launch_topk_row(scores, K_in, ids, K_in, nullptr, nullptr, cnt, 1, 0, rows, K, out_idx, out_cnt, 0,
+                                   nullptr, nullptr, K_in, sel_scratch, st);
         return launch_topk_cluster(scores, K_in, ids, K_in, nullptr, nullptr, cnt, 1, 0, rows, K, out_idx, out_cnt, 0,
                                    nullptr, nullptr, K_in, st);
-    const int64_t stride = (int64_t)G * K_in;
+    }
     float *c_scores = reinterpret_cast<float *>(workspace);
     int32_t *c_ids = reinterpret_cast<int32_t *>(c_scores + (size_t)rows * stride);
     int32_t *c_n = c_ids + (size_t)rows * stride;
@@ -123,6 +152,9 @@ cudaError_t launch_topk_merge_shards(const float *scores, const int32_t *ids, co
     note_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (row_path)
+        return launch_topk_row(c_scores, stride, c_ids, stride, nullptr, nullptr, c_n, 1, 0, rows, K, out_idx, out_cnt,
+                               0, nullptr, nullptr, stride, sel_scratch, st);
     return launch_topk_cluster(c_scores, stride, c_ids, (int)stride, nullptr, nullptr, c_n, 1, 0, rows, K,
                                out_idx, out_cnt, 0, nullptr, nullptr, stride, st);
 }

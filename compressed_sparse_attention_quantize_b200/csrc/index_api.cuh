@@ -33,7 +33,7 @@ struct IndexLaunch {
 };
 
 // Scratch bytes for `rows` query rows with up to `n` candidates each.
-size_t index_topk_workspace_bytes(int rows, int64_t n, int K);
+size_t index_topk_workspace_bytes(int rows, int64_t n, int K, int P);
 cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st);
 
 // Device-side error word (bounded waits that expire write a csa2_status here).

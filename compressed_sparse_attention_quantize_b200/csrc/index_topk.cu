@@ -205,10 +205,21 @@ static int64_t index_rows_per_chunk(int rows, int64_t max_n) {
     return per < rows ? per : rows;
 }
 
-size_t index_topk_workspace_bytes(int rows, int64_t n, int K) {
-    (void)K;
+int64_t topk_row_max_n();
+int topk_row_chunks(int64_t max_n, int K, int P);
+size_t topk_row_scratch_bytes(int rows, int64_t max_n, int K, int P);
+cudaError_t launch_topk_row(const float *scores, int64_t score_stride, const int32_t *cand, int64_t cand_stride,
+                            const int32_t *n_entries, const int32_t *q_pos, const int32_t *pool_len, int T,
+                            int row0, int nrows, int K, int32_t *out_idx, int32_t *out_cnt, int P,
+                            int32_t *out_pool, int32_t *out_pool_len, int64_t max_n, void *scratch,
+                            cudaStream_t st);
+
+// Scores of a row chunk, then the selection's scratch (two-phase path for long rows).
+static size_t score_bytes(int64_t chunk, int64_t n) { return ((size_t)(chunk * (n > 0 ? n : 1) * 4) + 255) / 256 * 256; }
+
+size_t index_topk_workspace_bytes(int rows, int64_t n, int K, int P) {
     const int64_t chunk = index_rows_per_chunk(rows, n);
-    return (size_t)(chunk * (n > 0 ? n : 1) * 4 + 256);
+    return score_bytes(chunk, n) + topk_row_scratch_bytes((int)chunk, n, K, P) + 256;
 }
 
 cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, float *scores,
@@ -247,6 +258,17 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
         if (max_n > 0) {
             cudaError_t e = launch_index_score_tc(L, (int)r0, nr, scores, sa.score_stride, st);
             if (e != cudaSuccess) return e;
+        }
+        const int sel_P = reindex ? 0 : L.P;
+        if (topk_row_chunks(max_n, L.K, sel_P) > 0) {
+            void *scratch = reinterpret_cast<uint8_t *>(L.workspace) + score_bytes(chunk, max_n);
+            cudaError_t e = launch_topk_row(scores, sa.score_stride, sa.pool, sa.P_in, sa.n_entries, sa.q_pos,
+                                            sa.pool_len, sa.T, sa.row0, nr, L.K, L.out_idx, L.out_cnt, sel_P,
+                                            L.out_pool, L.out_pool_len, max_n, scratch, st);
+            if (e == cudaSuccess && L.out_scores && !reindex)
+                e = launch_gather_scores(scores, sa.score_stride, L.out_idx, L.K, sa.row0, nr, L.out_scores, st);
+            if (e != cudaSuccess) return e;
+            continue;
         }
         if (max_n <= topk_cluster_max_n()) {
             cudaError_t e = launch_topk_cluster(scores, sa.score_stride, sa.pool, sa.P_in, sa.n_entries,

@@ -328,7 +328,8 @@ def test_full_size_sampled(cfg, rows):
     _check_rows(r, wl, rows)
 
 
-def test_topk_heavy_ties_full_pool_reindex():
+@pytest.mark.parametrize("long_rows", [False, True])
+def test_topk_heavy_ties_full_pool_reindex(long_rows):
     """Selections where exact score ties straddle the K-th and P-th places.
 
     Keys of sequence 0 repeat with period 13, so its ~30000 scores take 13 values and the
@@ -341,7 +342,9 @@ def test_topk_heavy_ties_full_pool_reindex():
     """
     rng = np.random.default_rng(4242)
     H_I, K, P = 8, 2048, 3000
-    n = [30000, 4097, 2048, 0, 30000]
+    # long_rows: rows beyond what one CTA holds in shared memory, so every chunk of a row selects
+    # first and the union is selected again (tie classes then cross chunk boundaries)
+    n = [100000, 4097, 2048, 0, 70000] if long_rows else [30000, 4097, 2048, 0, 30000]
     B = len(n)
     starts = np.concatenate([[0], np.cumsum(n)[:-1]]).astype(np.int64)
     total = int(sum(n))
