@@ -105,7 +105,7 @@ csa2_status check_attn_args(const uint16_t *q, int B, int T, int H, int D, const
     if (kv_row_stride < kKvRowBytes) return CSA2_ERR_SHAPE;
     if (!aligned16(kv) || (kv_row_stride & 15)) return CSA2_ERR_ALIGN;
     if (swa_codes && !aligned16(swa_codes)) return CSA2_ERR_ALIGN;
-    if (!aligned16(q)) return CSA2_ERR_ALIGN;
+    if (!aligned16(q) || !aligned16(out)) return CSA2_ERR_ALIGN;
     return CSA2_OK;
 }
 
@@ -326,6 +326,7 @@ csa2_status csa2_sparse_attn(const uint16_t *q, int B, int T, int H, int D, cons
     if (s != CSA2_OK) return s;
     const int rows = B * T;
     if (!workspace || ws_bytes < attn_ws(rows, H, K)) return CSA2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return CSA2_ERR_ALIGN;
     AttnArgs a;
     a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
     a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start; a.n_entries = n_entries;
@@ -352,6 +353,7 @@ csa2_status csa2_sparse_attn_shard(const uint16_t *q, int B, int T, int H, int D
     if (s != CSA2_OK) return s;
     const int rows = B * T;
     if (!workspace || ws_bytes < attn_ws(rows, H, K)) return CSA2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return CSA2_ERR_ALIGN;
     AttnArgs a;
     a.q = q; a.rows = rows; a.T = T; a.H = H; a.K = K;
     a.kv = kv; a.kv_row_stride = kv_row_stride; a.seq_start = seq_start; a.n_entries = nullptr;
@@ -440,6 +442,7 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     csa2_status s = group_layout(g, layers, n_layers, &idx_off, &pool_off, &iws_off, &attn_off, &total);
     if (s != CSA2_OK) return s;
     if (!workspace || ws_bytes < total) return CSA2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return CSA2_ERR_ALIGN;
     const int rows = g->B * g->T;
     bool need_pool = false;
     for (int l = 0; l < n_layers; ++l) need_pool |= layers[l].mode == CSA2_MODE_REINDEX;

@@ -48,8 +48,17 @@ constexpr int kPBytes = kTile * kHeads * 2;          // 16 KB (one of P_hi, P_lo
 constexpr int kThreads = 288;             // warp 0: MMA issuer; warps 1-8: workers
 constexpr int kWorkers = 256;
 constexpr int kTmemCols = 512;
-constexpr int kOCol = 256;                 // O^T accumulators at columns 256..511
 constexpr int kLCol = 64;                  // per-key row-sum partials at columns 64..127
+// O^T accumulators from column 128.  The first kFolded 128-channel blocks run the P_hi and P_lo
+// products as one N=128 MMA (B = [P_hi | P_lo]: the descriptor's leading-byte offset is the
+// P_hi -> P_lo distance), so V is read once for both; their accumulators are [O(P_hi) | O(P_lo)]
+// (128 columns, added in the epilogue).  The other blocks take both products into one 64-column
+// accumulator.  TMEM holds two folded blocks next to S^T and the row sums.
+constexpr int kFolded = 2;
+CSA2_HD constexpr int o_col(int mb) {
+    return mb < kFolded ? 128 + 128 * mb : 128 + 128 * kFolded + 64 * (mb - kFolded);
+}
+static_assert(o_col(kBlocks - 1) + kHeads <= kTmemCols, "O^T accumulators fit in TMEM");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int32_t kNoKey = INT32_MIN;
 
@@ -57,6 +66,8 @@ struct Smem {
     uint64_t v_full[kBlocks];              // 128-channel block mb of the tile is written
     uint64_t v_empty[kBlocks];             // P.V of 128-channel block mb has completed
     uint64_t s_full, p_full, pv_done, drain;
+    uint64_t q_full;                       // the bulk copy of Q has landed in the staging area
+    uint64_t q_ready;                      // the workers have written the fp16 Q operand
     uint32_t tmem_base;
     int abort_flag;
     int q_exp_max;
@@ -253,6 +264,7 @@ __device__ __noinline__ void issue_mmas(uint32_t tmem, uint8_t *sQ, uint8_t *sV,
                                         Smem &S, int ntiles, volatile int *abort_flag) {
     constexpr uint32_t idesc_s = ptx::idesc_f16_f32(128, kHeads, false, false);
     constexpr uint32_t idesc_pv = ptx::idesc_f16_f32(128, kHeads, true, true);
+    constexpr uint32_t idesc_pv2 = ptx::idesc_f16_f32(128, 2 * kHeads, true, true);
     // S^T = V . Q^T: A = V (K-major), B = Q (K-major); K step = 32 bytes, region = 64 channels
     const uint64_t s_a0 = ptx::sdesc_sw128(ptx::smem_u32(sV), 16, 1024);
     const uint64_t s_b0 = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
@@ -265,6 +277,7 @@ __device__ __noinline__ void issue_mmas(uint32_t tmem, uint8_t *sQ, uint8_t *sV,
         const uint32_t ph = j & 1;
         // S(j) is issued after P.V(j-1), whose P the softmax warps released before p_full(j-1),
         // and s_full(j) completes only after P.V(j-1) has: no separate S-buffer hand-off.
+        if (j == 0 && !ptx::mbar_wait(&S.q_ready, 0, abort_flag)) goto done;      // the fp16 Q operand
 #pragma unroll
         for (int mb = 0; mb < kBlocks; ++mb) {
             if (!ptx::mbar_wait(&S.v_full[mb], ph, abort_flag)) goto done;
@@ -280,20 +293,27 @@ __device__ __noinline__ void issue_mmas(uint32_t tmem, uint8_t *sQ, uint8_t *sV,
         ptx::mma_commit(&S.s_full);
         if (!ptx::mbar_wait(&S.p_full, ph, abort_flag)) break;
         ptx::tc_fence_after();
-        // per 128-channel block: fp16(P) then P - fp16(P) (P exact to ~2^-22) into the same
-        // accumulators, then the block's V bytes are released to the dequantisers
+        // per 128-channel block: fp16(P) and P - fp16(P) (P exact to ~2^-22), then the block's V
+        // bytes are released to the dequantisers.  Folded blocks: one N=128 MMA per key step into
+        // [O(P_hi) | O(P_lo)]; the others: the two halves one after the other into one accumulator.
 #pragma unroll
         for (int mb = 0; mb < kBlocks; ++mb) {
+            const uint64_t a_mb = pv_a0 + (uint64_t)(mb * ((2 * kVRegion) >> 4));
+            if (mb < kFolded) {
 #pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-                ptx::mma_f16_ss(tmem + kOCol + mb * kHeads,
-                                pv_a0 + (uint64_t)(mb * ((2 * kVRegion) >> 4) + kk * (2048 >> 4)),
-                                pv_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    ptx::mma_f16_ss(tmem + o_col(mb), a_mb + (uint64_t)(kk * (2048 >> 4)),
+                                    pv_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv2, (j > 0 || kk > 0) ? 1u : 0u);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-                ptx::mma_f16_ss(tmem + kOCol + mb * kHeads,
-                                pv_a0 + (uint64_t)(mb * ((2 * kVRegion) >> 4) + kk * (2048 >> 4)),
-                                pvlo_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv, 1u);
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    ptx::mma_f16_ss(tmem + o_col(mb), a_mb + (uint64_t)(kk * (2048 >> 4)),
+                                    pv_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    ptx::mma_f16_ss(tmem + o_col(mb), a_mb + (uint64_t)(kk * (2048 >> 4)),
+                                    pvlo_b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv, 1u);
+            }
             ptx::mma_commit(&S.v_empty[mb]);
         }
         ptx::mma_commit(&S.pv_done);
@@ -359,6 +379,8 @@ attn_tc_kernel(AttnArgs a) {
         ptx::mbar_init(&S.p_full, kWorkers);
         ptx::mbar_init(&S.pv_done, 1);
         ptx::mbar_init(&S.drain, 1);
+        ptx::mbar_init(&S.q_full, 1);
+        ptx::mbar_init(&S.q_ready, kWorkers);
         S.abort_flag = 0;
         S.q_exp_max = 0;
         ptx::fence_async_smem();
@@ -368,56 +390,18 @@ attn_tc_kernel(AttnArgs a) {
         ptx::tmem_alloc(&S.tmem_base, kTmemCols);
         ptx::tmem_relinquish();
     }
-    // Q: every thread loads its chunks once; the largest bf16 exponent of the head group picks a
-    // power-of-two pre-scale so the fp16 copy keeps full precision for small values.
-    const uint16_t *qrow = a.q + (int64_t)r * a.H * kLatent;
+    // Q arrives by bulk copy (hcount heads x 1 KB, contiguous) into the upper half of the V buffer,
+    // which the first tile's dequantisation writes last; the workers turn it into the swizzled fp16
+    // operand between the first tile's channel blocks 1 and 2 (stage_q below).
+    const uint16_t *qrow = a.q + ((int64_t)r * a.H + h0) * kLatent;
     const int hcount = min(kHeads, a.H - h0);
-    constexpr int kQChunks = kHeads * (kLatent / 8);                 // 16-byte chunks
-    constexpr int kQPer = (kQChunks + kThreads - 1) / kThreads;
-    uint4 qreg[kQPer];
-    {
-        int emax = 0;
-#pragma unroll
-        for (int k = 0; k < kQPer; ++k) {
-            const int i = threadIdx.x + k * kThreads;
-            const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
-            qreg[k] = make_uint4(0u, 0u, 0u, 0u);
-            if (i < kQChunks && h < hcount)
-                qreg[k] = *reinterpret_cast<const uint4 *>(qrow + (int64_t)(h0 + h) * kLatent + c8 * 8);
-        }
-#pragma unroll
-        for (int k = 0; k < kQPer; ++k) {
-            const uint32_t w[4] = {qreg[k].x, qreg[k].y, qreg[k].z, qreg[k].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                emax = max(emax, (int)((w[e] >> 7) & 0xFFu));
-                emax = max(emax, (int)((w[e] >> 23) & 0xFFu));
-            }
-        }
-        emax = __reduce_max_sync(0xffffffffu, emax);
-        __syncthreads();                                   // barrier init visible
-        if (lane == 0) atomicMax(&S.q_exp_max, emax);
-    }
-    __syncthreads();
-    // the largest |q| lands in [2^13, 2^14): far from fp16 overflow, far above its subnormals
-    const int qshift = S.q_exp_max == 0 ? 0 : (13 - (S.q_exp_max - 127));
-    const float qmul = exp2f((float)qshift);
-#pragma unroll
-    for (int k = 0; k < kQPer; ++k) {
-        const int i = threadIdx.x + k * kThreads;
-        if (i < kQChunks) {
-            const int h = i / (kLatent / 8), c8 = i % (kLatent / 8);
-            const uint32_t w[4] = {qreg[k].x, qreg[k].y, qreg[k].z, qreg[k].w};
-            uint32_t packed[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const __half2 hh = __floats2half2_rn(__uint_as_float(w[e] << 16) * qmul,
-                                                     __uint_as_float(w[e] & 0xFFFF0000u) * qmul);
-                packed[e] = *reinterpret_cast<const uint32_t *>(&hh);
-            }
-            *reinterpret_cast<uint4 *>(sQ + (c8 >> 3) * kQRegion + sw128_off(h, c8 & 7)) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        }
+    uint8_t *sQstage = sV + 4 * kVRegion;                 // V regions 4..7 (64 KB)
+    if (threadIdx.x == 0 && ntiles > 0) {
+        const uint32_t bytes = (uint32_t)hcount * kLatent * 2;
+        ptx::mbar_arrive_expect_tx(&S.q_full, bytes);
+        for (uint32_t off = 0; off < bytes; off += 16384u)
+            ptx::bulk_load_g2s(sQstage + off, reinterpret_cast<const uint8_t *>(qrow) + off,
+                               min(16384u, bytes - off), &S.q_full);
     }
     ptx::fence_async_smem();
     ptx::tc_fence_before();
@@ -435,10 +419,59 @@ attn_tc_kernel(AttnArgs a) {
         const int half = hsel;
         const int wt = threadIdx.x - 32;                 // 0..255
         const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
-        const float qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-qshift);
         // A wait that fails (abort or timeout) only marks `bad`; every worker keeps taking the
         // same barriers, and the decision to stop is collective (bar.red.or) once per tile.
         bool bad = false, aborted = false;
+        // Q from the staging area into the swizzled fp16 operand (workers only, once, between the
+        // first tile's channel blocks 1 and 2): the largest bf16 exponent of the head group picks
+        // a power-of-two pre-scale so that the fp16 copy keeps full precision for small values;
+        // heads past the last are zero.  Returns that shift.
+        auto stage_q = [&]() -> int {
+            constexpr int kChunksPer = kHeads * (kLatent / 8) / kWorkers;    // 16-byte chunks per worker
+            if (!ptx::mbar_wait(&S.q_full, 0, abort_flag)) bad = true;
+            int emax = 0;
+#pragma unroll 4
+            for (int k = 0; k < kChunksPer; ++k) {
+                const int i = wt + k * kWorkers;
+                if ((i >> 6) < hcount) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(sQstage + i * 16);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        emax = max(emax, (int)((w[e] >> 7) & 0xFFu));
+                        emax = max(emax, (int)((w[e] >> 23) & 0xFFu));
+                    }
+                }
+            }
+            emax = __reduce_max_sync(0xffffffffu, emax);
+            if (lane == 0) atomicMax(&S.q_exp_max, emax);
+            ptx::named_barrier(1, kWorkers);
+            // the largest |q| lands in [2^13, 2^14): far from fp16 overflow, far above its subnormals
+            const int qs = S.q_exp_max == 0 ? 0 : (13 - (S.q_exp_max - 127));
+            const float qmul = exp2f((float)qs);
+#pragma unroll 4
+            for (int k = 0; k < kChunksPer; ++k) {
+                const int i = wt + k * kWorkers;
+                const int h = i >> 6, c8 = i & 63;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (h < hcount) v = *reinterpret_cast<const uint4 *>(sQstage + i * 16);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t packed[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __half2 hh = __floats2half2_rn(__uint_as_float(w[e] << 16) * qmul,
+                                                         __uint_as_float(w[e] & 0xFFFF0000u) * qmul);
+                    packed[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                }
+                *reinterpret_cast<uint4 *>(sQ + (c8 >> 3) * kQRegion + sw128_off(h, c8 & 7)) =
+                    make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+            ptx::fence_async_smem();
+            ptx::mbar_arrive(&S.q_ready);
+            ptx::named_barrier(1, kWorkers);             // every worker is done with the staging area
+            return qs;
+        };
+        float qk_scale = 0.0f;
         // this key's share of the row sums lives in TMEM (lane = key, 32 columns per half)
         const uint32_t l_addr = lane_addr + kLCol + half * 32;
         {
@@ -456,6 +489,8 @@ attn_tc_kernel(AttnArgs a) {
             //      finished with it
 #pragma unroll
             for (int mb = 0; mb < kBlocks; ++mb) {
+                if (j == 0 && mb == 2)                   // Q's staging area is blocks 2 and 3
+                    qk_scale = a.softmax_scale * 1.4426950408889634f * exp2f((float)-stage_q());
                 if (j > 0 && !ptx::mbar_wait(&S.v_empty[mb], ph ^ 1, abort_flag)) bad = true;
                 const int rg = 2 * mb + hsel;
                 uint4 out[8];
@@ -574,9 +609,10 @@ attn_tc_kernel(AttnArgs a) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) al[i] = S.alpha[half * 32 + i];
 #pragma unroll 1
-                for (int mb = 0; mb < kBlocks; ++mb) {
+                for (int acc = 0; acc < kBlocks + kFolded; ++acc) {      // every accumulator, lo halves last
                     uint32_t u[32];
-                    const uint32_t addr = lane_addr + kOCol + mb * kHeads + half * 32;
+                    const int mb = acc < kBlocks ? acc : acc - kBlocks;
+                    const uint32_t addr = lane_addr + o_col(mb) + (acc < kBlocks ? 0 : kHeads) + half * 32;
                     ptx::tmem_ld32(addr, u);
                     ptx::tmem_ld_wait();
 #pragma unroll
@@ -609,27 +645,38 @@ attn_tc_kernel(AttnArgs a) {
         }
         ptx::named_barrier(1, kWorkers);
         if (!aborted) {
+            // The result goes through shared memory (the Q and V buffers are free: every MMA has
+            // completed) and leaves with bulk stores: a split's partial [m(64) | l(64) | O(64 x 512)]
+            // fp32, or the single split's normalised output rows (heads h0 .. h0 + hcount - 1 of
+            // row r are contiguous).  One worker issues the stores and waits for them.
             const bool single = a.splits == 1;
-            const int64_t part_idx = ((int64_t)r * a.hgroups + hg) * a.splits + split;
-            float *part = a.partials + part_idx * kPartialFloats;
+            float *stg = reinterpret_cast<float *>(sQ);
             if (wt < kHeads) {
                 const float l = ntiles > 0 ? X.red[0][wt] + X.red[1][wt] + X.red[2][wt] + X.red[3][wt] : 0.0f;
                 X.inv_l[wt] = l > 0.0f ? 1.0f / l : 0.0f;       // 1/l for the single-split output
                 if (!single) {
-                    part[wt] = ntiles > 0 ? S.m_run[wt] : -INFINITY;
-                    part[kHeads + wt] = l;
+                    stg[wt] = ntiles > 0 ? S.m_run[wt] : -INFINITY;
+                    stg[kHeads + wt] = l;
                 } else if (a.lse && h0 + wt < a.H) {
                     a.lse[(int64_t)r * a.H + h0 + wt] =
                         (l > 0.0f) ? (S.m_run[wt] + log2f(l)) * 0.6931471805599453f : -INFINITY;
                 }
             }
             ptx::named_barrier(1, kWorkers);
+            const bool bf16_out = single && a.out_dtype == CSA2_DTYPE_BF16;
 #pragma unroll 1
             for (int mb = 0; mb < kBlocks; ++mb) {
                 const int c = mb * 128 + t;               // this thread's channel
                 uint32_t u[32];
                 if (ntiles > 0) {
-                    ptx::tmem_ld32(lane_addr + kOCol + mb * kHeads + half * 32, u);
+                    ptx::tmem_ld32(lane_addr + o_col(mb) + half * 32, u);
+                    if (mb < kFolded) {                   // add the P_lo accumulator
+                        uint32_t v[32];
+                        ptx::tmem_ld32(lane_addr + o_col(mb) + kHeads + half * 32, v);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) + __uint_as_float(v[i]));
+                    }
                     ptx::tmem_ld_wait();
                 } else {
 #pragma unroll
@@ -638,24 +685,41 @@ attn_tc_kernel(AttnArgs a) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int h = half * 32 + i;
-                    if (h0 + h >= a.H) continue;
                     const float o = __uint_as_float(u[i]);
-                    if (!single) {
-                        part[2 * kHeads + h * kLatent + c] = o;
-                    } else {
-                        const float val = o * X.inv_l[h];
-                        const int64_t oi = ((int64_t)r * a.H + h0 + h) * kLatent + c;
-                        if (a.out_dtype == CSA2_DTYPE_F32)
-                            reinterpret_cast<float *>(a.out)[oi] = val;
-                        else
-                            reinterpret_cast<__nv_bfloat16 *>(a.out)[oi] = __float2bfloat16_rn(val);
-                    }
+                    if (!single)
+                        stg[2 * kHeads + h * kLatent + c] = o;
+                    else if (!bf16_out)
+                        stg[h * kLatent + c] = o * X.inv_l[h];
+                    else
+                        reinterpret_cast<__nv_bfloat16 *>(stg)[h * kLatent + c] = __float2bfloat16_rn(o * X.inv_l[h]);
                 }
+            }
+            ptx::fence_async_smem();
+            ptx::named_barrier(1, kWorkers);
+            if (wt == 0) {
+                uint8_t *dst;
+                uint32_t bytes;
+                if (!single) {
+                    const int64_t part_idx = ((int64_t)r * a.hgroups + hg) * a.splits + split;
+                    dst = reinterpret_cast<uint8_t *>(a.partials + part_idx * kPartialFloats);
+                    bytes = (uint32_t)(kPartialFloats * sizeof(float));
+                } else {
+                    const int es = bf16_out ? 2 : 4;
+                    dst = reinterpret_cast<uint8_t *>(a.out) + ((int64_t)r * a.H + h0) * kLatent * es;
+                    bytes = (uint32_t)(hcount * kLatent * es);
+                }
+                const uint8_t *src8 = reinterpret_cast<const uint8_t *>(stg);
+                for (uint32_t off = 0; off < bytes; off += 16384u)
+                    ptx::bulk_store_s2g(dst + off, src8 + off, min(16384u, bytes - off));
+                ptx::bulk_commit();
+                ptx::bulk_wait_all();
             }
         }
     }
 
     // ---------------- teardown ----------------
+    // the bulk copy of Q has landed before the CTA exits (already so unless the CTA gave up early)
+    if (threadIdx.x == 0 && ntiles > 0) ptx::mbar_wait_drain(&S.q_full, 0);
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 0) {

@@ -7,19 +7,21 @@
 //
 // A list is a sequence of (score, id) candidates whose ids ascend with the position (a row's
 // consecutive entries, a Reindex pool, or the concatenated per-chunk selections of a long row),
-// so "lower index first" on ties is "earlier position first".  One CTA:
-//   1. loads the list's order-preserving 32-bit keys into shared memory and builds the histogram
-//      of their top 11 bits on the way (warp-aggregated shared atomics);
-//   2. finds the exact threshold key of the k-th place in three digits (11, 11 and 10 bits): the
-//      first from that histogram, the others from histograms of the keys that match the prefix
-//      found so far (one pass over shared memory each);
+// so "lower index first" on ties is "earlier position first".  One CTA of 1024 threads:
+//   1. loads the list's order-preserving 32-bit keys into shared memory (16 independent loads in
+//      flight per thread) and counts their top 8 bits on the way;
+//   2. finds the exact threshold key of the k-th place in four 8-bit digits.  Histograms are
+//      per lane (bin b of lane l at b * 32 + l), so the 32 lanes of a warp always add into 32
+//      different banks.  After the first digit the keys of the threshold bin are copied into a
+//      candidate array (when they fit), and the three refinement digits scan only those;
 //   3. writes the selection in position order: each thread owns a consecutive run of keys, and
 //      two block scans (equal keys before the run, then selected keys before it) give every
-//      thread its output offset.
+//      thread its output offset.  Lists with explicit ids first write positions, then map them
+//      to ids in a second, coalesced pass.
 // The pool (top-P of the same order) is a second selection over the same keys, reusing the first
-// histogram.  Lists longer than shared memory holds go through two phases: every chunk of a row
-// selects its top-max(K, P) with their scores, then one CTA per row selects from the union of the
-// chunk selections (the row's top-k lies inside it, and the union keeps position order).
+// digit's histogram.  Lists longer than shared memory holds go through two phases: every chunk of
+// a row selects its top-max(K, P) with their scores, then one CTA per row selects from the union
+// of the chunk selections (the row's top-k lies inside it, and the union keeps position order).
 #include "common.cuh"
 
 namespace csa2 {
@@ -27,9 +29,11 @@ namespace tkr {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxKeys = 45056;                    // keys per CTA in shared memory (176 KB)
+constexpr int kUnroll = 16;                        // independent loads in flight per thread
+constexpr int kMaxKeys = 36864;                    // keys per CTA in shared memory (144 KB)
+constexpr int kCandCap = 8192;                     // keys of the threshold bin kept apart (32 KB)
 constexpr int kChunk = 32768;                      // chunk length of the two-phase path
-constexpr int kBins = 2048;                        // 11-bit digits (the last one has 10 bits)
+constexpr int kBins = 256;                         // 8-bit digits
 constexpr int kMaxSeg = 32;                        // segments of a phase-2 list
 
 // One CTA's list: nseg segments in order; segment s holds cnt[s] candidates with scores at
@@ -79,12 +83,14 @@ struct Args {
 };
 
 struct Shared {
-    unsigned int hist1[kBins];                     // top-digit histogram of all keys (kept)
-    unsigned int hist[kBins];                      // histogram of the current refinement digit
+    unsigned int hp[kBins * 32];                   // per-lane histograms
+    unsigned int hist[kBins];                      // their sum (current digit)
+    unsigned int hist1[kBins];                     // the first digit's sum over all keys (kept)
     int seg_start[kMaxSeg + 1];
     int warp_sums[kWarps + 1];
     uint32_t prefix, mask;
     int remaining;
+    int ncand;
     List list;
 };
 
@@ -122,22 +128,34 @@ CSA2_D int block_excl_sum(int v, int *ws, int &total) {
     return res;
 }
 
-// Warp-aggregated histogram add: lanes with the same bin add once (nearby scores share their top
-// digits, which would serialise plain shared-memory atomics).
-CSA2_D void hist_add(unsigned int *h, bool in, uint32_t bin) {
-    const uint32_t b = in ? bin : 0xFFFFFFFFu;
-    const unsigned peers = __match_any_sync(0xffffffffu, b);
-    if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], (unsigned)__popc(peers));
+CSA2_D void hist_add(Shared &S, uint32_t bin) { atomicAdd(&S.hp[bin * 32 + (threadIdx.x & 31)], 1u); }
+
+CSA2_D void hist_clear(Shared &S) {
+    for (int i = threadIdx.x; i < kBins * 32; i += kThreads) S.hp[i] = 0u;
 }
 
-// Warp 0 finds, in histogram h, the digit d where the count from the top crosses `rem`; it sets
-// S.prefix |= d << shift, S.mask |= digit mask, S.remaining = rem - (count above d).
-CSA2_D void pick_digit(Shared &S, const unsigned int *h, int nbins, int shift) {
+// dst[b] = sum over lanes of hp[b * 32 + lane]; warp w sums bins w, w + 32, ...
+CSA2_D void hist_reduce(Shared &S, unsigned int *dst) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int b = warp; b < kBins; b += kWarps) {
+        const unsigned v = __reduce_add_sync(0xffffffffu, S.hp[b * 32 + lane]);
+        if (lane == 0) dst[b] = v;
+    }
+}
+
+// Warp 0 finds, in histogram h, the digit d where the count from the top crosses S.remaining;
+// it sets S.prefix |= d << shift, S.mask |= 0xFF << shift, S.remaining -= (count above d).
+CSA2_D void pick_digit(Shared &S, const unsigned int *h, int shift) {
     if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
-    const int per = nbins / 32;                    // bins owned by a lane: [per*lane, per*lane+per)
+    constexpr int per = kBins / 32;                // bins owned by a lane: [per*lane, per*lane+per)
+    unsigned int bins[per];
     unsigned int local = 0;
-    for (int i = 0; i < per; ++i) local += h[lane * per + i];
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+        bins[i] = h[lane * per + i];
+        local += bins[i];
+    }
     unsigned int suffix = local;                   // sum over lanes >= lane
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -153,37 +171,54 @@ CSA2_D void pick_digit(Shared &S, const unsigned int *h, int nbins, int shift) {
         int acc = (int)above;
         int d = per - 1;
         for (; d > 0; --d) {
-            const int c = (int)h[lane * per + d];
-            if (acc + c >= rem) break;
-            acc += c;
+            if (acc + (int)bins[d] >= rem) break;
+            acc += (int)bins[d];
         }
         S.remaining = rem - acc;
         S.prefix |= (uint32_t)(lane * per + d) << shift;
-        S.mask |= (uint32_t)(nbins - 1) << shift;
+        S.mask |= 0xFFu << shift;
     }
 }
 
 // Threshold key of the k-th place among the m keys (k < m) and how many keys equal to it are
-// taken.  hist1 must hold the top-digit histogram of all keys.
-CSA2_D void threshold(Shared &S, const uint32_t *keys, int m, int k, uint32_t &thr, int &need_eq) {
-    if (threadIdx.x == 0) { S.prefix = 0u; S.mask = 0u; S.remaining = k; }
+// taken.  S.hist1 holds the first digit's histogram of all keys.
+CSA2_D void threshold(Shared &S, const uint32_t *keys, uint32_t *cand, int m, int k, uint32_t &thr,
+                      int &need_eq) {
+    if (threadIdx.x == 0) { S.prefix = 0u; S.mask = 0u; S.remaining = k; S.ncand = 0; }
     __syncthreads();
-    pick_digit(S, S.hist1, kBins, 21);
+    pick_digit(S, S.hist1, 24);
     __syncthreads();
-    // digits 2 (bits 20..10) and 3 (bits 9..0) over the keys matching the prefix
-    for (int pass = 0; pass < 2; ++pass) {
-        const int shift = pass == 0 ? 10 : 0;
-        const int nb = pass == 0 ? kBins : kBins / 2;
-        for (int i = threadIdx.x; i < nb; i += kThreads) S.hist[i] = 0u;
-        __syncthreads();
-        const uint32_t prefix = S.prefix, mask = S.mask;
+    // the keys of the threshold bin, when they fit the candidate array (order does not matter)
+    const uint32_t d1 = S.prefix >> 24;
+    const bool compact = S.hist1[d1] <= (unsigned)kCandCap;
+    if (compact) {
         for (int base = 0; base < m; base += kThreads) {
             const int i = base + threadIdx.x;
             const uint32_t key = i < m ? keys[i] : 0u;
-            hist_add(S.hist, i < m && (key & mask) == prefix, (key >> shift) & (uint32_t)(nb - 1));
+            const bool in = i < m && (key >> 24) == d1;
+            const unsigned bal = __ballot_sync(0xffffffffu, in);
+            int off = 0;
+            if ((threadIdx.x & 31) == 0 && bal) off = atomicAdd(&S.ncand, __popc(bal));
+            off = __shfl_sync(0xffffffffu, off, 0);
+            if (in) cand[off + __popc(bal & ((1u << (threadIdx.x & 31)) - 1u))] = key;
         }
         __syncthreads();
-        pick_digit(S, S.hist, nb, shift);
+    }
+    const uint32_t *src = compact ? cand : keys;
+    const int n = compact ? S.ncand : m;
+    for (int pass = 1; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        hist_clear(S);
+        __syncthreads();
+        const uint32_t prefix = S.prefix, mask = S.mask;
+        for (int i = threadIdx.x; i < n; i += kThreads) {
+            const uint32_t key = src[i];
+            if ((key & mask) == prefix) hist_add(S, (key >> shift) & 255u);
+        }
+        __syncthreads();
+        hist_reduce(S, S.hist);
+        __syncthreads();
+        pick_digit(S, S.hist, shift);
         __syncthreads();
     }
     thr = S.prefix;
@@ -196,10 +231,23 @@ CSA2_D int seg_of(const Shared &S, int pos, int s) {
     return s;
 }
 
+CSA2_D int32_t id_at(const Shared &S, int pos) {
+    int lo = 0, hi = S.list.nseg - 1;              // last segment whose start <= pos
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (S.seg_start[mid] <= pos) lo = mid; else hi = mid - 1;
+    }
+    const int j = pos - S.seg_start[lo];
+    return S.list.id[lo] ? __ldg(S.list.id[lo] + j) : (int32_t)(S.list.id_base[lo] + j);
+}
+
 // Writes the selection (k < m) or every candidate (k >= m) in position order to out[0..k) (ids),
-// out_scores (optional), pads with -1 and stores the count.
+// out_scores (optional), pads with -1 and stores the count.  `direct`: ids are positions plus
+// id_base[0] (one segment without explicit ids), so they are written at once; otherwise the
+// positions are written first and mapped to ids in a second pass.
 CSA2_D void emit(Shared &S, const uint32_t *keys, int m, int k, bool select, uint32_t thr, int need_eq,
                  int32_t *out, float *out_scores, int32_t *cnt_out) {
+    const bool direct = S.list.nseg == 1 && S.list.id[0] == nullptr;
     const int per = ((m + kThreads - 1) / kThreads) | 1;     // odd: a warp's lanes hit 32 banks
     const int i0 = min(m, (int)threadIdx.x * per), i1 = min(m, i0 + per);
     int my_gt = 0, my_eq = 0;
@@ -218,16 +266,13 @@ CSA2_D void emit(Shared &S, const uint32_t *keys, int m, int k, bool select, uin
     int sel_tot;
     int o = block_excl_sum(my_gt + take, S.warp_sums, sel_tot);
     int eq_seen = 0;
-    int s = i0 < m ? seg_of(S, i0, 0) : 0;
+    const int64_t base = S.list.id_base[0];
     for (int i = i0; i < i1; ++i) {
         const uint32_t key = keys[i];
         const bool sel = !select || key > thr || (key == thr && eq_seen++ < take);
         if (sel) {
-            s = seg_of(S, i, s);
-            const int j = i - S.seg_start[s];
-            const int32_t id = S.list.id[s] ? S.list.id[s][j] : (int32_t)(S.list.id_base[s] + j);
             if (o < k) {
-                out[o] = id;
+                out[o] = direct ? (int32_t)(base + i) : i;
                 if (out_scores) out_scores[o] = key_to_float(key);
             }
             ++o;
@@ -239,6 +284,22 @@ CSA2_D void emit(Shared &S, const uint32_t *keys, int m, int k, bool select, uin
         if (out_scores) out_scores[i] = -INFINITY;
     }
     if (threadIdx.x == 0 && cnt_out) *cnt_out = c;
+    if (!direct) {
+        __syncthreads();                            // every position is written
+        for (int i0b = 0; i0b < c; i0b += kThreads * 8) {
+            int32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0b + u * kThreads + threadIdx.x;
+                v[u] = i < c ? id_at(S, out[i]) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0b + u * kThreads + threadIdx.x;
+                if (i < c) out[i] = v[u];
+            }
+        }
+    }
     __syncthreads();
 }
 
@@ -255,7 +316,8 @@ CSA2_D int64_t row_len(const Args &a, int r) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(Args a) {
-    extern __shared__ __align__(16) uint32_t keys[];
+    extern __shared__ __align__(16) uint32_t keys[];     // kMaxKeys keys, then kCandCap candidates
+    uint32_t *cand = keys + kMaxKeys;
     __shared__ Shared S;
     const int lr = blockIdx.y;
     const int r = a.row0 + lr;
@@ -292,20 +354,40 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(Args a) {
         }
         for (int s = L.nseg; s <= kMaxSeg; ++s) S.seg_start[s] = acc;
     }
-    for (int i = threadIdx.x; i < kBins; i += kThreads) S.hist1[i] = 0u;
+    hist_clear(S);
     __syncthreads();
     const int m = S.seg_start[kMaxSeg];
-    // ---- keys into shared memory, top-digit histogram on the way
-    for (int base = 0; base < m; base += kThreads) {
-        const int i = base + threadIdx.x;
-        uint32_t key = 0u;
-        if (i < m) {
-            const int s = seg_of(S, i, 0);
-            key = float_key(S.list.score[s][i - S.seg_start[s]]);
-            keys[i] = key;
+    // ---- keys into shared memory, kUnroll independent loads per thread at a time; the first
+    //      digit's histogram on the way
+    const bool one_seg = S.list.nseg == 1;
+    const float *sc0 = S.list.score[0];
+    for (int base = 0; base < m; base += kThreads * kUnroll) {
+        float v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = base + u * kThreads + threadIdx.x;
+            v[u] = 0.0f;
+            if (i < m) {
+                if (one_seg) {
+                    v[u] = __ldg(sc0 + i);
+                } else {
+                    const int s = seg_of(S, i, 0);
+                    v[u] = __ldg(S.list.score[s] + (i - S.seg_start[s]));
+                }
+            }
         }
-        hist_add(S.hist1, i < m, key >> 21);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = base + u * kThreads + threadIdx.x;
+            if (i < m) {
+                const uint32_t key = float_key(v[u]);
+                keys[i] = key;
+                hist_add(S, key >> 24);
+            }
+        }
     }
+    __syncthreads();
+    hist_reduce(S, S.hist1);
     __syncthreads();
     // ---- selections
     if (a.phase1) {
@@ -313,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(Args a) {
         uint32_t thr = 0u;
         int need_eq = 0;
         const bool sel = a.kc < m;
-        if (sel) threshold(S, keys, m, a.kc, thr, need_eq);
+        if (sel) threshold(S, keys, cand, m, a.kc, thr, need_eq);
         emit(S, keys, m, a.kc, sel, thr, need_eq, a.ph1_ids + o, a.ph1_scores + o,
              a.ph1_cnt + (int64_t)lr * gridDim.x + blockIdx.x);
         return;
@@ -327,12 +409,12 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(Args a) {
         uint32_t thr = 0u;
         int need_eq = 0;
         const bool sel = k < m;
-        if (sel) threshold(S, keys, m, k, thr, need_eq);
+        if (sel) threshold(S, keys, cand, m, k, thr, need_eq);
         emit(S, keys, m, k, sel, thr, need_eq, out, nullptr, cnt);
     }
 }
 
-constexpr size_t kSmemBytes = (size_t)kMaxKeys * sizeof(uint32_t);
+constexpr size_t kSmemBytes = (size_t)(kMaxKeys + kCandCap) * sizeof(uint32_t);
 
 }  // namespace tkr
 
@@ -340,8 +422,8 @@ static SmemLimit g_topk_row_smem;
 
 int64_t topk_row_max_n() { return tkr::kMaxKeys; }
 
-// Chunks per row and candidates per chunk of the two-phase path for rows of up to max_n
-// candidates, or 0 when the union of the chunks' selections would not fit one CTA.
+// Chunks per row of the two-phase path for rows of up to max_n candidates (1: one CTA per row),
+// or 0 when the union of the chunks' selections would not fit one CTA.
 int topk_row_chunks(int64_t max_n, int K, int P) {
     if (max_n <= tkr::kMaxKeys) return 1;
     const int64_t chunks = ceil_div(max_n, (int64_t)tkr::kChunk);

@@ -247,7 +247,8 @@ CSA2_API csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uin
  *   becomes CSA2_ERR_SHAPE (read and clear it with csa2_device_error).  The row of such a
  *   call is not meaningful, but nothing outside the caller's buffers is read.
  * Limits: D == 512; H a multiple of 16, 16 <= H <= CSA2_MAX_HEADS; 1 <= K <=
- *   CSA2_MAX_TOPK; swa_len <= CSA2_SWA_WINDOW; kv and kv_row_stride 16-byte aligned.
+ *   CSA2_MAX_TOPK; swa_len <= CSA2_SWA_WINDOW; q, kv, kv_row_stride, swa_codes, out and
+ *   workspace 16-byte aligned.
  * Workspace: csa2_sparse_attn_workspace_size(B*T, H, K, &bytes).
  * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED (D != 512), WORKSPACE, CUDA.
  * ---------------------------------------------------------------------------------- */
