@@ -369,3 +369,63 @@ def layer_group_indices(modes: Sequence[str], layer_index_inputs, k_codes, k_sca
             raise ValueError(f"unknown mode {m!r}")
         out.append((idx, cnt))
     return out
+
+
+# --------------------------------------------------------------------------
+# pool maintenance across decode steps
+# --------------------------------------------------------------------------
+def extend_pool(pool: np.ndarray, pool_len: int, n_ref: int, n_vis: int) -> np.ndarray:
+    """Reindex candidates between pool refreshes: the kept pool (built when the sequence had
+    n_ref entries) followed by every entry written since that the query may see (ids n_ref ..
+    n_vis - 1), ascending."""
+    kept = np.asarray(pool[:pool_len], np.int32)
+    new = np.arange(int(n_ref), max(int(n_ref), int(n_vis)), dtype=np.int32)
+    return np.concatenate([kept, new]).astype(np.int32)
+
+
+def decode_steps_with_pool(modes: Sequence[str], step_inputs, k_codes, k_scales, n_steps: Sequence[int],
+                           K: int, P: int, R: int):
+    """Per-step, per-layer selections of one query row over consecutive decode steps, with the
+    candidate pool kept across steps.
+
+    [A: 压缩吸收注意力（二代）]: the first layer's scan picks a candidate pool that the later layers
+    search.  The pages do not say how a pool is kept or refreshed as the context grows; the rule
+    here (this library's own, documented with the layer group) is:
+      * at steps s with s % R == 0 the Full layer's scan rebuilds the pool -- the top-min(P, n)
+        of its own order, as in layer_group_indices -- and records n_ref = n, the entry count;
+      * at the other steps the pool is kept, and the Reindex layers search the kept pool followed
+        by every entry written since the rebuild (ids n_ref .. n - 1);
+      * the Full layer's own top-K is always taken over the whole visible context.
+    R = 1 rebuilds the pool every step, which is layer_group_indices step by step.
+
+    step_inputs[s][l] = (q_codes, q_scales, w) or None (Reuse); n_steps[s] = visible entries at
+    step s (non-decreasing).  Returns [step][layer] -> (idx, cnt).
+    """
+    out = []
+    pool = pool_len = None
+    n_ref = 0
+    for s, n in enumerate(n_steps):
+        refresh = (s % R) == 0 or pool is None
+        res = []
+        cand = None
+        for l, m in enumerate(modes):
+            if m == FULL:
+                qc, qs, w = step_inputs[s][l]
+                idx, cnt, p, pl, _ = full_index(qc, qs, w, k_codes, k_scales, n, K, P if refresh else 0)
+                if refresh:
+                    pool, pool_len, n_ref = p, pl, int(n)
+                cand = pool[:pool_len] if refresh else extend_pool(pool, pool_len, n_ref, n)
+            elif m == REINDEX:
+                if cand is None:
+                    raise ValueError("Reindex layer before any Full layer")
+                qc, qs, w = step_inputs[s][l]
+                idx, cnt = reindex(qc, qs, w, k_codes, k_scales, cand, len(cand), K)
+            elif m == REUSE:
+                if not res:
+                    raise ValueError("Reuse layer before any Full layer")
+                idx, cnt = res[-1]
+            else:
+                raise ValueError(f"unknown mode {m!r}")
+            res.append((idx, cnt))
+        out.append(res)
+    return out
