@@ -18,7 +18,7 @@ __all__ = [
     "CSA2Error", "lib", "library_path",
     "csa2_quantize_kv", "csa2_quantize_kv_batch", "quant_job", "QuantJob", "csa2_compress_quantize_kv", "csa2_index_topk", "csa2_index_topk_workspace_size",
     "csa2_index_topk_scored", "csa2_topk_merge_shards", "csa2_topk_merge_shards_workspace_size",
-    "csa2_attn_merge_shards", "csa2_sparse_attn_shard",
+    "csa2_attn_merge_shards", "csa2_sparse_attn_shard", "csa2_pool_extend",
     "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_plan", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error", "csa2_selftest_bounded_wait",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
@@ -62,6 +62,10 @@ class QuantJob(ctypes.Structure):
     ]
 
 
+# the csa2_version() the descriptors and signatures below mirror
+ABI_VERSION = 4
+
+
 class GroupDesc(ctypes.Structure):
     """Mirror of ``csa2_group_desc``."""
     _fields_ = [
@@ -73,6 +77,7 @@ class GroupDesc(ctypes.Structure):
         ("q_pos", _vp),
         ("swa_cap", _i32), ("swa_start", _vp), ("swa_len", _vp),
         ("softmax_scale", _f32), ("out_dtype", _i32),
+        ("pool_keep", _vp), ("pool_keep_len", _vp), ("pool_keep_n", _vp), ("refresh", _i32), ("max_new", _i32),
     ]
 
 
@@ -102,6 +107,9 @@ def lib():
     L.csa2_status_string.argtypes = [_i32]
     L.csa2_version.restype = _i32
     L.csa2_version.argtypes = []
+    if L.csa2_version() != ABI_VERSION:
+        raise CSA2Error(f"{_LIB_PATH} has ABI version {L.csa2_version()}, this binding expects "
+                        f"{ABI_VERSION}; rebuild it with `python -m compressed_sparse_attention_quantize_b200.build`")
     L.csa2_quantize_kv.restype = _i32
     L.csa2_quantize_kv.argtypes = [_i32, _vp, _i32, _i64, _i32, _i64, _vp, _i64, _vp, _i64, _vp, _vp]
     L.csa2_quantize_kv_batch.restype = _i32
@@ -127,6 +135,8 @@ def lib():
     L.csa2_index_topk.argtypes = [_i32, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _vp, _i64,
                                   _vp, _vp, _i64, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _vp,
                                   _vp, _vp, _sz, _vp]
+    L.csa2_pool_extend.restype = _i32
+    L.csa2_pool_extend.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
     L.csa2_sparse_attn_plan.restype = _i32
     L.csa2_sparse_attn_plan.argtypes = [_i32, _i32, _i32, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
                                         ctypes.POINTER(_i32)]
@@ -275,6 +285,12 @@ def csa2_index_topk(mode, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_strid
                                  _ptr(pool_len), P_in, K, _ptr(out_idx), _ptr(out_cnt), P,
                                  _ptr(out_pool), _ptr(out_pool_len), _ptr(workspace), ws_bytes,
                                  _stream(stream)))
+
+
+def csa2_pool_extend(pool, pool_len, P_in, n_ref, n_entries, q_pos, B, T, P_out, out_pool, out_len,
+                     stream=None) -> None:
+    _check(lib().csa2_pool_extend(_ptr(pool), _ptr(pool_len), P_in, _ptr(n_ref), _ptr(n_entries), _ptr(q_pos),
+                                  B, T, P_out, _ptr(out_pool), _ptr(out_len), _stream(stream)))
 
 
 def csa2_sparse_attn_plan(rows, H, K):

@@ -23,6 +23,8 @@ cudaError_t launch_quant_fp4(const void *, int, int64_t, int, int64_t, uint8_t *
 cudaError_t launch_quant_fp8_token(const void *, int, int64_t, int, int64_t, uint8_t *, int64_t,
                                    uint8_t *, int64_t, const int64_t *, cudaStream_t);
 cudaError_t launch_quant_batch(const csa2_quant_job *, int, cudaStream_t);
+cudaError_t launch_pool_extend(const int32_t *, const int32_t *, int, const int32_t *, const int32_t *,
+                               const int32_t *, int, int, int, int32_t *, int32_t *, cudaStream_t);
 }  // namespace csa2
 
 #include "index_api.cuh"
@@ -134,7 +136,7 @@ const char *csa2_status_string(csa2_status s) {
     return "CSA2: unknown status";
 }
 
-int csa2_version(void) { return 3; }
+int csa2_version(void) { return 4; }
 
 const char *csa2_last_error_string(void) { return t_last_error; }
 
@@ -288,6 +290,17 @@ csa2_status csa2_topk_merge_shards(const float *scores, const int32_t *ids, cons
                                                 workspace, as_stream(stream)));
 }
 
+csa2_status csa2_pool_extend(const int32_t *pool, const int32_t *pool_len, int P_in, const int32_t *n_ref,
+                             const int32_t *n_entries, const int32_t *q_pos, int B, int T, int P_out,
+                             int32_t *out_pool, int32_t *out_len, void *stream) {
+    const Range range("csa2_pool_extend");
+    if (!pool || !pool_len || !n_ref || !n_entries || !out_pool || !out_len) return CSA2_ERR_INVALID_ARG;
+    if (B <= 0 || T <= 0 || (int64_t)B * T > (1 << 30) || P_in < 0 || P_out < 1 || P_out > CSA2_MAX_POOL)
+        return CSA2_ERR_SHAPE;
+    return cuda_status(launch_pool_extend(pool, pool_len, P_in, n_ref, n_entries, q_pos, B * T, T, P_out, out_pool,
+                                          out_len, as_stream(stream)));
+}
+
 csa2_status csa2_attn_merge_shards(const float *outs, const float *lses, int G, int rows, int H, int D,
                                    void *out, int out_dtype, float *lse, void *stream) {
     const Range range("csa2_attn_merge_shards");
@@ -385,15 +398,22 @@ static csa2_status group_layout(const csa2_group_desc *g, const csa2_layer_desc 
     }
     if (need_pool && g->P <= 0) return CSA2_ERR_INVALID_ARG;
     if (g->B <= 0 || g->T <= 0) return CSA2_ERR_SHAPE;
+    const bool keep = need_pool && g->pool_keep;
+    if (keep) {
+        if (!g->pool_keep_len || !g->pool_keep_n || g->q_pos) return CSA2_ERR_INVALID_ARG;
+        if (g->max_new < 0 || (int64_t)g->P + g->max_new > CSA2_MAX_POOL) return CSA2_ERR_SHAPE;
+    }
+    // candidates the Reindex layers search: the pool, or the kept pool and the entries since
+    const int p_search = keep ? g->P + g->max_new : g->P;
     const int rows = g->B * g->T;
     size_t off = 0;
     *idx_off = off; off += round_up((size_t)rows * g->K * 4 + (size_t)rows * 4);
     *pool_off = off;
-    if (need_pool) off += round_up((size_t)rows * g->P * 4 + (size_t)rows * 4);
+    if (need_pool) off += round_up((size_t)rows * p_search * 4 + (size_t)rows * 4);
     *idx_ws_off = off;
     size_t iw = index_ws(CSA2_MODE_FULL, rows, g->max_n, g->K, need_pool ? g->P : 0);
     if (need_pool) {
-        size_t iw2 = index_ws(CSA2_MODE_REINDEX, rows, g->max_n, g->K, g->P);
+        size_t iw2 = index_ws(CSA2_MODE_REINDEX, rows, g->max_n, g->K, p_search);
         if (iw2 > iw) iw = iw2;
     }
     *attn_off = off + iw;
@@ -446,6 +466,10 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     const int rows = g->B * g->T;
     bool need_pool = false;
     for (int l = 0; l < n_layers; ++l) need_pool |= layers[l].mode == CSA2_MODE_REINDEX;
+    // kept pool: rebuilt by the Full layer on refresh, else extended by the entries written since
+    const bool keep = need_pool && g->pool_keep;
+    const bool rebuild = need_pool && (!keep || g->refresh);
+    const int p_search = keep && !g->refresh ? g->P + g->max_new : g->P;
     // validate every layer before launching anything
     for (int l = 0; l < n_layers; ++l) {
         const csa2_layer_desc &L = layers[l];
@@ -455,8 +479,8 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
                                  g->seq_start, g->n_entries, g->max_n,
                                  L.mode == CSA2_MODE_REINDEX ? (const int32_t *)1 : nullptr,
                                  L.mode == CSA2_MODE_REINDEX ? (const int32_t *)1 : nullptr,
-                                 g->P, g->K, (int32_t *)1,
-                                 L.mode == CSA2_MODE_FULL && need_pool ? g->P : 0, (int32_t *)1);
+                                 p_search, g->K, (int32_t *)1,
+                                 L.mode == CSA2_MODE_FULL && rebuild ? g->P : 0, (int32_t *)1);
             if (s != CSA2_OK) return s;
         }
         s = check_attn_args(L.q, g->B, g->T, g->H, g->D, g->kv, g->kv_row_stride, g->seq_start,
@@ -468,7 +492,11 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     int32_t *idx = reinterpret_cast<int32_t *>(ws + idx_off);
     int32_t *cnt = idx + (size_t)rows * g->K;
     int32_t *pool = need_pool ? reinterpret_cast<int32_t *>(ws + pool_off) : nullptr;
-    int32_t *pool_len = need_pool ? pool + (size_t)rows * g->P : nullptr;
+    int32_t *pool_len = need_pool ? pool + (size_t)rows * p_search : nullptr;
+    if (keep && g->refresh) {
+        pool = g->pool_keep;
+        pool_len = g->pool_keep_len;
+    }
     void *iws = ws + iws_off;
     const size_t iws_bytes = attn_off - iws_off;
     void *aws = ws + attn_off;
@@ -477,6 +505,11 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
     GroupAux *aux = nullptr;
     {
         cudaError_t e = group_aux(&aux);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    if (keep && !g->refresh) {
+        cudaError_t e = launch_pool_extend(g->pool_keep, g->pool_keep_len, g->P, g->pool_keep_n,
+                                           g->n_entries, g->q_pos, rows, g->T, p_search, pool, pool_len, st);
         if (e != cudaSuccess) return cuda_status(e);
     }
     bool merge_pending[2] = {false, false};
@@ -491,13 +524,18 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
             s = csa2_index_topk(CSA2_MODE_FULL, L.iq_codes, L.iq_scales, L.iw, g->B, g->T, g->H_I,
                                 g->k_codes, g->k_code_stride, g->k_scales, g->k_scale_stride,
                                 g->seq_start, g->n_entries, g->max_n, g->q_pos, nullptr, nullptr, 0,
-                                g->K, idx, cnt, need_pool ? g->P : 0, pool, pool_len, iws,
-                                iws_bytes, stream);
+                                g->K, idx, cnt, rebuild ? g->P : 0, rebuild ? pool : nullptr,
+                                rebuild ? pool_len : nullptr, iws, iws_bytes, stream);
+            if (s == CSA2_OK && keep && g->refresh) {
+                cudaError_t e = cudaMemcpyAsync(g->pool_keep_n, g->n_entries, (size_t)g->B * 4,
+                                                cudaMemcpyDeviceToDevice, st);
+                if (e != cudaSuccess) return cuda_status(e);
+            }
         } else if (L.mode == CSA2_MODE_REINDEX) {
             s = csa2_index_topk(CSA2_MODE_REINDEX, L.iq_codes, L.iq_scales, L.iw, g->B, g->T,
                                 g->H_I, g->k_codes, g->k_code_stride, g->k_scales,
                                 g->k_scale_stride, g->seq_start, g->n_entries, g->max_n, g->q_pos,
-                                pool, pool_len, g->P, g->K, idx, cnt, 0, nullptr, nullptr, iws,
+                                pool, pool_len, p_search, g->K, idx, cnt, 0, nullptr, nullptr, iws,
                                 iws_bytes, stream);
         }
         if (s != CSA2_OK) return s;

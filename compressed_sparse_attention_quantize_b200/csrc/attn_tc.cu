@@ -171,35 +171,35 @@ CSA2_D void ldg_32B(const void *p, uint4 &lo, uint4 &hi) {
                  : "l"(p));
 }
 
-CSA2_D void prefetch_part(const KeySrc &src, int hsel, RowPart &rp) {
+// Half hb of prefetch: the code bytes of blocks mb = 2hb, 2hb + 1 (regions 2mb + hsel) and their
+// scale words.  The next tile's first half is requested before the softmax and its second half
+// after it, so that only one half's registers stay live across the softmax.
+CSA2_D void prefetch_half(const KeySrc &src, int hsel, int hb, RowPart &rp) {
     if (src.valid && !src.swa && (reinterpret_cast<uintptr_t>(src.ptr) & 31u) == 0) {
-        // aligned rows: one 256-bit load per region and one for the 32 scale bytes (5 requests
-        // instead of 10 -- the gather's request count throttled the load pipe)
+        // aligned rows: one 256-bit load per region (fewer requests: the gather's request count
+        // throttled the load pipe)
 #pragma unroll
-        for (int mb = 0; mb < kBlocks; ++mb) ldg_32B(src.ptr + 32 * (2 * mb + hsel), rp.codes[2 * mb], rp.codes[2 * mb + 1]);
-        uint4 s0, s1;
-        ldg_32B(src.ptr + 256, s0, s1);
-        rp.sc[0] = hsel ? s0.y : s0.x;
-        rp.sc[1] = hsel ? s0.w : s0.z;
-        rp.sc[2] = hsel ? s1.y : s1.x;
-        rp.sc[3] = hsel ? s1.w : s1.z;
+        for (int k = 0; k < 2; ++k) {
+            const int mb = 2 * hb + k;
+            ldg_32B(src.ptr + 32 * (2 * mb + hsel), rp.codes[2 * mb], rp.codes[2 * mb + 1]);
+        }
     } else if (src.valid && !src.swa) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
 #pragma unroll
-        for (int mb = 0; mb < kBlocks; ++mb) {
+        for (int k = 0; k < 2; ++k) {
+            const int mb = 2 * hb + k;
             rp.codes[2 * mb] = __ldg(p + 2 * (2 * mb + hsel));
             rp.codes[2 * mb + 1] = __ldg(p + 2 * (2 * mb + hsel) + 1);
         }
-        const uint4 s0 = __ldg(p + 16), s1 = __ldg(p + 17);     // scale bytes of regions 0-3, 4-7
-        rp.sc[0] = hsel ? s0.y : s0.x;
-        rp.sc[1] = hsel ? s0.w : s0.z;
-        rp.sc[2] = hsel ? s1.y : s1.x;
-        rp.sc[3] = hsel ? s1.w : s1.z;
+    }
+    if (src.valid && !src.swa) {
+        const uint4 s = __ldg(reinterpret_cast<const uint4 *>(src.ptr + 256) + hb);   // regions 4hb .. 4hb+3
+        rp.sc[2 * hb] = hsel ? s.y : s.x;
+        rp.sc[2 * hb + 1] = hsel ? s.w : s.z;
     } else {                                     // always assigned: no stale registers live
 #pragma unroll
-        for (int i = 0; i < 8; ++i) rp.codes[i] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) rp.sc[i] = 0u;
+        for (int i = 0; i < 4; ++i) rp.codes[4 * hb + i] = make_uint4(0u, 0u, 0u, 0u);
+        rp.sc[2 * hb] = rp.sc[2 * hb + 1] = 0u;
     }
 }
 
@@ -368,7 +368,8 @@ attn_tc_kernel(AttnArgs a) {
     RowPart rp;
     if (warp > 0) {
         src = source_of(a, r, b, seq_start, n_lim, entry_of(a, r, x_begin + t, x_end, n_sel));
-        prefetch_part(src, hsel, rp);
+        prefetch_half(src, hsel, 0, rp);
+        prefetch_half(src, hsel, 1, rp);
     }
 
     // ---------------- setup ----------------
@@ -503,32 +504,39 @@ attn_tc_kernel(AttnArgs a) {
             }
             const bool cur_valid = src.valid;
             const float cur_scale = src.scale;
-            // ---- the next tile's rows are requested now, while the tensor core is idle until P
-            //      is ready (issued during P.V they slowed its operand reads); the softmax below
-            //      works on 16 heads at a time so these registers stay live without spilling
+            // ---- the first half of the next tile's rows is requested now, while the tensor core
+            //      is idle until P is ready; the second half after the softmax, so that only one
+            //      half's registers are live across it
             src = source_of(a, r, b, seq_start, n_lim, e_next);
-            prefetch_part(src, hsel, rp);
+            prefetch_half(src, hsel, 0, rp);
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             if (!ptx::mbar_wait(&S.s_full, ph, abort_flag)) bad = true;
-            if (block_any(bad || *abort_flag != 0, 1, kWorkers)) { aborted = true; break; }
             ptx::tc_fence_after();
             const float zs = qk_scale * cur_scale;
             const uint32_t s_addr = lane_addr + half * 32;
             bool over = false;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t u[16];
-                ptx::tmem_ld16(s_addr + hh * 16, u);
+            {
+                uint32_t u[2][16];
+                ptx::tmem_ld16(s_addr, u[0]);
+                ptx::tmem_ld16(s_addr + 16, u[1]);
                 ptx::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float zi = cur_valid ? __uint_as_float(u[i]) * zs : -INFINITY;
-                    over |= zi > S.m_run[half * 32 + hh * 16 + i] + kRescaleThreshold;
-                }
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float zi = cur_valid ? __uint_as_float(u[hh][i]) * zs : -INFINITY;
+                        over |= zi > S.m_run[half * 32 + hh * 16 + i] + kRescaleThreshold;
+                    }
             }
             // the running max moves only when some logit exceeds it by more than 2^8.  The max
-            // scratch lives in P_lo, free here: s_full(j) completed after P.V(j-1).
-            const bool move = block_any(over, 1, kWorkers);
+            // scratch lives in P_lo, free here: s_full(j) completed after P.V(j-1).  One barrier
+            // decides both whether to stop (a failed wait anywhere) and whether the max moves;
+            // a second one separates the two only when either happened.
+            bool move = false;
+            if (block_any(over || bad || *abort_flag != 0, 1, kWorkers)) {
+                if (block_any(bad || *abort_flag != 0, 1, kWorkers)) { aborted = true; break; }
+                move = true;
+            }
             bool rescale = false;
             if (move) {
                 float v[32];
@@ -624,6 +632,7 @@ attn_tc_kernel(AttnArgs a) {
             ptx::fence_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&S.p_full);
+            prefetch_half(src, hsel, 1, rp);
         }
         // ---------------- epilogue ----------------
         if (!aborted && ntiles > 0 && !ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag)) bad = true;

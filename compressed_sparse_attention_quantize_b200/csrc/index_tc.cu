@@ -31,7 +31,8 @@ constexpr int kTile = 128;
 constexpr int kThreads = 128;
 constexpr int kMaxN = 4 * CSA2_MAX_INDEX_HEADS;      // 64 columns
 constexpr int kDepth = 2;                            // gathered tiles in flight per thread
-constexpr int kStages = 8;                           // contiguous tiles in flight per CTA
+constexpr int kStages = 4;                           // contiguous tiles in flight per CTA (a 16 KB
+                                                     // ring lets 8 CTAs share an SM)
 constexpr int kRingBytes = kStages * kTile * 32;     // raw key rows, 32 bytes each
 
 struct Args {
@@ -56,11 +57,11 @@ struct Args {
 };
 
 struct __align__(16) Smem {
-    uint8_t a[2][2 * kTile * 16];      // keys of tiles i (i % 2): two 16-byte planes each
+    uint8_t a[2 * kTile * 16];         // keys: two 16-byte planes
     uint8_t b[2 * kMaxN * 16];         // block-diagonal query
     float qs[CSA2_MAX_INDEX_HEADS * 4];// query block scales
     float w[CSA2_MAX_INDEX_HEADS];
-    uint64_t done[2], drain;           // MMA of tile i (accumulator i % 2) has completed
+    uint64_t done, drain;
     uint64_t full[kStages];            // ring stage s holds its tile's key rows
     uint32_t tmem_base;
     int abort_flag;
@@ -115,14 +116,13 @@ index_score_tc_kernel(Args a) {
     const int H = a.H;
     const int N = ((4 * H + 15) / 16) * 16;
     const uint32_t tmem_cols = a.tmem_cols;
-    const uint32_t sf_col = 2 * N;                     // after the two accumulators
+    const uint32_t sf_col = N;
 
     // ---- setup: query (block-diagonal B), scales, weights, barriers, TMEM ----
     for (int i = t; i < (int)(sizeof(S.b) / 16); i += kThreads)
         reinterpret_cast<uint4 *>(S.b)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (t == 0) {
-        ptx::mbar_init(&S.done[0], 1);
-        ptx::mbar_init(&S.done[1], 1);
+        ptx::mbar_init(&S.done, 1);
         ptx::mbar_init(&S.drain, 1);
         for (int i = 0; i < kStages; ++i) ptx::mbar_init(&S.full[i], 1);
         S.abort_flag = 0;
@@ -169,44 +169,41 @@ index_score_tc_kernel(Args a) {
     volatile int *abort_flag = &S.abort_flag;
     const int64_t sbase = a.seq_start[b];
 
-    const uint64_t adesc[2] = {sdesc_noswizzle(ptx::smem_u32(S.a[0]), kTile * 16, 128),
-                               sdesc_noswizzle(ptx::smem_u32(S.a[1]), kTile * 16, 128)};
+    const uint64_t adesc = sdesc_noswizzle(ptx::smem_u32(S.a), kTile * 16, 128);
 
-    // Tiles are software-pipelined: the MMA of tile i + 1 (accumulator (i + 1) % 2, key buffer
-    // (i + 1) % 2) runs while the epilogue reads tile i's accumulator.
-    // stage_issue: every thread writes its key row of tile i into the two planes of buffer i % 2,
-    // one barrier (which also tells every thread whether the CTA gave up), then thread 0 issues the
-    // MMA.  Buffer i % 2 and accumulator i % 2 were last used by tile i - 2, whose MMA completed
-    // and whose epilogue every thread finished before this barrier.
-    auto stage_issue = [&](int i, const uint4 &k0, const uint4 &k1) -> bool {
-        uint8_t *abuf = S.a[i & 1];
-        *reinterpret_cast<uint4 *>(abuf + t * 16) = k0;
-        *reinterpret_cast<uint4 *>(abuf + kTile * 16 + t * 16) = k1;
+    // One tile: stage this thread's key row in the two 16-byte planes, one MMA, then the
+    // fixed-order epilogue.  Returns false when the CTA gives up (collective).
+    // k0, k1: this thread's key row (planes 0 and 1), or with `chunked` the 16-byte chunks t and
+    // t + 128 of the tile's raw rows (chunk c is plane c % 2 of row c / 2), which keeps both the
+    // ring reads and the plane writes free of bank conflicts.
+    auto run_tile = [&](int i, const uint4 &k0, const uint4 &k1, bool chunked, uint32_t sc_this,
+                        bool valid_this) -> bool {
+        if (chunked) {
+            uint8_t *plane = S.a + (t & 1) * (kTile * 16);
+            *reinterpret_cast<uint4 *>(plane + (t >> 1) * 16) = k0;
+            *reinterpret_cast<uint4 *>(plane + (kTile / 2 + (t >> 1)) * 16) = k1;
+        } else {
+            *reinterpret_cast<uint4 *>(S.a + t * 16) = k0;
+            *reinterpret_cast<uint4 *>(S.a + kTile * 16 + t * 16) = k1;
+        }
         ptx::fence_async_smem();
         ptx::tc_fence_before();
-        if (__syncthreads_or(*abort_flag != 0)) return false;
+        __syncthreads();
         if (t == 0) {
             ptx::tc_fence_after();
-            mma_mxf4(tmem + (uint32_t)((i & 1) * N), adesc[i & 1], bdesc, idesc, sf, sf);
-            ptx::mma_commit(&S.done[i & 1]);
+            mma_mxf4(tmem, adesc, bdesc, idesc, sf, sf);
+            ptx::mma_commit(&S.done);
         }
-        return true;
-    };
-    // epilogue of tile i: wait for its MMA, then the fixed-order fp32 score of this thread's key.
-    // A wait that fails skips the TMEM read for the whole warp (the CTA then stops at the next
-    // barrier; the device error word already says why).
-    auto epilogue = [&](int i, uint32_t sc_this, bool valid_this) {
-        const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&S.done[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag));
-        if (!ok) return;
+        ptx::mbar_wait(&S.done, i & 1, abort_flag);
+        if (__syncthreads_or(*abort_flag != 0)) return false;
         ptx::tc_fence_after();
         float sk[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
-        const uint32_t dcol = lane_addr + (uint32_t)((i & 1) * N);
         float acc = 0.0f;
         for (int hb = 0; hb * 8 < H; ++hb) {
             uint32_t u[32];
-            ptx::tmem_ld32(dcol + hb * 32, u);
+            ptx::tmem_ld32(lane_addr + hb * 32, u);
             ptx::tmem_ld_wait();
 #pragma unroll
             for (int hh = 0; hh < 8; ++hh) {
@@ -224,6 +221,7 @@ index_score_tc_kernel(Args a) {
         }
         if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
         if (valid_this) a.scores[(int64_t)blockIdx.y * a.score_stride + j0 + (int64_t)i * kTile + t] = acc;
+        return true;
     };
 
     // the four E4M3 block scales of key j (0 past the end)
@@ -236,10 +234,8 @@ index_score_tc_kernel(Args a) {
         return (uint32_t)__ldg(ks) | ((uint32_t)__ldg(ks + 1) << 8) | ((uint32_t)__ldg(ks + 2) << 16) |
                ((uint32_t)__ldg(ks + 3) << 24);
     };
-    auto valid_of = [&](int i) -> bool { return j0 + (int64_t)i * kTile + t < n; };
 
     bool aborted = false;
-    int issued_mmas = 0;                 // tiles whose MMA thread 0 has issued
     const bool contiguous = a.pool == nullptr && a.k_code_stride == 32;
     if (contiguous) {
         // ---- Full mode: the CTA's keys are consecutive rows; thread 0 keeps kStages tiles of raw
@@ -255,46 +251,35 @@ index_score_tc_kernel(Args a) {
         int issued = 0;
         if (t == 0)
             for (; issued < kStages && issued < ntiles; ++issued) issue(issued);
-        // key row of tile i from its ring stage (after the stage's copy has landed)
-        auto row_of = [&](int i, uint4 &k0, uint4 &k1) {
+        uint32_t s0 = scale_of(0), s1 = scale_of(1), s2 = scale_of(2);
+        int i = 0;
+        for (; i < ntiles; ++i) {
             const int st = i % kStages;
             ptx::mbar_wait(&S.full[st], (uint32_t)(i / kStages) & 1u, abort_flag);   // a miss aborts below
-            k0 = k1 = make_uint4(0u, 0u, 0u, 0u);
-            if (valid_of(i)) {
-                const uint4 *row = reinterpret_cast<const uint4 *>(ring + st * kTile * 32 + t * 32);
-                k0 = row[0];
-                k1 = row[1];
-            }
-        };
-        uint32_t s0 = scale_of(0), s1 = scale_of(1), s2 = scale_of(2);
-        uint4 k0, k1;
-        row_of(0, k0, k1);
-        if (!stage_issue(0, k0, k1)) aborted = true;
-        else ++issued_mmas;
-        int i = 0;
-        for (; i < ntiles && !aborted; ++i) {
-            if (i + 1 < ntiles) {
-                row_of(i + 1, k0, k1);
-                if (!stage_issue(i + 1, k0, k1)) { aborted = true; break; }
-                ++issued_mmas;
-                // every thread has read the stage of tile i + 1: it may take tile i + 1 + kStages
-                if (t == 0 && issued < ntiles && issued <= i + 1 + kStages) issue(issued++);
-            }
-            epilogue(i, s0, valid_of(i));
+            const bool valid_this = j0 + (int64_t)i * kTile + t < n;
+            // rows past the end were not copied: their codes are stale but finite (E2M1 has no
+            // NaN), and their scores are never stored
+            const uint4 *stage = reinterpret_cast<const uint4 *>(ring + st * kTile * 32);
+            const uint4 k0 = stage[t], k1 = stage[t + kTile];
+            const uint32_t sc_this = s0;
             s0 = s1;
             s1 = s2;
             s2 = scale_of(i + 3);
+            if (!run_tile(i, k0, k1, true, sc_this, valid_this)) { aborted = true; break; }
+            // every thread has read stage st (run_tile synchronised after staging)
+            if (t == 0 && issued < ntiles) issue(issued++);
         }
         if (aborted && t == 0) {       // let the copies still in flight land before exiting
-            for (int k = i + 1; k < issued; ++k)
+            for (int k = i; k < issued; ++k)
                 ptx::mbar_wait_drain(&S.full[k % kStages], (uint32_t)(k / kStages) & 1u);
         }
     } else {
         // ---- gathered keys (Reindex pool) or strided rows: kDepth tiles in registers per thread
-        auto key_row = [&](int i, uint4 &c0, uint4 &c1) {
+        auto key_row = [&](int i, uint4 &c0, uint4 &c1, bool &valid) {
+            const int64_t j = j0 + (int64_t)i * kTile + t;
+            valid = j < n;
             c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
-            if (i < ntiles && valid_of(i)) {
-                const int64_t j = j0 + (int64_t)i * kTile + t;
+            if (valid) {
                 const int64_t e = sbase + (a.pool ? (int64_t)a.pool[(int64_t)r * a.P_in + j] : j);
                 const uint4 *kc = reinterpret_cast<const uint4 *>(a.k_codes + e * a.k_code_stride);
                 c0 = __ldg(kc);
@@ -303,33 +288,29 @@ index_score_tc_kernel(Args a) {
         };
         uint4 c0[kDepth], c1[kDepth];
         uint32_t sc[kDepth];
+        bool valid[kDepth];
 #pragma unroll
         for (int k = 0; k < kDepth; ++k) {
-            key_row(k + 1, c0[k], c1[k]);
+            key_row(k, c0[k], c1[k], valid[k]);
             sc[k] = scale_of(k);
         }
-        uint4 r0, r1;
-        key_row(0, r0, r1);
-        if (!stage_issue(0, r0, r1)) aborted = true;
-        else ++issued_mmas;
         for (int i0 = 0; i0 < ntiles && !aborted; i0 += kDepth) {
 #pragma unroll
             for (int k = 0; k < kDepth; ++k) {
                 const int i = i0 + k;
                 if (i >= ntiles) break;
-                // c0/c1[k] hold tile i + 1, sc[k] tile i's scales
-                if (i + 1 < ntiles) {
-                    if (!stage_issue(i + 1, c0[k], c1[k])) { aborted = true; break; }
-                    ++issued_mmas;
-                }
+                const uint4 k0 = c0[k], k1 = c1[k];
                 const uint32_t sc_this = sc[k];
-                key_row(i + 1 + kDepth, c0[k], c1[k]);
-                sc[k] = scale_of(i + kDepth);
-                epilogue(i, sc_this, valid_of(i));
+                const bool valid_this = valid[k];
+                if (i + kDepth < ntiles) {
+                    key_row(i + kDepth, c0[k], c1[k], valid[k]);
+                    sc[k] = scale_of(i + kDepth);
+                }
+                if (!run_tile(i, k0, k1, false, sc_this, valid_this)) { aborted = true; break; }
             }
         }
     }
-    if (t == 0 && issued_mmas > 0) {   // every issued MMA has completed before TMEM is released
+    if (aborted && t == 0) {           // drain the tensor pipe before TMEM is released
         ptx::mma_commit(&S.drain);
         ptx::mbar_wait_drain(&S.drain, 0);
     }
@@ -393,10 +374,10 @@ cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, flo
     a.row0 = row0;
     a.scores = scores;
     a.score_stride = score_stride;
-    // TMEM per CTA: two accumulators (2 x N columns) + 32 columns of unit scale factors
+    // TMEM per CTA: D (N columns) + 32 columns of unit scale factors
     const int N = ((4 * L.H + 15) / 16) * 16;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * N + 32)) cols <<= 1;
+    while (cols < (uint32_t)(N + 32)) cols <<= 1;
     a.tmem_cols = cols;
     // reserve shared memory so that at most 512/cols CTAs are resident on an SM
     // (and at least the bulk-copy ring of the contiguous path)

@@ -260,7 +260,10 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
             if (e != cudaSuccess) return e;
         }
         const int sel_P = reindex ? 0 : L.P;
-        if (topk_row_chunks(max_n, L.K, sel_P) > 0) {
+        // Few rows that the cluster kernel can hold: one cluster of CTAs per row keeps more SMs
+        // busy than one CTA per row (measured faster for 16 and 32 rows of 32K-64K scores).
+        const bool few_rows = max_n <= topk_cluster_max_n() && nr <= 64;
+        if (!few_rows && topk_row_chunks(max_n, L.K, sel_P) > 0) {
             void *scratch = reinterpret_cast<uint8_t *>(L.workspace) + score_bytes(chunk, max_n);
             cudaError_t e = launch_topk_row(scores, sa.score_stride, sa.pool, sa.P_in, sa.n_entries, sa.q_pos,
                                             sa.pool_len, sa.T, sa.row0, nr, L.K, L.out_idx, L.out_cnt, sel_P,
@@ -298,6 +301,44 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------------------
+// pool kept across decode steps: the kept pool followed by the entries written since
+// ---------------------------------------------------------------------------------------
+__global__ void pool_extend_kernel(const int32_t *__restrict__ pool, const int32_t *__restrict__ pool_len,
+                                   int P_in, const int32_t *__restrict__ n_ref,
+                                   const int32_t *__restrict__ n_entries, const int32_t *__restrict__ q_pos,
+                                   int T, int P_out, int32_t *__restrict__ out_pool, int32_t *__restrict__ out_len) {
+    const int r = blockIdx.x;
+    const int b = r / T;
+    const int kept = max(0, min(pool_len[r], P_in));
+    int64_t n = n_entries[b];
+    if (q_pos) {
+        const int64_t v = ((int64_t)q_pos[r] + 1) / 4;
+        n = v < n ? v : n;
+    }
+    const int64_t lo = max(0, n_ref[b]);
+    const int64_t fresh = n > lo ? n - lo : 0;
+    int64_t total = kept + fresh;
+    if (total > P_out) {
+        if (threadIdx.x == 0) raise_device_error(CSA2_ERR_SHAPE);
+        total = P_out;
+    }
+    const int32_t *src = pool + (int64_t)r * P_in;
+    int32_t *dst = out_pool + (int64_t)r * P_out;
+    for (int64_t i = threadIdx.x; i < total; i += blockDim.x)
+        dst[i] = i < kept ? src[i] : (int32_t)(lo + (i - kept));
+    if (threadIdx.x == 0) out_len[r] = (int32_t)total;
+}
+
+cudaError_t launch_pool_extend(const int32_t *pool, const int32_t *pool_len, int P_in, const int32_t *n_ref,
+                               const int32_t *n_entries, const int32_t *q_pos, int rows, int T, int P_out,
+                               int32_t *out_pool, int32_t *out_len, cudaStream_t st) {
+    pool_extend_kernel<<<rows, 256, 0, st>>>(pool, pool_len, P_in, n_ref, n_entries, q_pos, T, P_out, out_pool,
+                                             out_len);
+    note_launches(1);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------------------

@@ -190,6 +190,21 @@ class GroupRunner:
         g.softmax_scale, g.out_dtype = self.softmax_scale, self.out_dtype
         return g
 
+    def keep_pool(self, max_new: int) -> None:
+        """Keep the Reindex layers' candidate pool across decode calls (csa2_group_desc's
+        pool_keep): ``run(refresh=True)`` rebuilds it, ``run(refresh=False)`` searches it followed
+        by the at most ``max_new`` entries per sequence written since.  The first call after
+        this one must refresh."""
+        d, wl = self.dev, self.wl
+        self.pool_keep = torch.full((self.rows, max(wl.P, 1)), -1, dtype=torch.int32, device=d)
+        self.pool_keep_len = torch.zeros((self.rows,), dtype=torch.int32, device=d)
+        self.pool_keep_n = torch.zeros((wl.B,), dtype=torch.int32, device=d)
+        g = self.g
+        g.pool_keep, g.pool_keep_len = self.pool_keep.data_ptr(), self.pool_keep_len.data_ptr()
+        g.pool_keep_n, g.max_new, g.refresh = self.pool_keep_n.data_ptr(), int(max_new), 1
+        self.ws_bytes = csa2_layer_group_workspace_size(self.g, self.layer_descs)
+        self.workspace = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=d)
+
     def _layer_desc(self, l: int) -> LayerDesc:
         ld = self.layer_data[l]
         L = LayerDesc()
@@ -208,7 +223,10 @@ class GroupRunner:
             L.ready_event = ready[l] if ready else None
             L.done_event = done[l] if done else None
 
-    def run(self, stream=None) -> None:
+    def run(self, stream=None, refresh: Optional[bool] = None) -> None:
+        """The layer group; ``refresh`` sets whether a kept pool (keep_pool) is rebuilt."""
+        if refresh is not None:
+            self.g.refresh = 1 if refresh else 0
         csa2_layer_group(self.g, self.layer_descs, self.workspace, self.ws_bytes, stream)
 
     def write_step(self, stream=None) -> None:

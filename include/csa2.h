@@ -216,6 +216,25 @@ CSA2_API csa2_status csa2_index_topk(int mode, const uint8_t *q_codes, const uin
                             void *workspace, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa2_pool_extend -- Reindex candidates between pool refreshes ([A] section
+ * "压缩吸收注意力（二代）": later layers search the first layer's candidate pool; this call keeps
+ * such a pool useful as entries are written after it was built).  For query row r (b = r / T):
+ *     out_pool[r] = pool[r][0 .. pool_len[r]) followed by ids n_ref[b] .. n_vis(r) - 1
+ * with n_vis(r) as in csa2_index_topk (n_entries[b], or min(n_entries[b], (q_pos[r] + 1) / 4)
+ * when q_pos is given); out_len[r] = the count.  The kept pool's ids lie below n_ref[b], so the
+ * list stays ascending.  Rows with more than P_out candidates keep the first P_out and the
+ * device error word becomes CSA2_ERR_SHAPE (csa2_device_error).
+ *   pool int32 [B*T][P_in], pool_len / out_len int32 [B*T], n_ref / n_entries int32 [B],
+ *   q_pos int32 [B*T] or NULL, out_pool int32 [B*T][P_out] (may not overlap pool).
+ * Errors: INVALID_ARG (NULL pool, pool_len, n_ref, n_entries, out_pool or out_len), SHAPE
+ *   (B or T <= 0, P_in < 0, P_out < 1 or P_out > CSA2_MAX_POOL), CUDA.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_pool_extend(const int32_t *pool, const int32_t *pool_len, int P_in,
+                                      const int32_t *n_ref, const int32_t *n_entries,
+                                      const int32_t *q_pos, int B, int T, int P_out,
+                                      int32_t *out_pool, int32_t *out_len, void *stream);
+
+/* ------------------------------------------------------------------------------------
  * csa2_sparse_attn -- attention of each query row over its selected compressed entries
  * merged with its own 8-bit sliding window.
  *
@@ -333,6 +352,23 @@ typedef struct csa2_group_desc {
     const int32_t *q_pos;        /* NULL = decode (all entries visible)                */
     int swa_cap;                 const int32_t *swa_start;  const int32_t *swa_len;
     float softmax_scale;         int out_dtype;
+    /* Candidate pool kept across decode steps (optional; pool_keep == NULL rebuilds it in every
+     * call).  [A] section "压缩吸收注意力（二代）" has the first layer's scan build a pool that the
+     * later layers search; how a pool is kept as the context grows is this library's own rule:
+     *   refresh != 0: the Full layer rebuilds the pool -- top-min(P, n) of its order -- into
+     *                 pool_keep [B*T][P] / pool_keep_len [B*T] and records pool_keep_n[b] =
+     *                 n_entries[b] (the entry count at the rebuild);
+     *   refresh == 0: the pool is kept, and the Reindex layers search it followed by the entries
+     *                 written since (ids pool_keep_n[b] .. n - 1, see csa2_pool_extend), at most
+     *                 max_new per sequence (P + max_new <= CSA2_MAX_POOL).
+     * The caller owns the three arrays and calls with refresh != 0 first and every R steps.  The
+     * Full layer's own top-K is always taken over every visible entry.  Ignored without REINDEX
+     * layers.  Decode only: INVALID_ARG with q_pos != NULL or a NULL pool_keep_len /
+     * pool_keep_n; SHAPE when max_new < 0 or P + max_new > CSA2_MAX_POOL; a step that has
+     * written more than max_new entries since the refresh sets CSA2_ERR_SHAPE in the device
+     * error word and searches the first P + max_new candidates. */
+    int32_t *pool_keep;          int32_t *pool_keep_len;    int32_t *pool_keep_n;
+    int refresh;                 int max_new;
 } csa2_group_desc;
 
 typedef struct csa2_layer_desc {

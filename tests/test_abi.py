@@ -150,6 +150,41 @@ def test_layer_group_mode_table_validation(L):
     assert L.csa2_layer_group(ctypes.byref(g), arr, 2, 16, 8, None) == WS
 
 
+def test_layer_group_kept_pool_validation(L):
+    F, I, U = csa2.MODE_FULL, csa2.MODE_REINDEX, csa2.MODE_REUSE
+    g, layers = _group([F, I, U], P=300)
+    base = csa2.csa2_layer_group_workspace_size(g, layers)
+    g.pool_keep, g.pool_keep_len, g.pool_keep_n, g.max_new = 16, 16, 16, 64
+    # the Reindex candidates grow by max_new, and so does the workspace
+    assert csa2.csa2_layer_group_workspace_size(g, layers) > base
+    g.max_new = -1
+    with pytest.raises(csa2.CSA2Error, match="SHAPE"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    g.max_new = 32768 - 300 + 1
+    with pytest.raises(csa2.CSA2Error, match="SHAPE"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    g.max_new = 64
+    g.pool_keep_n = None
+    with pytest.raises(csa2.CSA2Error, match="INVALID_ARG"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    g.pool_keep_n, g.q_pos = 16, 16                 # decode only
+    with pytest.raises(csa2.CSA2Error, match="INVALID_ARG"):
+        csa2.csa2_layer_group_workspace_size(g, layers)
+    # without Reindex layers the kept-pool fields are ignored
+    g, layers = _group([F, U])
+    g.pool_keep, g.max_new = 16, -5
+    assert csa2.csa2_layer_group_workspace_size(g, layers) > 0
+
+
+def test_pool_extend_validation(L):
+    pe = L.csa2_pool_extend
+    assert pe(None, 16, 10, 16, 16, None, 2, 1, 20, 16, 16, None) == INVALID
+    assert pe(16, 16, 10, 16, 16, None, 0, 1, 20, 16, 16, None) == SHAPE
+    assert pe(16, 16, -1, 16, 16, None, 2, 1, 20, 16, 16, None) == SHAPE
+    assert pe(16, 16, 10, 16, 16, None, 2, 1, 0, 16, 16, None) == SHAPE
+    assert pe(16, 16, 10, 16, 16, None, 2, 1, 32769, 16, 16, None) == SHAPE
+
+
 def test_attention_plan_invariants():
     """The split plan covers the K + window keys with no empty split, in whole 128-key tiles,
     and the workspace query holds exactly one partial per (row, head group, split)."""

@@ -220,6 +220,87 @@ def test_reindex_group_scaled():
     _check_rows(r, wl, range(3))
 
 
+@pytest.mark.parametrize("R", [1, 3])
+def test_pool_kept_across_decode_steps(R):
+    """Kept candidate pool over consecutive decode steps: the context grows by a few entries per
+    step (sequence 1 not at all), the pool is rebuilt every R steps and the Reindex layers
+    search it plus the entries written since; every layer's selection at every step equals the
+    oracle's decode_steps_with_pool."""
+    n = [3000, 5000, 700]
+    growth = [37, 0, 5]
+    steps = 7
+    wl = synth.scaled(synth.workload(2), B=3, n=n, K=128, P=600, name="pool_kept")
+    r = runtime.GroupRunner(wl, layers=4)
+    r.keep_pool(max_new=max(growth) * steps)
+    n_steps = [[n[b] - (steps - 1 - s) * growth[b] for s in range(steps)] for b in range(3)]
+    got = []
+    for s in range(steps):
+        r.n_entries.copy_(torch.tensor([n_steps[b][s] for b in range(3)], dtype=torch.int32))
+        r.run(refresh=(s % R == 0))
+        torch.cuda.synchronize()
+        got.append([r.layer_data[l]["idx"].cpu().numpy().copy() for l in range(4)])
+    assert csa2.csa2_device_error() == 0
+    for b in range(3):
+        os_ = OracleSeq(wl, b)
+        inputs = [None if m == "U" else (os_.layer(l)["qc"][0], os_.layer(l)["qs"][0], os_.layer(l)["w"][0])
+                  for l, m in enumerate(r.modes)]
+        ref = oracle.decode_steps_with_pool(r.modes, [inputs] * steps, os_.k_codes, os_.k_scales,
+                                            n_steps[b], wl.K, wl.P, R)
+        for s in range(steps):
+            for l in range(4):
+                assert np.array_equal(got[s][l][b], ref[s][l][0]), f"step {s} layer {l} seq {b}"
+    # attention of the last step reads the last step's selections
+    os_ = OracleSeq(wl, 0)
+    out, _ = os_.attention(1, 0, got[-1][1][0], r.softmax_scale)
+    check_attention(r.layer_data[1]["out"][0].cpu().numpy(), out, "layer 1 seq 0")
+
+
+def test_pool_extend_matches_oracle():
+    rng = np.random.default_rng(11)
+    B, T, P_in, P_out = 5, 3, 40, 70
+    rows = B * T
+    n_ref = np.array([0, 100, 500, 64, 9], np.int32)
+    n_ent = n_ref + np.array([0, 29, 30, 3, 0], np.int32)
+    pool = np.full((rows, P_in), -1, np.int32)
+    plen = np.zeros(rows, np.int32)
+    for r in range(rows):
+        b = r // T
+        k = int(rng.integers(0, min(P_in, n_ref[b]) + 1))
+        pool[r, :k] = np.sort(rng.choice(max(n_ref[b], 1), size=k, replace=False)) if k else []
+        plen[r] = k
+    dev = torch.device("cuda")
+    out = torch.full((rows, P_out), -7, dtype=torch.int32, device=dev)
+    olen = torch.zeros(rows, dtype=torch.int32, device=dev)
+    tp = [torch.from_numpy(x).to(dev) for x in (pool, plen, n_ref, n_ent)]
+    csa2.csa2_pool_extend(tp[0], tp[1], P_in, tp[2], tp[3], None, B, T, P_out, out, olen)
+    torch.cuda.synchronize()
+    assert csa2.csa2_device_error() == 0
+    out, olen = out.cpu().numpy(), olen.cpu().numpy()
+    for r in range(rows):
+        b = r // T
+        ref = oracle.extend_pool(pool[r], plen[r], n_ref[b], n_ent[b])
+        assert olen[r] == len(ref)
+        assert np.array_equal(out[r, :len(ref)], ref)
+        assert np.all(out[r, len(ref):] == -7)          # nothing written past the count
+
+
+def test_pool_kept_overflow_flags_shape():
+    """More new entries than max_new since the refresh: the device error word reads
+    CSA2_ERR_SHAPE and the call still completes."""
+    wl = synth.scaled(synth.workload(2), B=1, n=[2000], K=64, P=300, name="pool_overflow")
+    r = runtime.GroupRunner(wl, layers=2)
+    r.keep_pool(max_new=8)
+    r.n_entries.fill_(1900)
+    r.run(refresh=True)
+    torch.cuda.synchronize()
+    assert csa2.csa2_device_error() == 0
+    r.n_entries.fill_(2000)
+    r.run(refresh=False)
+    torch.cuda.synchronize()
+    assert csa2.csa2_device_error() == csa2.CSA2_ERR_SHAPE
+    assert csa2.csa2_device_error() == 0
+
+
 def test_long_rows_scaled():
     wl = synth.scaled(synth.workload(3), B=2, n=[70000, 41000], K=512, name="long_scaled")
     r = _run_group(wl, layers=2)
