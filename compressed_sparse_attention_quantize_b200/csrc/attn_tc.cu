@@ -171,35 +171,24 @@ CSA2_D void ldg_32B(const void *p, uint4 &lo, uint4 &hi) {
                  : "l"(p));
 }
 
-// Half hb of prefetch: the code bytes of blocks mb = 2hb, 2hb + 1 (regions 2mb + hsel) and their
-// scale words.  The next tile's first half is requested before the softmax and its second half
-// after it, so that only one half's registers stay live across the softmax.
-CSA2_D void prefetch_half(const KeySrc &src, int hsel, int hb, RowPart &rp) {
-    if (src.valid && !src.swa && (reinterpret_cast<uintptr_t>(src.ptr) & 31u) == 0) {
-        // aligned rows: one 256-bit load per region (fewer requests: the gather's request count
-        // throttled the load pipe)
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int mb = 2 * hb + k;
-            ldg_32B(src.ptr + 32 * (2 * mb + hsel), rp.codes[2 * mb], rp.codes[2 * mb + 1]);
-        }
-    } else if (src.valid && !src.swa) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(src.ptr);
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int mb = 2 * hb + k;
-            rp.codes[2 * mb] = __ldg(p + 2 * (2 * mb + hsel));
-            rp.codes[2 * mb + 1] = __ldg(p + 2 * (2 * mb + hsel) + 1);
-        }
-    }
+// Block mb of prefetch: the 32 code bytes of region 2mb + hsel and its scale word.  A tile's
+// rows are requested one block at a time, each right after the previous tile's block has been
+// dequantised, so that at most a few KB of gathers are in flight per block: a load queue full of
+// gathers holds up every shared-memory access of the SM behind it (measured: the MMA issuer's
+// barrier polls and the softmax's P stores waited for the gathers).
+CSA2_D void prefetch_block(const KeySrc &src, int hsel, int mb, RowPart &rp) {
     if (src.valid && !src.swa) {
-        const uint4 s = __ldg(reinterpret_cast<const uint4 *>(src.ptr + 256) + hb);   // regions 4hb .. 4hb+3
-        rp.sc[2 * hb] = hsel ? s.y : s.x;
-        rp.sc[2 * hb + 1] = hsel ? s.w : s.z;
+        const uint8_t *p = src.ptr + 32 * (2 * mb + hsel);
+        if ((reinterpret_cast<uintptr_t>(p) & 31u) == 0) {
+            ldg_32B(p, rp.codes[2 * mb], rp.codes[2 * mb + 1]);
+        } else {
+            rp.codes[2 * mb] = __ldg(reinterpret_cast<const uint4 *>(p));
+            rp.codes[2 * mb + 1] = __ldg(reinterpret_cast<const uint4 *>(p) + 1);
+        }
+        rp.sc[mb] = __ldg(reinterpret_cast<const uint32_t *>(src.ptr + 256) + 2 * mb + hsel);
     } else {                                     // always assigned: no stale registers live
-#pragma unroll
-        for (int i = 0; i < 4; ++i) rp.codes[4 * hb + i] = make_uint4(0u, 0u, 0u, 0u);
-        rp.sc[2 * hb] = rp.sc[2 * hb + 1] = 0u;
+        rp.codes[2 * mb] = rp.codes[2 * mb + 1] = make_uint4(0u, 0u, 0u, 0u);
+        rp.sc[mb] = 0u;
     }
 }
 
@@ -368,8 +357,8 @@ attn_tc_kernel(AttnArgs a) {
     RowPart rp;
     if (warp > 0) {
         src = source_of(a, r, b, seq_start, n_lim, entry_of(a, r, x_begin + t, x_end, n_sel));
-        prefetch_half(src, hsel, 0, rp);
-        prefetch_half(src, hsel, 1, rp);
+#pragma unroll
+        for (int mb = 0; mb < kBlocks; ++mb) prefetch_block(src, hsel, mb, rp);
     }
 
     // ---------------- setup ----------------
@@ -482,10 +471,12 @@ attn_tc_kernel(AttnArgs a) {
             ptx::tmem_st32(l_addr, zero);
             ptx::tmem_st_wait();
         }
+        // the entry number of the next tile is read one tile ahead of its use
+        int32_t e_next = ntiles > 1 ? entry_of(a, r, x_begin + kTile + t, x_end, n_sel) : kNoKey;
         for (int j = 0; j < ntiles; ++j) {
             const uint32_t ph = j & 1;
-            // the next tile's entry number is read now and used after the dequantisation
-            const int32_t e_next = (j + 1 < ntiles) ? entry_of(a, r, x_begin + (j + 1) * kTile + t, x_end, n_sel) : kNoKey;
+            const KeySrc src_next = source_of(a, r, b, seq_start, n_lim, e_next);
+            e_next = (j + 2 < ntiles) ? entry_of(a, r, x_begin + (j + 2) * kTile + t, x_end, n_sel) : kNoKey;
             // ---- dequantise regions 2mb + hsel of key t; block mb is free once P.V(j-1) has
             //      finished with it
 #pragma unroll
@@ -501,14 +492,12 @@ attn_tc_kernel(AttnArgs a) {
                 for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + sw128_off(t, c)) = out[c];
                 ptx::fence_async_smem();
                 ptx::mbar_arrive(&S.v_full[mb]);
+                // block mb of the next tile into the registers just consumed
+                if (j + 1 < ntiles) prefetch_block(src_next, hsel, mb, rp);
             }
             const bool cur_valid = src.valid;
             const float cur_scale = src.scale;
-            // ---- the first half of the next tile's rows is requested now, while the tensor core
-            //      is idle until P is ready; the second half after the softmax, so that only one
-            //      half's registers are live across it
-            src = source_of(a, r, b, seq_start, n_lim, e_next);
-            prefetch_half(src, hsel, 0, rp);
+            src = src_next;
             // ---- softmax over this thread's key for heads 32*half .. 32*half+31
             if (!ptx::mbar_wait(&S.s_full, ph, abort_flag)) bad = true;
             ptx::tc_fence_after();
@@ -632,7 +621,6 @@ attn_tc_kernel(AttnArgs a) {
             ptx::fence_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&S.p_full);
-            prefetch_half(src, hsel, 1, rp);
         }
         // ---------------- epilogue ----------------
         if (!aborted && ntiles > 0 && !ptx::mbar_wait(&S.pv_done, (ntiles - 1) & 1, abort_flag)) bad = true;

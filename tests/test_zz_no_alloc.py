@@ -21,11 +21,21 @@ from tests._parity import check_attention
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,K", [(4, 256), (32, 2048)])
+def _rows_beyond_array():
+    for rows in range(1, 161):
+        if csa2.csa2_sparse_attn_workspace_size(rows, 64, 2048) > (20 << 20):
+            return rows
+    raise AssertionError("no decode batch up to 160 rows exceeds the no-allocation array")
+
+
+@pytest.mark.parametrize("B,K", [(4, 256), (32, 2048), ("beyond", 2048)])
 def test_noalloc_matches_workspace_entry_point_twice(B, K):
-    # 4 rows x 64 heads and top-256 + a 128-token window: 3 key splits per row, so the split
-    # partials (the scratch) are really used.  32 rows x top-2048 is the 128K decode shape, whose
-    # default plan needs more partials than the array holds: the call runs a plan fitted to it.
+    # 4 rows x 64 heads and top-256 + a 128-token window: several splits per row, so the split
+    # partials (the scratch) are really used.  32 rows x top-2048 is the 128K decode shape; the
+    # third case takes the fewest rows whose default plan needs more partials than the array
+    # holds: the call runs a plan fitted to it.
+    if B == "beyond":
+        B = _rows_beyond_array()
     wl = synth.scaled(synth.workload(1), B=B, n=3000, K=K, name="noalloc")
     r = runtime.GroupRunner(wl, layers=2)
     r.run()
