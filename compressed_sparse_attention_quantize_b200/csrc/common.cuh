@@ -123,6 +123,19 @@ inline int current_device() {
     return dev;
 }
 
+// Makes the current device's primary context current for driver-API calls of this thread (the
+// runtime binds it lazily, and a thread whose first call encodes a tensor map has none bound
+// yet: the encode then fails).  Once per thread and device.
+inline cudaError_t bind_current_context() {
+    thread_local int bound = -1;
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (dev == bound) return cudaSuccess;
+    const cudaError_t e = cudaSetDevice(dev);
+    if (e == cudaSuccess) bound = dev;
+    return e;
+}
+
 // SM count of the current device; 148 (a B200) when no device can be queried, so that plans
 // can still be inspected on a host without a GPU.
 inline int device_sm_count() {

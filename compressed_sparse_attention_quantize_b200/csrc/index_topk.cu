@@ -224,6 +224,9 @@ size_t index_topk_workspace_bytes(int rows, int64_t n, int K, int P) {
 
 cudaError_t launch_index_score_tc(const IndexLaunch &L, int row0, int nrows, float *scores,
                                   int64_t score_stride, cudaStream_t st);
+bool index_pipe_applies(const IndexLaunch &L);
+cudaError_t launch_index_score_pipe(const IndexLaunch &L, int row0, int nrows, int R, float *scores,
+                                    int64_t score_stride, cudaStream_t st);
 
 int64_t topk_cluster_max_n();
 cudaError_t launch_gather_scores(const float *scores, int64_t score_stride, const int32_t *idx, int K,
@@ -248,6 +251,8 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
     const int rows = L.B * L.T;
     const int64_t max_n = reindex ? (int64_t)L.P_in : L.max_n;
     const int64_t chunk = index_rows_per_chunk(rows, max_n);
+    // contiguous key ranges (Full mode) go to the pipelined score kernel
+    const bool pipe = index_pipe_applies(L);
     float *scores = reinterpret_cast<float *>(L.workspace);
     for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
         const int nr = (int)((rows - r0) < chunk ? (rows - r0) : chunk);
@@ -256,7 +261,8 @@ cudaError_t launch_index_topk(const IndexLaunch &L, cudaStream_t st) {
         sa.scores = scores;
         sa.score_stride = max_n > 0 ? max_n : 1;
         if (max_n > 0) {
-            cudaError_t e = launch_index_score_tc(L, (int)r0, nr, scores, sa.score_stride, st);
+            cudaError_t e = pipe ? launch_index_score_pipe(L, (int)r0, nr, 1, scores, sa.score_stride, st)
+                                 : launch_index_score_tc(L, (int)r0, nr, scores, sa.score_stride, st);
             if (e != cudaSuccess) return e;
         }
         const int sel_P = reindex ? 0 : L.P;

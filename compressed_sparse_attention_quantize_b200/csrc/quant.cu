@@ -120,6 +120,50 @@ CSA2_D uint32_t e4m3_code_of_quotient(float a, float s) {
     return c;
 }
 
+// One token row by one warp: the scale s = amax / 448 and every code.  Rows of up to 512
+// channels are read once, all loads issued before the first is used (a loop that waits for each
+// load in turn made a step's small window write latency-bound); longer rows take two passes.
+template <typename Load>
+CSA2_D void fp8_token_row(int lane, int dim, Load load, uint8_t *cd, float *scale) {
+    constexpr int kPer = 16;
+    if (dim <= 32 * kPer) {
+        float v[kPer];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = lane + 32 * k;
+            v[k] = i < dim ? load(i) : 0.0f;
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) amax = fmaxf(amax, fabsf(v[k]));
+        // non-negative floats order like their bit patterns
+        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+        const float s = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = lane + 32 * k;
+            if (i < dim) {
+                uint32_t c = 0u;
+                if (s != 0.0f) c = e4m3_code_of_quotient(fabsf(v[k]), s) | (signbit(v[k]) ? 0x80u : 0u);
+                cd[i] = (uint8_t)c;
+            }
+        }
+        if (lane == 0) *scale = s;
+        return;
+    }
+    float amax = 0.0f;
+    for (int i = lane; i < dim; i += 32) amax = fmaxf(amax, fabsf(load(i)));
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    const float s = __fdiv_rn(amax, 448.0f);
+    for (int i = lane; i < dim; i += 32) {
+        const float v = load(i);
+        uint32_t c = 0u;
+        if (s != 0.0f) c = e4m3_code_of_quotient(fabsf(v), s) | (signbit(v) ? 0x80u : 0u);
+        cd[i] = (uint8_t)c;
+    }
+    if (lane == 0) *scale = s;
+}
+
 // One warp per row.
 template <typename T>
 __global__ void quant_fp8_token_kernel(const T *__restrict__ x, int64_t rows, int dim,
@@ -131,20 +175,9 @@ __global__ void quant_fp8_token_kernel(const T *__restrict__ x, int64_t rows, in
     for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
          r += warps) {
         const T *xr = x + r * x_stride;
-        float amax = 0.0f;
-        for (int i = lane; i < dim; i += 32) amax = fmaxf(amax, fabsf(load_as_f32<T>(xr + i)));
-        // non-negative floats order like their bit patterns
-        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
-        const float s = __fdiv_rn(amax, 448.0f);
         const int64_t d = dst_rows ? dst_rows[r] : r;
-        uint8_t *cd = codes + d * code_stride;
-        for (int i = lane; i < dim; i += 32) {
-            const float v = load_as_f32<T>(xr + i);
-            uint32_t c = 0u;
-            if (s != 0.0f) c = e4m3_code_of_quotient(fabsf(v), s) | (signbit(v) ? 0x80u : 0u);
-            cd[i] = (uint8_t)c;
-        }
-        if (lane == 0) *reinterpret_cast<float *>(scales + d * scale_stride) = s;
+        fp8_token_row(lane, dim, [&](int i) { return load_as_f32<T>(xr + i); }, codes + d * code_stride,
+                      reinterpret_cast<float *>(scales + d * scale_stride));
     }
 }
 
@@ -202,19 +235,9 @@ __global__ void __launch_bounds__(kQuantThreads) quant_batch_kernel(const __grid
         const int64_t r = lb * (kQuantThreads / 32) + (threadIdx.x >> 5);
         if (r >= q.rows) return;                                   // uniform per warp
         const int64_t base = r * q.x_stride;
-        float amax = 0.0f;
-        for (int i = lane; i < q.dim; i += 32) amax = fmaxf(amax, fabsf(load_elem(q.x, q.x_dtype, base + i)));
-        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
-        const float sc = __fdiv_rn(amax, 448.0f);
         const int64_t d = q.dst_rows ? q.dst_rows[r] : r;
-        uint8_t *cd = q.codes + d * q.code_stride;
-        for (int i = lane; i < q.dim; i += 32) {
-            const float v = load_elem(q.x, q.x_dtype, base + i);
-            uint32_t c = 0u;
-            if (sc != 0.0f) c = e4m3_code_of_quotient(fabsf(v), sc) | (signbit(v) ? 0x80u : 0u);
-            cd[i] = (uint8_t)c;
-        }
-        if (lane == 0) *reinterpret_cast<float *>(q.scales + d * q.scale_stride) = sc;
+        fp8_token_row(lane, q.dim, [&](int i) { return load_elem(q.x, q.x_dtype, base + i); },
+                      q.codes + d * q.code_stride, reinterpret_cast<float *>(q.scales + d * q.scale_stride));
     }
 }
 

@@ -3,6 +3,8 @@
 // descriptors.  Field layouts follow the PTX ISA descriptions of the tcgen05 instruction and
 // shared-memory descriptors (also mirrored by CUTLASS's cute/arch/mma_sm100_desc.hpp).
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace csa2 {
@@ -79,6 +81,16 @@ CSA2_D void bulk_store_s2g(void *dst, const void *src, uint32_t bytes) {
 CSA2_D void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk group of this thread has completed (its writes are done).
 CSA2_D void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Tiled 2D tensor copy (no multicast) of one box at element coordinates (x, y) into this CTA's
+// shared memory; completes the box's bytes on `bar`.  x times the element size must be a
+// multiple of 16 bytes.
+CSA2_D void tma_load_2d(void *dst, const void *tmap, int32_t x, int32_t y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 
 // Arrive once and add `bytes` to the transaction count the current phase waits for.
 CSA2_D void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
