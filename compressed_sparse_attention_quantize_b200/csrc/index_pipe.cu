@@ -202,7 +202,6 @@ index_score_pipe_kernel(const Args a, const __grid_constant__ CUtensorMap keys) 
     if (warp == 0) {
         // ================= producer =================
         int issued = 0;
-        bool tail_used = false;
         for (int i = 0; i < ntiles; ++i) {
             const int st = i % kStages;
             if (i >= kStages) {
@@ -231,7 +230,6 @@ index_score_pipe_kernel(const Args a, const __grid_constant__ CUtensorMap keys) 
                     ptx::bulk_load_g2s(S.tail, a.k_codes + (sbase + j) * 32, (uint32_t)rows * 32u, &S.tail_bar);
                     ok = ptx::mbar_wait(&S.tail_bar, 0, abort_flag);
                 }
-                tail_used = true;
                 if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
                 for (int row = lane; row < kTile; row += 32) {
                     uint4 p0 = make_uint4(0u, 0u, 0u, 0u), p1 = p0;
@@ -254,7 +252,6 @@ index_score_pipe_kernel(const Args a, const __grid_constant__ CUtensorMap keys) 
             for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
                 ptx::mbar_wait_drain(&S.full[i % kStages], (i / kStages) & 1);
         }
-        (void)tail_used;
         __syncwarp();
     } else if (warp == 1) {
         // ================= MMA issuer =================

@@ -1,4 +1,4 @@
-// Top-K (and pool) selection by a cluster of 8 CTAs per query row.
+// Top-K (and pool) selection by a cluster of 8 (or, for few rows, 16) CTAs per query row.
 //
 // [A] page "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径", section
 // "压缩吸收注意力（二代）": the indexer keeps 2048 blocks per query and the first layer's
@@ -7,7 +7,7 @@
 // Each CTA of the cluster owns a contiguous chunk of the row's candidates and keeps their
 // order-preserving 32-bit keys in shared memory (read from global once).  Four 8-bit radix
 // passes find the exact threshold key: every CTA builds a 256-bin histogram of its chunk,
-// the cluster barrier publishes them, and every CTA sums the 8 histograms through distributed
+// the cluster barrier publishes them, and every CTA sums the cluster's histograms through distributed
 // shared memory (identical totals -> identical decisions, no broadcast needed).  Compaction:
 // each CTA publishes how many of its keys are above / equal to the threshold; the CTA's output
 // offset and its share of the "equal" keys (lowest indices first) follow from the lower-ranked
@@ -23,7 +23,8 @@ namespace tkc {
 
 namespace cg = cooperative_groups;
 
-constexpr int kCluster = 8;
+constexpr int kCluster = 8;                        // the portable cluster size
+constexpr int kClusterWide = 16;                   // for few rows: twice the SMs per row
 constexpr int kThreads = 512;
 constexpr int kMaxChunk = 32768;                   // keys per CTA (128 KB of shared memory)
 
@@ -99,6 +100,7 @@ CSA2_D int block_excl_sum(int v, int *ws, int &total) {
 }
 
 // One selection of the k largest keys of the row (k < n): writes ids ascending to out[0..k).
+template <int kC>
 CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *keys, int chunk_len,
                            int64_t chunk_base, const int32_t *ids, int k, int32_t *out) {
     const int rank = (int)cl.block_rank();
@@ -121,13 +123,13 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
             if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], (unsigned)__popc(peers));
         }
         cl.sync();                                  // every CTA's histogram is complete
-        if (threadIdx.x < 256) {                    // bin t summed over the cluster (8 DSMEM loads)
-            unsigned int v[kCluster];
+        if (threadIdx.x < 256) {                    // bin t summed over the cluster (kC DSMEM loads)
+            unsigned int v[kC];
 #pragma unroll
-            for (int c = 0; c < kCluster; ++c) v[c] = cl.map_shared_rank(h, c)[threadIdx.x];
+            for (int c = 0; c < kC; ++c) v[c] = cl.map_shared_rank(h, c)[threadIdx.x];
             unsigned int sum = 0;
 #pragma unroll
-            for (int c = 0; c < kCluster; ++c) sum += v[c];
+            for (int c = 0; c < kC; ++c) sum += v[c];
             S.total[threadIdx.x] = sum;
         }
         __syncthreads();
@@ -217,17 +219,18 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
     cl.sync();                                      // counts may be reused by the next selection
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
-topk_cluster_kernel(Args a) {
+// Launched with a cluster of kC CTAs per row (launch attribute).
+template <int kC>
+__global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(Args a) {
     extern __shared__ __align__(16) uint32_t keys[];
     __shared__ Shared S;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
-    const int lr = blockIdx.x / kCluster;
+    const int lr = blockIdx.x / kC;
     const int r = a.row0 + lr;
     int64_t n = row_n(a, r);
     if (n > a.score_stride) n = a.score_stride;
-    const int chunk = (int)((n + kCluster - 1) / kCluster);
+    const int chunk = (int)((n + kC - 1) / kC);
     const int64_t cbase = (int64_t)rank * chunk;
     const int clen = (int)max((int64_t)0, min((int64_t)chunk, n - cbase));
     const float *s = a.scores + (int64_t)lr * a.score_stride;
@@ -246,7 +249,7 @@ topk_cluster_kernel(Args a) {
                 out[j] = ids ? ids[j] : (int32_t)j;
             }
         } else {
-            select_cluster(cl, S, keys, clen, cbase, ids, k, out);
+            select_cluster<kC>(cl, S, keys, clen, cbase, ids, k, out);
         }
         // padding: rank 0 writes -1 to out[c..k)
         if (rank == 0) {
@@ -260,7 +263,66 @@ topk_cluster_kernel(Args a) {
 
 int64_t topk_cluster_max_n() { return (int64_t)tkc::kCluster * tkc::kMaxChunk; }
 
-static SmemLimit g_topk_smem;
+static SmemLimit g_topk_smem, g_topk_smem_wide;
+static std::atomic<int> g_topk_wide_ok[kMaxDevices];      // 0 unknown, 1 yes, -1 no
+
+template <int kC>
+static cudaError_t launch_topk_cluster_n(const tkc::Args &a, int nrows, int64_t max_n, SmemLimit &lim,
+                                         cudaStream_t st) {
+    const int chunk = (int)((max_n + kC - 1) / kC);
+    const size_t smem = (size_t)(chunk > 0 ? chunk : 1) * sizeof(uint32_t);
+    cudaError_t e = ensure_smem_limit(lim, tkc::topk_cluster_kernel<kC>, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nrows * kC));
+    cfg.blockDim = dim3(tkc::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kC;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, tkc::topk_cluster_kernel<kC>, a);
+    note_launches(1);
+    return e;
+}
+
+// Whether clusters of 16 CTAs with `smem` bytes each can be resident on the current device (the
+// size is not portable: it needs the opt-in attribute and enough SMs per GPC).  Once per device.
+static bool topk_wide_clusters(size_t smem) {
+    const int dev = current_device();
+    if (dev < 0) return false;
+    const int known = g_topk_wide_ok[dev].load(std::memory_order_acquire);
+    if (known != 0) return known > 0;
+    std::lock_guard<std::mutex> lock(settings_mutex());
+    bool ok = cudaFuncSetAttribute(tkc::topk_cluster_kernel<tkc::kClusterWide>,
+                                   cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+              cudaFuncSetAttribute(tkc::topk_cluster_kernel<tkc::kClusterWide>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)(tkc::kMaxChunk * sizeof(uint32_t))) == cudaSuccess;
+    if (ok) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(tkc::kClusterWide);
+        cfg.blockDim = dim3(tkc::kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = tkc::kClusterWide;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        ok = cudaOccupancyMaxActiveClusters(&clusters, tkc::topk_cluster_kernel<tkc::kClusterWide>, &cfg) ==
+                 cudaSuccess && clusters > 0;
+    }
+    (void)cudaGetLastError();                   // a refused query leaves no error behind
+    g_topk_wide_ok[dev].store(ok ? 1 : -1, std::memory_order_release);
+    return ok;
+}
 
 // Selection for rows [row0, row0+nrows) from scores in global memory (max_n <= topk_cluster_max_n()).
 cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const int32_t *cand,
@@ -274,13 +336,14 @@ cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const
     a.n_entries = n_entries; a.q_pos = q_pos; a.pool_len = pool_len; a.T = T;
     a.row0 = row0; a.K = K; a.out_idx = out_idx; a.out_cnt = out_cnt;
     a.P = P; a.out_pool = out_pool; a.out_pool_len = out_pool_len;
-    const int chunk = (int)((max_n + tkc::kCluster - 1) / tkc::kCluster);
-    const size_t smem = (size_t)(chunk > 0 ? chunk : 1) * sizeof(uint32_t);
-    cudaError_t e = ensure_smem_limit(g_topk_smem, tkc::topk_cluster_kernel, (int)smem);
-    if (e != cudaSuccess) return e;
-    tkc::topk_cluster_kernel<<<nrows * tkc::kCluster, tkc::kThreads, smem, st>>>(a);
-    note_launches(1);
-    return cudaGetLastError();
+    // few rows: clusters of 16 put twice the SMs on each row when the grid still has one CTA per
+    // SM (measured: 4 rows x 256K scores 78 -> 59 us; 16 rows x 64K with a 16K pool, two CTAs per
+    // SM, was slower at 16 than at 8)
+    const int64_t wide_chunk = (max_n + tkc::kClusterWide - 1) / tkc::kClusterWide;
+    if ((int64_t)nrows * tkc::kClusterWide <= (int64_t)device_sm_count() && wide_chunk >= 1024 &&
+        topk_wide_clusters((size_t)wide_chunk * sizeof(uint32_t)))
+        return launch_topk_cluster_n<tkc::kClusterWide>(a, nrows, max_n, g_topk_smem_wide, st);
+    return launch_topk_cluster_n<tkc::kCluster>(a, nrows, max_n, g_topk_smem, st);
 }
 
 }  // namespace csa2
