@@ -63,7 +63,7 @@ class QuantJob(ctypes.Structure):
 
 
 # the csa2_version() the descriptors and signatures below mirror
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 
 class GroupDesc(ctypes.Structure):
@@ -86,7 +86,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [
         ("mode", _i32), ("q", _vp), ("iq_codes", _vp), ("iq_scales", _vp), ("iw", _vp),
         ("swa_codes", _vp), ("swa_scale", _vp), ("out", _vp), ("lse", _vp), ("idx_out", _vp),
-        ("ready_event", _vp), ("done_event", _vp),
+        ("ready_event", _vp), ("done_event", _vp), ("attn_ready_event", _vp),
     ]
 
 

@@ -136,7 +136,7 @@ const char *csa2_status_string(csa2_status s) {
     return "CSA2: unknown status";
 }
 
-int csa2_version(void) { return 4; }
+int csa2_version(void) { return 5; }
 
 const char *csa2_last_error_string(void) { return t_last_error; }
 
@@ -543,6 +543,10 @@ csa2_status csa2_layer_group(const csa2_group_desc *g, const csa2_layer_desc *la
         if (L.idx_out) {
             cudaError_t e = cudaMemcpyAsync(L.idx_out, idx, (size_t)rows * g->K * 4,
                                             cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+        if (L.attn_ready_event) {
+            cudaError_t e = cudaStreamWaitEvent(st, reinterpret_cast<cudaEvent_t>(L.attn_ready_event), 0);
             if (e != cudaSuccess) return cuda_status(e);
         }
         // attention on `st`; its split merge on the side stream, overlapping the next layers.

@@ -216,12 +216,14 @@ class GroupRunner:
         L.out, L.lse, L.idx_out = ld["out"].data_ptr(), ld["lse"].data_ptr(), ld["idx"].data_ptr()
         return L
 
-    def set_layer_events(self, ready=None, done=None) -> None:
+    def set_layer_events(self, ready=None, done=None, attn_ready=None) -> None:
         """Per-layer cudaEvent_t handles (ints, or None) that the group call waits on before a
-        layer (``ready``) and records after it (``done``); see csa2_layer_group."""
+        layer (``ready``) and before its attention (``attn_ready``), and records after it
+        (``done``); see csa2_layer_group."""
         for l, L in enumerate(self.layer_descs):
             L.ready_event = ready[l] if ready else None
             L.done_event = done[l] if done else None
+            L.attn_ready_event = attn_ready[l] if attn_ready else None
 
     def run(self, stream=None, refresh: Optional[bool] = None) -> None:
         """The layer group; ``refresh`` sets whether a kept pool (keep_pool) is rebuilt."""

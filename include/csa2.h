@@ -337,9 +337,11 @@ CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t *q, int B, int T, i
  * Every layer then runs csa2_sparse_attn with its own main query and its own window over
  * the shared main KV.  Layers run in order on `stream`.
  * Per-layer events (optional, cudaEvent_t passed as void*, owned by the caller): the work of
- * layer l waits on `ready_event` (cudaStreamWaitEvent), e.g. the copy of that layer's query on
- * another stream, and `done_event` is recorded once layer l's work is queued, e.g. to start
- * reading its output back while later layers run.  NULL skips either.
+ * layer l waits on `ready_event` (cudaStreamWaitEvent), e.g. the copy of that layer's indexer
+ * query on another stream; its attention also waits on `attn_ready_event`, e.g. the copy of its
+ * main query, so that the indexer can run while that copy is still in flight; `done_event` is
+ * recorded once layer l's work is queued, e.g. to start reading its output back while later
+ * layers run.  NULL skips any of them.
  * Rejected (INVALID_ARG): a REUSE or REINDEX layer before any FULL layer; REINDEX with
  * P == 0.
  * ---------------------------------------------------------------------------------- */
@@ -384,6 +386,8 @@ typedef struct csa2_layer_desc {
     int32_t *idx_out;            /* optional copy of this layer's selection [B*T][K]   */
     void *ready_event;           /* cudaEvent_t or NULL: the layer's kernels wait for it */
     void *done_event;            /* cudaEvent_t or NULL: recorded after the layer's work */
+    void *attn_ready_event;      /* cudaEvent_t or NULL: the layer's attention (not its
+                                    indexer) also waits for it, e.g. the copy of q        */
 } csa2_layer_desc;
 
 CSA2_API csa2_status csa2_layer_group_workspace_size(const csa2_group_desc *g,

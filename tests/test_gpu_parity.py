@@ -355,28 +355,38 @@ def test_bf16_output():
 
 
 def test_layer_events_same_result():
-    """Per-layer ready/done events (csa2_layer_desc) only order work: the group's outputs with a
-    side stream feeding each layer's query are bit-identical to a plain call."""
+    """Per-layer ready/attn_ready/done events (csa2_layer_desc) only order work: the group's
+    outputs and selections with a side stream feeding each layer's indexer inputs (ready) and
+    then its main query (attn_ready) are bit-identical to a plain call."""
     wl = synth.scaled(synth.workload(2), B=3, n=5000, K=256, P=1200, name="events")
     r = _run_group(wl)
     ref = [ld["out"].clone() for ld in r.layer_data]
+    ref_idx = [ld["idx"].clone() for ld in r.layer_data]
+    names = ("iq_codes", "iq_scales", "iw")
     host_q = [ld["q"].cpu().pin_memory() for ld in r.layer_data]
+    host_i = [{k: ld[k].cpu().pin_memory() for k in names if k in ld} for ld in r.layer_data]
     for ld in r.layer_data:
-        ld["q"].zero_()
-        ld["out"].zero_()
+        for k in ("q", "out", "idx") + names:
+            if k in ld:
+                ld[k].zero_()
     cur = torch.cuda.current_stream()
     side = torch.cuda.Stream()
     ready = [torch.cuda.Event() for _ in r.modes]
+    attn_ready = [torch.cuda.Event() for _ in r.modes]
     done = [torch.cuda.Event() for _ in r.modes]
-    for ev in ready + done:
+    for ev in ready + attn_ready + done:
         ev.record(cur)
     torch.cuda.synchronize()
-    r.set_layer_events([e.cuda_event for e in ready], [e.cuda_event for e in done])
+    r.set_layer_events([e.cuda_event for e in ready], [e.cuda_event for e in done],
+                       [e.cuda_event for e in attn_ready])
     side.wait_stream(cur)
     with torch.cuda.stream(side):
         for l, ld in enumerate(r.layer_data):
-            ld["q"].copy_(host_q[l], non_blocking=True)
+            for k, h in host_i[l].items():
+                ld[k].copy_(h, non_blocking=True)
             ready[l].record(side)
+            ld["q"].copy_(host_q[l], non_blocking=True)
+            attn_ready[l].record(side)
     r.run()
     for l in range(len(r.modes)):
         done[l].synchronize()
@@ -384,6 +394,7 @@ def test_layer_events_same_result():
     r.set_layer_events(None, None)
     for l, ld in enumerate(r.layer_data):
         assert torch.equal(ld["out"], ref[l]), l
+        assert torch.equal(ld["idx"], ref_idx[l]), l
 
 
 def test_graph_replay_same_result():
