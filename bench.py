@@ -323,15 +323,22 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
     aws_bytes = csa2.csa2_sparse_attn_workspace_size(rows, wl.H, wl.K)
     aws = torch.empty((aws_bytes,), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
-    write_graph = None
+    write_graph = floor_graph = None
     if writes:
         runner.write_step()
         torch.cuda.synchronize()
         write_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(write_graph):
             runner.write_step()
+        # the same measurement of a one-element add: what any one-node graph costs here
+        one = torch.zeros((1,), dtype=torch.float32, device=dev)
+        one.add_(1.0)
         torch.cuda.synchronize()
-    times = {"step_writes": [], "index_topk": [], "reindex_topk": [], "sparse_attn": []}
+        floor_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(floor_graph):
+            one.add_(1.0)
+        torch.cuda.synchronize()
+    times = {"step_writes": [], "graph_floor": [], "index_topk": [], "reindex_topk": [], "sparse_attn": []}
     for _ in range(steps):
         flush()
         marks = []
@@ -343,6 +350,11 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
             e0 = ev()
             write_graph.replay()
             marks.append(("step_writes", e0, ev()))
+            flush()
+            e0 = ev()
+            floor_graph.replay()
+            marks.append(("graph_floor", e0, ev()))
+            flush()
         for l, m in enumerate(runner.modes):
             ld = runner.layer_data[l]
             if m != "U":
@@ -370,7 +382,7 @@ def breakdown(torch, csa2, runner, steps, flush, writes=False):
         torch.cuda.synchronize()
         for name, a, b in marks:
             times[name].append(a.elapsed_time(b))
-    del write_graph
+    del write_graph, floor_graph
     return {k: v for k, v in times.items() if v}
 
 
@@ -457,9 +469,9 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     from compressed_sparse_attention_quantize_b200 import runtime, synth
     wl = runner.wl
     def pinned_copy(t):
-        # fresh page-locked buffers: copies of tensor.pin_memory() results ran at a third of
-        # the bandwidth of torch.empty(..., pin_memory=True) buffers on the B200 hosts
-        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        # the library's host buffers (csa2_host_alloc: page-locked, 2 MB pages): copies from
+        # 4 KB-page buffers ran at 32 GB/s and slowed the group beside them by 10-50 %
+        h = csa2.host_empty(t.shape, t.dtype)
         h.copy_(t)
         return h
 
@@ -484,12 +496,13 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
                 iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
                 e["iq"] = pinned_copy(torch.from_numpy(iq))
                 e["iq_dev"] = torch.empty_like(e["iq"], device=ld["q"].device)
+                e["iq_job"] = csa2.quant_job(csa2.FMT_FP4, e["iq_dev"], csa2.DTYPE_F32, e["iq_dev"].shape[0], 64,
+                                             64, ld["iq_codes"], 32, ld["iq_scales"], 4)
                 e["iw"] = pinned_copy(ld["iw"].cpu())
                 h2d += e["iq"].numel() * 4 + e["iw"].numel() * 4
             host.append(e)
         out_last = runner.layer_data[-1]["out"]
-        out_host = torch.empty(out_last.shape, dtype=out_last.dtype, pin_memory=True)
-        out_host.zero_()
+        out_host = csa2.host_empty(out_last.shape, out_last.dtype)
     d2h = out_host.numel() * out_host.element_size()
     cur = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
@@ -502,25 +515,27 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     def body(main):
         copy_stream.wait_stream(main)
         with torch.cuda.stream(copy_stream):
-            if step_host is not None:                 # the step's new entries and window tokens
-                if "kv" in step_host:
-                    runner.step_kv.copy_(step_host["kv"], non_blocking=True)
-                    runner.step_ik.copy_(step_host["ik"], non_blocking=True)
-                if "win" in step_host:
-                    runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
-                jobs = runner.entry_jobs + runner.window_jobs
-                if jobs:
-                    csa2.csa2_quantize_kv_batch(jobs, stream=copy_stream)
             for l, m in enumerate(runner.modes):
                 ld, e = runner.layer_data[l], host[l]
-                # the indexer's inputs first: the layer's indexer starts while its main query,
-                # which only the attention needs, is still being copied
+                # a layer's indexer inputs first, and before the first layer the step's new
+                # entries (the indexer scores them): the indexer starts while the main query and
+                # the window tokens, which only the attention needs, are still being copied
+                jobs = []
                 if m != "U":
                     e["iq_dev"].copy_(e["iq"], non_blocking=True)
                     ld["iw"].copy_(e["iw"], non_blocking=True)
-                    runtime.quantize_fp4_rows(e["iq_dev"], ld["iq_codes"], ld["iq_scales"], 32, 4,
-                                              stream=copy_stream)
+                    jobs.append(e["iq_job"])
+                if l == 0 and step_host is not None and "kv" in step_host:
+                    runner.step_kv.copy_(step_host["kv"], non_blocking=True)
+                    runner.step_ik.copy_(step_host["ik"], non_blocking=True)
+                    jobs += runner.entry_jobs
+                if jobs:
+                    csa2.csa2_quantize_kv_batch(jobs, stream=copy_stream)
                 ready[l].record(copy_stream)
+                if l == 0 and step_host is not None and "win" in step_host:
+                    runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
+                    if runner.window_jobs:
+                        csa2.csa2_quantize_kv_batch(runner.window_jobs, stream=copy_stream)
                 ld["q"].copy_(e["q"], non_blocking=True)
                 attn_ready[l].record(copy_stream)
         runner.run()
@@ -572,11 +587,14 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": sum(ms) / steps,
-            "overlap": "per-layer input copies on a second stream (indexer inputs, then the main query)",
+            "ms_per_step_min_median_max": [min(ms), statistics.median(ms), max(ms)],
+            "overlap": "input copies on a second stream, per layer: indexer inputs (and, before the first "
+                       "layer, the step's new entries), then the window tokens (first layer) and the main query",
             "copy_ms_per_step": copy_ms, "copy_gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
             "copy_note": "the step's copies alone, back to back on one stream (no kernels)",
             "step": "cuda graph" if graph is not None else "eager",
-            "host_buffers": "GPU-local NUMA node" if local.used else "default placement"}
+            "host_buffers": "csa2_host_alloc (page-locked, 2 MB pages), "
+                            + ("GPU-local NUMA node" if local.used else "default placement")}
 
 
 def kernel_table(wl, runner, bd, peaks, out_bytes):
@@ -595,6 +613,9 @@ def kernel_table(wl, runner, bd, peaks, out_bytes):
         wb = write_work(runner)
         kernels["step_writes"] = {"launches_per_step": 1, "calls": write_calls(runner), "avg_ms": t_ms,
                                   "algorithmic_bytes": wb, "achieved_gbs": wb / (t_ms * 1e-3) / 1e9}
+        if "graph_floor" in bd:
+            # the same events around a one-node graph of a one-element add, also after a flush
+            kernels["step_writes"]["one_node_graph_floor_ms"] = statistics.median(bd["graph_floor"])
     if "index_topk" in bd:
         t_ms = statistics.mean(bd["index_topk"])
         ib = index_work(wl)

@@ -22,6 +22,7 @@ __all__ = [
     "csa2_sparse_attn", "csa2_sparse_attn_workspace_size", "csa2_sparse_attn_plan", "csa2_sparse_attn_noalloc",
     "csa2_layer_group", "csa2_layer_group_workspace_size", "csa2_device_error", "csa2_selftest_bounded_wait",
     "csa2_status_string", "csa2_version", "csa2_launch_count", "GroupDesc", "LayerDesc",
+    "csa2_host_alloc", "csa2_host_free", "host_empty",
     "FMT_FP4", "FMT_FP8_TOKEN", "DTYPE_F32", "DTYPE_BF16", "MODE_FULL", "MODE_REINDEX",
     "MODE_REUSE", "CSA2_OK", "CSA2_ERR_INVALID_ARG", "CSA2_ERR_SHAPE", "CSA2_ERR_TIMEOUT",
 ]
@@ -63,7 +64,7 @@ class QuantJob(ctypes.Structure):
 
 
 # the csa2_version() the descriptors and signatures below mirror
-ABI_VERSION = 5
+ABI_VERSION = 6
 
 
 class GroupDesc(ctypes.Structure):
@@ -110,6 +111,10 @@ def lib():
     if L.csa2_version() != ABI_VERSION:
         raise CSA2Error(f"{_LIB_PATH} has ABI version {L.csa2_version()}, this binding expects "
                         f"{ABI_VERSION}; rebuild it with `python -m compressed_sparse_attention_quantize_b200.build`")
+    L.csa2_host_alloc.restype = _i32
+    L.csa2_host_alloc.argtypes = [_sz, ctypes.POINTER(_vp)]
+    L.csa2_host_free.restype = _i32
+    L.csa2_host_free.argtypes = [_vp]
     L.csa2_quantize_kv.restype = _i32
     L.csa2_quantize_kv.argtypes = [_i32, _vp, _i32, _i64, _i32, _i64, _vp, _i64, _vp, _i64, _vp, _vp]
     L.csa2_quantize_kv_batch.restype = _i32
@@ -285,6 +290,39 @@ def csa2_index_topk(mode, q_codes, q_scales, w, B, T, H_I, k_codes, k_code_strid
                                  _ptr(pool_len), P_in, K, _ptr(out_idx), _ptr(out_cnt), P,
                                  _ptr(out_pool), _ptr(out_pool_len), _ptr(workspace), ws_bytes,
                                  _stream(stream)))
+
+
+def csa2_host_alloc(nbytes: int) -> int:
+    """Page-locked host buffer of at least ``nbytes`` on 2 MB pages (address as an int)."""
+    p = _vp()
+    _check(lib().csa2_host_alloc(int(nbytes), ctypes.byref(p)))
+    return int(p.value)
+
+
+def csa2_host_free(ptr: int) -> None:
+    _check(lib().csa2_host_free(ptr))
+
+
+def host_empty(shape, dtype):
+    """A CPU torch tensor in a csa2_host_alloc buffer (page-locked, 2 MB pages, zero-filled by
+    the calling thread); the buffer is freed when the tensor and its views are gone.  Use it for
+    the inputs and outputs a step copies between host and device."""
+    import weakref
+
+    import numpy as np
+    import torch
+    shape = tuple(int(d) for d in shape)
+    numel = 1
+    for d in shape:
+        numel *= d
+    if numel == 0:
+        return torch.empty(shape, dtype=dtype)
+    nbytes = numel * torch.empty((), dtype=dtype).element_size()
+    ptr = csa2_host_alloc(nbytes)
+    buf = (ctypes.c_uint8 * nbytes).from_address(ptr)
+    weakref.finalize(buf, lib().csa2_host_free, ptr)
+    raw = torch.from_numpy(np.frombuffer(buf, dtype=np.uint8))   # holds buf through numpy
+    return raw.view(dtype)[:numel].view(shape)
 
 
 def csa2_pool_extend(pool, pool_len, P_in, n_ref, n_entries, q_pos, B, T, P_out, out_pool, out_len,

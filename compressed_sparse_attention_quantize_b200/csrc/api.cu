@@ -132,11 +132,12 @@ const char *csa2_status_string(csa2_status s) {
         case CSA2_ERR_CUDA: return "CSA2_ERR_CUDA: the CUDA runtime refused a launch";
         case CSA2_ERR_TIMEOUT: return "CSA2_ERR_TIMEOUT: a bounded device wait expired";
         case CSA2_ERR_WORKSPACE: return "CSA2_ERR_WORKSPACE: workspace missing or too small";
+        case CSA2_ERR_HOST: return "CSA2_ERR_HOST: the operating system refused host memory";
     }
     return "CSA2: unknown status";
 }
 
-int csa2_version(void) { return 5; }
+int csa2_version(void) { return 6; }
 
 const char *csa2_last_error_string(void) { return t_last_error; }
 

@@ -55,14 +55,6 @@ CSA2_D uint32_t e4m3_code_mag_rne(float a) {
     return code > 0x7Eu ? 0x7Eu : code;
 }
 
-// Round a non-negative fp32 magnitude to an E2M1 magnitude code (0..7), nearest-even,
-// saturating at 6.  Midpoints: 0.25->0, 0.75->1.0, 1.25->1.0, 1.75->2, 2.5->2, 3.5->4, 5->4.
-CSA2_D uint32_t e2m1_code_mag_rne(float a) {
-    return (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
-           (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
-           (uint32_t)(a > 5.0f);
-}
-
 // E2M1 magnitude table (codes 0..7).
 CSA2_D float e2m1_mag(uint32_t c) {
     // 0, .5, 1, 1.5, 2, 3, 4, 6 without a memory table

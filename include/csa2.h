@@ -49,7 +49,8 @@ typedef enum csa2_status {
     CSA2_ERR_UNSUPPORTED = 4,   /* valid but not implemented (e.g. latent width != 512)  */
     CSA2_ERR_CUDA = 5,          /* the CUDA runtime refused a launch                     */
     CSA2_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (see csa2_device_error) */
-    CSA2_ERR_WORKSPACE = 7      /* workspace NULL or smaller than the size query returned */
+    CSA2_ERR_WORKSPACE = 7,     /* workspace NULL or smaller than the size query returned */
+    CSA2_ERR_HOST = 8           /* the operating system refused host memory              */
 } csa2_status;
 
 /* quantised formats */
@@ -506,6 +507,26 @@ CSA2_API const char *csa2_last_error_string(void);
  * (all devices, all streams) since it was loaded.  A diagnostic for benchmarks.
  * ---------------------------------------------------------------------------------- */
 CSA2_API uint64_t csa2_launch_count(void);
+
+/* ------------------------------------------------------------------------------------
+ * csa2_host_alloc / csa2_host_free -- page-locked host staging buffers for the inputs and
+ * outputs a decode step copies between host and device (no page defines them; they serve
+ * the end-to-end path).  csa2_host_alloc maps `bytes` rounded up to a multiple of 2 MB,
+ * 2 MB-aligned, asks the kernel for transparent huge pages on it (where they are off the
+ * buffer is still valid, on 4 KB pages), writes zeros to every byte from the calling thread
+ * (so the pages sit on that thread's NUMA node under the default policy), page-locks and
+ * registers it with CUDA (cudaHostRegister, default flags: usable by asynchronous copies on
+ * every device and in CUDA graphs), and stores its address in *ptr.  Copies from 2 MB pages
+ * need 512 times fewer address translations than from 4 KB pages: on a B200 over PCIe they
+ * ran faster (50 against 32 GB/s for 2 MB copies) and slowed kernels running beside them less.
+ * The caller owns the buffer until csa2_host_free(ptr), which unregisters and unmaps it.
+ * Errors: INVALID_ARG (ptr NULL; csa2_host_free of an address csa2_host_alloc did not
+ * return, or returned and already freed), SHAPE (bytes == 0 or above 2^40), HOST (the mapping
+ * failed), CUDA (registration failed; nothing stays allocated).  csa2_host_free(NULL) is a
+ * no-op returning OK.  Thread-safe.
+ * ---------------------------------------------------------------------------------- */
+CSA2_API csa2_status csa2_host_alloc(size_t bytes, void **ptr);
+CSA2_API csa2_status csa2_host_free(void *ptr);
 
 #ifdef __cplusplus
 }

@@ -15,7 +15,7 @@ from compressed_sparse_attention_quantize_b200 import build as csa2_build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "csa2.h")
 
-OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT, WS = range(8)
+OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT, WS, HOST = range(9)
 
 
 @pytest.fixture(scope="module")
@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for s in range(8):
+    for s in range(9):
         assert csa2.csa2_status_string(s).startswith("CSA2")
     assert csa2.csa2_version() >= 1
 
@@ -249,3 +249,14 @@ def test_quantize_batch_validation(L):
     assert L.csa2_quantize_kv_batch(None, 0, None) == OK
     empty = csa2.quant_job(0, None, 0, 0, 512, 512, None, 256, None, 32)
     assert L.csa2_quantize_kv_batch((J * 1)(empty), 1, None) == OK        # rows == 0 only
+
+
+def test_host_alloc_validation(L):
+    """csa2_host_alloc / csa2_host_free argument checks (none of them maps or registers memory)."""
+    p = ctypes.c_void_p(1234)
+    assert L.csa2_host_alloc(1 << 20, None) == INVALID
+    assert L.csa2_host_alloc(0, ctypes.byref(p)) == SHAPE
+    assert p.value is None                                   # *ptr cleared on every error
+    assert L.csa2_host_alloc((1 << 40) + 1, ctypes.byref(p)) == SHAPE
+    assert L.csa2_host_free(None) == OK
+    assert L.csa2_host_free(ctypes.c_void_p(4096)) == INVALID  # not from csa2_host_alloc

@@ -30,10 +30,60 @@ def _special_rows(rng, rows, dim):
     return x
 
 
+def _e4m3_values():
+    return np.array([oracle.e4m3_value(c) for c in range(0x7F)], np.float64)
+
+
+def _nudge(x, steps):
+    """x moved by `steps` fp32 ulps (elementwise, towards +inf for positive steps)."""
+    x = x.astype(np.float32)
+    for k in range(int(np.abs(steps).max(initial=0))):
+        up = steps > k
+        dn = steps < -k
+        x = np.where(up, np.nextafter(x, np.float32(np.inf)), x)
+        x = np.where(dn, np.nextafter(x, np.float32(-np.inf)), x)
+    return x.astype(np.float32)
+
+
+def _fp8_tie_rows(rng, rows, dim, exps=(-40, 40)):
+    """Rows whose values sit on, or a few fp32 ulps from, mu * s for E4M3 midpoints mu, where
+    s = amax/448 is the row's fp32 scale (amax near 2^e, e drawn from `exps`): the codes then
+    depend on the exact quotient."""
+    v = _e4m3_values()
+    mids = 0.5 * (v[:-1] + v[1:])
+    x = np.empty((rows, dim), np.float32)
+    for r in range(rows):
+        amax = np.float32(rng.uniform(1.0, 2.0) * 2.0 ** rng.integers(*exps))
+        s = np.float32(amax / np.float32(448.0))
+        mu = rng.choice(mids, dim)
+        x[r] = _nudge(np.float32(mu * np.float64(s)), rng.integers(-2, 3, dim))
+        x[r] *= np.where(rng.random(dim) < 0.5, -1, 1).astype(np.float32)
+        x[r, rng.integers(dim)] = amax
+    return x
+
+
+def _fp4_tie_rows(rng, rows, dim):
+    """Rows whose 16-channel blocks hold 6s (so the block scale is the E4M3 value s) and values
+    on, or a few ulps from, mu * s for the E2M1 midpoints mu."""
+    v = _e4m3_values()
+    s_all = v[(v > 0) & (v <= 64)]
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    x = np.empty((rows, dim), np.float32)
+    for r in range(rows):
+        for b in range(dim // 16):
+            s = rng.choice(s_all)
+            blk = _nudge(np.float32(rng.choice(mids, 16) * s), rng.integers(-2, 3, 16))
+            blk *= np.where(rng.random(16) < 0.5, -1, 1).astype(np.float32)
+            blk[rng.integers(16)] = np.float32(6.0 * s)
+            x[r, b * 16:(b + 1) * 16] = blk
+    return x
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_quantize_fp4_bitexact(dtype):
     rng = np.random.default_rng(100)
     x = _special_rows(rng, 777, 512)
+    x[100:160] = _fp4_tie_rows(rng, 60, 512)
     xt = torch.from_numpy(x).cuda()
     if dtype == "bf16":
         xt = xt.to(torch.bfloat16)
@@ -82,6 +132,64 @@ def test_quantize_batch_bitexact():
     d = dst_8.cpu().numpy()
     assert np.array_equal(c8.cpu().numpy()[d], oc)
     assert np.array_equal(s8.cpu().numpy()[d].view(np.uint32), os_.view(np.uint32))
+
+
+def test_quantize_batch_ties_layouts():
+    """csa2_quantize_kv_batch on values at and next to the rounding midpoints, on row lengths
+    that end inside a thread's channels or exceed what a thread group holds, on rows that are
+    not 16-byte aligned (scalar loads) and code rows that are not 4-byte aligned (byte stores),
+    and on FP8 rows whose scale is too small or too large for the reciprocal shortcut."""
+    rng = np.random.default_rng(104)
+    f4 = _fp4_tie_rows(rng, 64, 512)
+    cases = []                                         # (fmt, x f32 [rows, dim], pad, code_pad)
+    cases.append((csa2.FMT_FP4, f4, 0, 0))
+    cases.append((csa2.FMT_FP4, _fp4_tie_rows(rng, 33, 64), 1, 1))
+    for dim in (16, 528, 2048, 2064):
+        cases.append((csa2.FMT_FP8_TOKEN, _fp8_tie_rows(rng, 9, dim), 0, 0))
+    odd = np.concatenate([_fp8_tie_rows(rng, 4, 512, (-96, -94)),     # scales below 2^-100
+                          _fp8_tie_rows(rng, 4, 512, (110, 113)),     # scales above 2^100
+                          _fp8_tie_rows(rng, 4, 512, (-136, -126))])  # subnormal amax
+    cases.append((csa2.FMT_FP8_TOKEN, odd, 3, 1))
+    jobs, outs = [], []
+    for fmt, x, pad, cpad in cases:
+        rows, dim = x.shape
+        if pad:                                        # rows start one element in: misaligned
+            xp = np.zeros((rows, dim + pad + 1), np.float32)
+            xp[:, 1:dim + 1] = x
+            xt = torch.from_numpy(xp).cuda()
+            xv = xt[:, 1:]
+        else:
+            xt = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+            xv = xt
+        if fmt == csa2.FMT_FP4:
+            cs = dim // 2 + dim // 16 + cpad
+            buf = torch.zeros((rows + 3, cs), dtype=torch.uint8, device="cuda")
+            dst = torch.from_numpy(rng.permutation(rows + 3)[:rows].astype(np.int64)).cuda()
+            jobs.append(csa2.quant_job(fmt, xv, csa2.DTYPE_F32, rows, dim, xv.stride(0), buf, cs,
+                                       buf[:, dim // 2:], cs, dst))
+            outs.append((fmt, x, buf, dst, None))
+        else:
+            cs = dim + cpad
+            buf = torch.zeros((rows + 3, cs), dtype=torch.uint8, device="cuda")
+            sc = torch.zeros((rows + 3,), dtype=torch.float32, device="cuda")
+            dst = torch.from_numpy(rng.permutation(rows + 3)[:rows].astype(np.int64)).cuda()
+            jobs.append(csa2.quant_job(fmt, xv, csa2.DTYPE_F32, rows, dim, xv.stride(0), buf, cs, sc, 4, dst))
+            outs.append((fmt, x, buf, dst, sc))
+        outs[-1] = outs[-1] + (xt,)
+    csa2.csa2_quantize_kv_batch(jobs)
+    torch.cuda.synchronize()
+    for fmt, x, buf, dst, sc, _ in outs:
+        d = dst.cpu().numpy()
+        dim = x.shape[1]
+        got = buf.cpu().numpy()[d]
+        if fmt == csa2.FMT_FP4:
+            oc, os_ = oracle.quantize_fp4(x)
+            assert np.array_equal(got[:, :dim // 2], oc), dim
+            assert np.array_equal(got[:, dim // 2:dim // 2 + dim // 16], os_), dim
+        else:
+            oc, os_ = oracle.quantize_fp8_token(x)
+            assert np.array_equal(got[:, :dim], oc), dim
+            assert np.array_equal(sc.cpu().numpy()[d].view(np.uint32), os_.view(np.uint32)), dim
 
 
 def test_quantize_fp4_scatter_rows():
@@ -140,6 +248,9 @@ def test_quantize_fp8_token_bitexact():
     # rows whose scale is exactly 1 put many values on E4M3 ties
     x[10] = np.float32(448.0)
     x[10, 1:100] = np.linspace(200, 250, 99, dtype=np.float32)
+    x[20:60] = _fp8_tie_rows(rng, 40, 512)
+    x[60:64] = _fp8_tie_rows(rng, 4, 512, (-136, -94))    # scales below 2^-100
+    x[64:68] = _fp8_tie_rows(rng, 4, 512, (110, 113))     # scales above 2^100
     xt = torch.from_numpy(x).cuda()
     codes = torch.empty((300, 512), dtype=torch.uint8, device="cuda")
     scales = torch.empty((300,), dtype=torch.float32, device="cuda")
@@ -688,3 +799,36 @@ def test_topk_merge_shards_matches_oracle(G):
         i = np.concatenate([ids[g, r, :cnt[g, r]] for g in range(G)])
         ref, rc = oracle.topk(s, K, ids=i)
         assert int(oc[r]) == rc and np.array_equal(out[r].cpu().numpy(), ref), r
+
+
+def test_host_buffers_copy_and_graph():
+    """csa2_host_alloc buffers (through host_empty): page-locked, asynchronous copies both ways
+    on a side stream and inside a CUDA graph return the bytes written; a second free of the
+    same address is refused."""
+    src = csa2.host_empty((1000, 512), torch.bfloat16)
+    assert src.is_pinned()
+    ref = torch.randn((1000, 512), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    src.copy_(ref)
+    dst = csa2.host_empty((1000, 512), torch.bfloat16)
+    dev = torch.empty((1000, 512), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dev.copy_(src, non_blocking=True)
+        dev.mul_(2)
+        dst.copy_(dev, non_blocking=True)
+    s.synchronize()
+    assert torch.equal(dst, ref * 2)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dev.copy_(src, non_blocking=True)
+        dev.add_(1)
+        dst.copy_(dev, non_blocking=True)
+    src.copy_(ref * 3)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(dst, ref * 3 + 1)
+    del g
+    p = csa2.csa2_host_alloc(3 << 20)
+    csa2.csa2_host_free(p)
+    with pytest.raises(csa2.CSA2Error):
+        csa2.csa2_host_free(p)
