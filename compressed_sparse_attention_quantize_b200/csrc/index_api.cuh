@@ -4,6 +4,18 @@
 
 namespace csa2 {
 
+// One head's dot product from its four block partials, added in block order: u[q] is the raw
+// E2M1 product sum of block q (a multiple of 1/4 below 2^10: at most 12 significant bits) and
+// c[q] = s_q * s_k the product of two E4M3 scales (at most 8 bits, exact), so every partial
+// u[q] * c[q] is exact in fp32 and a fused multiply-add rounds only the sum: the result equals
+// rounding each product (exactly) and then each sum.
+CSA2_D float head_block_sum(const uint32_t *u, const float (&c)[4]) {
+    float d = __fmul_rn(__uint_as_float(u[0]), c[0]);
+    d = __fmaf_rn(__uint_as_float(u[1]), c[1], d);
+    d = __fmaf_rn(__uint_as_float(u[2]), c[2], d);
+    return __fmaf_rn(__uint_as_float(u[3]), c[3], d);
+}
+
 struct IndexLaunch {
     int mode;
     const uint8_t *q_codes;

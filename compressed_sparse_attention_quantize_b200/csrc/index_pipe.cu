@@ -38,6 +38,7 @@ constexpr int kThreads = 192;
 constexpr int kStageBytes = kTile * 32;               // 4 KB: 128 key rows, 32-byte swizzle
 constexpr int kMaxN = kMaxR * 4 * CSA2_MAX_INDEX_HEADS; // B columns (rows x heads x blocks)
 constexpr int kSfCols = 32;
+constexpr int kRegHeads = 8;                          // heads of the register-held epilogue
 
 struct Args {
     const uint8_t *q_codes, *q_scales;
@@ -274,6 +275,54 @@ index_score_pipe_kernel(const Args a, const __grid_constant__ CUtensorMap keys) 
             ptx::mbar_wait_drain(&S.drain, 0);
         }
         __syncwarp();
+    } else if (R == 1 && H == kRegHeads) {
+        // ======= epilogue, one row of 8 heads: its scales and weights held in registers =======
+        const int sub = warp & 3;
+        const int key = sub * 32 + lane;                   // TMEM lane = key within the tile
+        const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
+        float qs[kRegHeads][4], wh[kRegHeads];
+#pragma unroll
+        for (int h = 0; h < kRegHeads; ++h) {
+            wh[h] = S.w[0][h];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) qs[h][q] = S.qs[0][h * 4 + q];
+        }
+        const int64_t n_row = S.n_row[0];
+        float *out = a.scores + (int64_t)(g0 - a.row0) * a.score_stride;
+        for (int i = 0; i < ntiles; ++i) {
+            const int buf = i % kNBuf;
+            if (!ptx::mbar_wait(&S.tfull[buf], (i / kNBuf) & 1, abort_flag)) break;
+            ptx::tc_fence_after();
+            // heads 0-3, then 4-7: 16 accumulator columns at a time keep the registers in budget
+            uint32_t u[16];
+            ptx::tmem_ld16(lane_addr + buf * NT, u);
+            const uint32_t sc_this = S.scales[i % kStages][key];
+            ptx::mbar_arrive(&S.empty[i % kStages]);
+            float sk[4];
+            ptx::e4m3x4_to_f32(sc_this, sk);
+            float acc = 0.0f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1) ptx::tmem_ld16(lane_addr + buf * NT + 16, u);
+                ptx::tmem_ld_wait();
+                if (half == 1) {
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(&S.tempty[buf]);      // the accumulator is in registers
+                }
+#pragma unroll
+                for (int hh = 0; hh < 4; ++hh) {
+                    const int h = half * 4 + hh;
+                    float c[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) c[q] = __fmul_rn(qs[h][q], sk[q]);
+                    const float dot = head_block_sum(u + hh * 4, c);
+                    acc = __fadd_rn(acc, __fmul_rn(wh[h], dot > 0.0f ? dot : 0.0f));
+                }
+            }
+            if (acc == 0.0f) acc = 0.0f;                     // -0 -> +0
+            const int64_t j = j0 + (int64_t)i * kTile + key;
+            if (j < n_row) out[j] = acc;
+        }
     } else {
         // ================= epilogue: one key per thread =================
         const int sub = warp & 3;
@@ -288,8 +337,7 @@ index_score_pipe_kernel(const Args a, const __grid_constant__ CUtensorMap keys) 
             const uint32_t sc_this = S.scales[i % kStages][key];
             ptx::mbar_arrive(&S.empty[i % kStages]);
             float sk[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
+            ptx::e4m3x4_to_f32(sc_this, sk);
             const int64_t j = j0 + (int64_t)i * kTile + key;
             for (int rr = 0; rr < R; ++rr) {
                 float acc = 0.0f;
@@ -301,11 +349,10 @@ index_score_pipe_kernel(const Args a, const __grid_constant__ CUtensorMap keys) 
                     for (int hh = 0; hh < 8; ++hh) {
                         const int h = hb * 8 + hh;
                         if (h < H) {
-                            float p[4];
+                            float c[4];
 #pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[rr][h * 4 + q], sk[q]));
-                            const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
+                            for (int q = 0; q < 4; ++q) c[q] = __fmul_rn(S.qs[rr][h * 4 + q], sk[q]);
+                            const float dot = head_block_sum(u + hh * 4, c);
                             const float rl = dot > 0.0f ? dot : 0.0f;
                             acc = __fadd_rn(acc, __fmul_rn(S.w[rr][h], rl));
                         }

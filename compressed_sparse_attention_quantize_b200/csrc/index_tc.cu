@@ -198,8 +198,7 @@ index_score_tc_kernel(Args a) {
         if (__syncthreads_or(*abort_flag != 0)) return false;
         ptx::tc_fence_after();
         float sk[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sk[q] = e4m3_to_f32((sc_this >> (8 * q)) & 0xFFu);
+        ptx::e4m3x4_to_f32(sc_this, sk);
         float acc = 0.0f;
         for (int hb = 0; hb * 8 < H; ++hb) {
             uint32_t u[32];
@@ -209,11 +208,10 @@ index_score_tc_kernel(Args a) {
             for (int hh = 0; hh < 8; ++hh) {
                 const int h = hb * 8 + hh;
                 if (h < H) {
-                    float p[4];
+                    float c[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        p[q] = __fmul_rn(__uint_as_float(u[hh * 4 + q]), __fmul_rn(S.qs[h * 4 + q], sk[q]));
-                    const float dot = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), p[2]), p[3]);
+                    for (int q = 0; q < 4; ++q) c[q] = __fmul_rn(S.qs[h * 4 + q], sk[q]);
+                    const float dot = head_block_sum(u + hh * 4, c);
                     const float rl = dot > 0.0f ? dot : 0.0f;
                     acc = __fadd_rn(acc, __fmul_rn(S.w[h], rl));
                 }

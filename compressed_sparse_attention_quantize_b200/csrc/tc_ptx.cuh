@@ -232,6 +232,14 @@ CSA2_D uint32_t e4m3x2_to_f16x2(uint16_t v) {
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
     return r;
 }
+// The four E4M3 bytes of a 32-bit word (byte q = block q) as floats: two hardware conversions to
+// f16 pairs, each exact (every finite E4M3 value is an f16 value), then f16 -> f32 (exact).
+CSA2_D void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
+    const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(w & 0xFFFFu)), hi = e4m3x2_to_f16x2((uint16_t)(w >> 16));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
 CSA2_D uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     __half2 x = *reinterpret_cast<__half2 *>(&a), y = *reinterpret_cast<__half2 *>(&b);
     __half2 z = __hmul2(x, y);
