@@ -58,13 +58,11 @@ CSA2_D int64_t row_n(const Args &a, int r) {
     return n;
 }
 
-struct Shared {
+struct alignas(16) Shared {
     unsigned int hist[2][256];
-    unsigned int total[256];
+    alignas(16) unsigned int total[256];
     int counts[2];              // [0] above threshold, [1] equal to it
     int warp_sums[33];
-    uint32_t prefix, mask;
-    int remaining;
 };
 
 static_assert(kThreads % 32 == 0 && kThreads <= 1024, "block scans need whole warps, at most 32");
@@ -99,19 +97,57 @@ CSA2_D int block_excl_sum(int v, int *ws, int &total) {
     return res;
 }
 
+// The digit of the k-th place from the cluster's histogram totals (S.total): every warp reads
+// the 256 totals and takes the same decision, so no barrier hands it out.  Updates the prefix,
+// mask and the count still needed inside the chosen bin.
+CSA2_D void choose_digit(const Shared &S, int shift, uint32_t &prefix, uint32_t &mask, int &remaining) {
+    const int lane = threadIdx.x & 31;
+    const uint4 t0 = reinterpret_cast<const uint4 *>(S.total)[2 * lane];
+    const uint4 t1 = reinterpret_cast<const uint4 *>(S.total)[2 * lane + 1];
+    const unsigned int bins[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+    unsigned int local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) local += bins[i];
+    unsigned int suffix = local;                    // sum over lanes >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned int x = __shfl_down_sync(0xffffffffu, suffix, o);
+        if (lane + o < 32) suffix += x;
+    }
+    const unsigned int above = suffix - local;
+    const bool crosses = (int)above < remaining && remaining <= (int)suffix;
+    const int owner = __ffs(__ballot_sync(0xffffffffu, crosses)) - 1;
+    // the owner lane walks its 8 bins from the top (unrolled: the bins stay in registers)
+    int acc = (int)above, dsel = 0;
+    bool found = false;
+#pragma unroll
+    for (int d = 7; d >= 0; --d) {
+        if (!found && (d == 0 || acc + (int)bins[d] >= remaining)) {
+            dsel = d;
+            found = true;
+        } else if (!found) {
+            acc += (int)bins[d];
+        }
+    }
+    const int take_rem = __shfl_sync(0xffffffffu, remaining - acc, owner);
+    const int digit = __shfl_sync(0xffffffffu, lane * 8 + dsel, owner);
+    remaining = take_rem;
+    prefix |= (uint32_t)digit << shift;
+    mask |= 255u << shift;
+}
+
 // One selection of the k largest keys of the row (k < n): writes ids ascending to out[0..k).
 template <int kC>
 CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *keys, int chunk_len,
                            int64_t chunk_base, const int32_t *ids, int k, int32_t *out) {
     const int rank = (int)cl.block_rank();
-    if (threadIdx.x == 0) { S.prefix = 0u; S.mask = 0u; S.remaining = k; }
-    __syncthreads();
+    uint32_t prefix = 0u, mask = 0u;
+    int remaining = k;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         unsigned int *h = S.hist[pass & 1];
         for (int i = threadIdx.x; i < 256; i += kThreads) h[i] = 0u;
         __syncthreads();
-        const uint32_t prefix = S.prefix, mask = S.mask;
         // warp-aggregated: lanes with the same bin add once (the top digits of nearby scores
         // collide heavily, which would serialise plain shared-memory atomics)
         for (int base = 0; base < chunk_len; base += kThreads) {
@@ -133,56 +169,28 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
             S.total[threadIdx.x] = sum;
         }
         __syncthreads();
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
-            unsigned int bins[8];
-            unsigned int local = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                bins[i] = S.total[lane * 8 + i];
-                local += bins[i];
-            }
-            unsigned int suffix = local;            // sum over lanes >= lane
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned int x = __shfl_down_sync(0xffffffffu, suffix, o);
-                if (lane + o < 32) suffix += x;
-            }
-            const int rem = S.remaining;
-            const unsigned int above = suffix - local;
-            const bool crosses = (int)above < rem && rem <= (int)suffix;
-            const unsigned bal = __ballot_sync(0xffffffffu, crosses);
-            const int owner = __ffs(bal) - 1;
-            if (lane == owner) {
-                int acc = (int)above;
-                int d = 7;
-                for (; d > 0; --d) {
-                    if (acc + (int)bins[d] >= rem) break;
-                    acc += (int)bins[d];
-                }
-                S.remaining = rem - acc;
-                S.prefix = prefix | ((uint32_t)(lane * 8 + d) << shift);
-                S.mask = mask | (255u << shift);
-            }
-        }
-        __syncthreads();
-        // histograms are double-buffered: the next pass writes the other buffer, and the pass
-        // after that is separated from these remote reads by the next pass's cluster barrier
+        choose_digit(S, shift, prefix, mask, remaining);
+        // S.total is rewritten only after the next pass's cluster barrier, and the histograms
+        // are double-buffered: the next pass writes the other buffer, and the pass after that is
+        // separated from these remote reads by the next pass's cluster barrier
     }
-    const uint32_t thr = S.prefix;
-    const int need_eq = S.remaining;
-    // counts of this chunk
-    int gt = 0, eq = 0;
-    for (int i = threadIdx.x; i < chunk_len; i += kThreads) {
+    const uint32_t thr = prefix;
+    const int need_eq = remaining;
+    // ordered compaction of this chunk: thread t owns the consecutive keys [t*per, (t+1)*per).
+    // One block scan of (above, equal) counts packed in 16-bit halves gives the thread's place
+    // among this CTA's selections; the CTA's place follows from the lower-ranked CTAs' totals.
+    const int per = ((chunk_len + kThreads - 1) / kThreads) | 1;     // odd: a warp's lanes hit 32 banks
+    const int i0 = min(chunk_len, threadIdx.x * per), i1 = min(chunk_len, i0 + per);
+    int my_gt = 0, my_eq = 0;
+    for (int i = i0; i < i1; ++i) {
         const uint32_t key = keys[i];
-        gt += key > thr;
-        eq += key == thr;
+        my_gt += key > thr;
+        my_eq += key == thr;
     }
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    eq = __reduce_add_sync(0xffffffffu, eq);
-    if (threadIdx.x == 0) { S.counts[0] = 0; S.counts[1] = 0; }
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) { atomicAdd(&S.counts[0], gt); atomicAdd(&S.counts[1], eq); }
+    int tot;
+    const int pre = block_excl_sum((my_gt << 16) | my_eq, S.warp_sums, tot);   // counts < 2^16
+    const int gt_pre = pre >> 16, eq_pre = pre & 0xFFFF;
+    if (threadIdx.x == 0) { S.counts[0] = tot >> 16; S.counts[1] = tot & 0xFFFF; }
     cl.sync();
     int out_base = 0, eq_before = 0;
     for (int c = 0; c < rank; ++c) {
@@ -192,21 +200,10 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
         out_base += g + take;
         eq_before += e;
     }
-    // ordered compaction of this chunk: thread t owns the consecutive keys [t*per, (t+1)*per),
-    // so two block scans (equal keys before it, selections before it) place every output
-    const int per = ((chunk_len + kThreads - 1) / kThreads) | 1;     // odd: a warp's lanes hit 32 banks
-    const int i0 = min(chunk_len, threadIdx.x * per), i1 = min(chunk_len, i0 + per);
-    int my_gt = 0, my_eq = 0;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t key = keys[i];
-        my_gt += key > thr;
-        my_eq += key == thr;
-    }
-    int eq_tot;
-    const int eq_pre = block_excl_sum(my_eq, S.warp_sums, eq_tot);
-    const int take = min(my_eq, max(0, need_eq - (eq_before + eq_pre)));     // my equal keys taken
-    int sel_tot;
-    int o = out_base + block_excl_sum(my_gt + take, S.warp_sums, sel_tot);
+    // equal keys go to the lowest positions first: this thread's share, and the ones before it
+    const int quota = max(0, need_eq - eq_before);
+    const int take = min(my_eq, max(0, quota - eq_pre));
+    int o = out_base + gt_pre + min(eq_pre, quota);
     int eq_seen = 0;
     for (int i = i0; i < i1; ++i) {
         const uint32_t key = keys[i];
@@ -259,6 +256,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(Args a) {
     }
 }
 
+// Dynamic shared memory of a CTA holding `chunk` keys.
+constexpr size_t smem_of(int chunk) { return (size_t)chunk * sizeof(uint32_t); }
+
 }  // namespace tkc
 
 int64_t topk_cluster_max_n() { return (int64_t)tkc::kCluster * tkc::kMaxChunk; }
@@ -270,7 +270,7 @@ template <int kC>
 static cudaError_t launch_topk_cluster_n(const tkc::Args &a, int nrows, int64_t max_n, SmemLimit &lim,
                                          cudaStream_t st) {
     const int chunk = (int)((max_n + kC - 1) / kC);
-    const size_t smem = (size_t)(chunk > 0 ? chunk : 1) * sizeof(uint32_t);
+    const size_t smem = tkc::smem_of(chunk > 0 ? chunk : 1);
     cudaError_t e = ensure_smem_limit(lim, tkc::topk_cluster_kernel<kC>, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -302,7 +302,7 @@ static bool topk_wide_clusters(size_t smem) {
                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
               cudaFuncSetAttribute(tkc::topk_cluster_kernel<tkc::kClusterWide>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)(tkc::kMaxChunk * sizeof(uint32_t))) == cudaSuccess;
+                                   (int)tkc::smem_of(tkc::kMaxChunk)) == cudaSuccess;
     if (ok) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(tkc::kClusterWide);
@@ -341,7 +341,7 @@ cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const
     // SM, was slower at 16 than at 8)
     const int64_t wide_chunk = (max_n + tkc::kClusterWide - 1) / tkc::kClusterWide;
     if ((int64_t)nrows * tkc::kClusterWide <= (int64_t)device_sm_count() && wide_chunk >= 1024 &&
-        topk_wide_clusters((size_t)wide_chunk * sizeof(uint32_t)))
+        topk_wide_clusters(tkc::smem_of((int)wide_chunk)))
         return launch_topk_cluster_n<tkc::kClusterWide>(a, nrows, max_n, g_topk_smem_wide, st);
     return launch_topk_cluster_n<tkc::kCluster>(a, nrows, max_n, g_topk_smem, st);
 }
