@@ -421,6 +421,40 @@ class gpu_local_cpus:
         return False
 
 
+def host_page_report(tensors):
+    """How the host buffers are backed, from /proc/self/smaps and numa_maps (read-only): resident
+    and transparent-huge-page kB, and pages per NUMA node, over the mappings that hold them."""
+    ranges = [(t.data_ptr(), t.data_ptr() + t.numel() * t.element_size()) for t in tensors if t.numel()]
+    rep = {"rss_kb": 0, "anon_huge_kb": 0, "nodes": {}}
+    try:
+        vmas = set()
+        cur = None
+        with open("/proc/self/smaps") as f:
+            for line in f:
+                head = line.split()
+                if "-" in head[0] and len(head) >= 5 and all(c in "0123456789abcdef-" for c in head[0]):
+                    lo, hi = (int(x, 16) for x in head[0].split("-"))
+                    cur = (lo, hi) if any(a < hi and b > lo for a, b in ranges) else None
+                    if cur:
+                        vmas.add(cur)
+                elif cur and head[0] == "Rss:":
+                    rep["rss_kb"] += int(head[1])
+                elif cur and head[0] == "AnonHugePages:":
+                    rep["anon_huge_kb"] += int(head[1])
+        starts = {lo for lo, _ in vmas}
+        with open("/proc/self/numa_maps") as f:
+            for line in f:
+                parts = line.split()
+                if int(parts[0], 16) in starts:
+                    for tok in parts[2:]:
+                        if tok.startswith("N") and "=" in tok:
+                            node, n = tok.split("=")
+                            rep["nodes"][node] = rep["nodes"].get(node, 0) + int(n)
+    except (OSError, ValueError, IndexError) as exc:
+        rep["error"] = f"{type(exc).__name__}: {exc}"[:120]
+    return rep
+
+
 def topk_side_reference(torch, csa2, wl, flush, reps=10):
     """torch.topk next to the library's top-K on the same fp32 score buffer (side reference only).
 
@@ -503,6 +537,8 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
             host.append(e)
         out_last = runner.layer_data[-1]["out"]
         out_host = csa2.host_empty(out_last.shape, out_last.dtype)
+    pages = host_page_report([t for e in host for k, t in e.items() if k in ("q", "iq", "iw")]
+                             + list((step_host or {}).values()) + [out_host])
     d2h = out_host.numel() * out_host.element_size()
     cur = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
@@ -593,8 +629,9 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
             "copy_ms_per_step": copy_ms, "copy_gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
             "copy_note": "the step's copies alone, back to back on one stream (no kernels)",
             "step": "cuda graph" if graph is not None else "eager",
-            "host_buffers": "csa2_host_alloc (page-locked, 2 MB pages), "
-                            + ("GPU-local NUMA node" if local.used else "default placement")}
+            "host_buffers": "csa2_host_alloc (page-locked, 2 MB pages requested), "
+                            + ("allocated on the GPU's local CPUs" if local.used else "default placement"),
+            "host_pages": pages}
 
 
 def kernel_table(wl, runner, bd, peaks, out_bytes):
