@@ -509,37 +509,71 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
         h.copy_(t)
         return h
 
+    class Stage:
+        """Several small inputs in one host buffer and one device buffer, so that they cross in
+        one copy (every copy pays a few microseconds before its first byte lands)."""
+
+        def __init__(self, parts):
+            offs, n = [], 0
+            for _, t in parts:
+                offs.append(n)
+                n += (t.numel() * t.element_size() + 255) // 256 * 256
+            self.host = csa2.host_empty((n,), torch.uint8)
+            self.dev = torch.empty((n,), dtype=torch.uint8, device="cuda")
+            self.views, self.bytes = {}, 0
+            for (name, t), o in zip(parts, offs):
+                nb = t.numel() * t.element_size()
+                self.host[o:o + nb].view(t.dtype).view(t.shape).copy_(t)
+                self.views[name] = self.dev[o:o + nb].view(t.dtype).view(t.shape)
+                self.bytes += nb
+
+        def copy(self):
+            self.dev.copy_(self.host, non_blocking=True)
+
     host = []
     h2d = 0
-    step_host = None
+    stages = [None] * len(runner.modes)      # per layer: its indexer inputs (+ the new entries)
+    win_stage = None
     with gpu_local_cpus(torch) as local:
-        if writes:
-            step_host = {}
-            if runner.step_rows is not None:
-                step_host["kv"] = pinned_copy(runner.step_kv.cpu())
-                step_host["ik"] = pinned_copy(runner.step_ik.cpu())
-            if runner.step_win_rows is not None:
-                step_host["win"] = pinned_copy(runner.step_win_lat.cpu())
-            h2d += sum(t.numel() * 4 for t in step_host.values())
         for l, m in enumerate(runner.modes):
             ld = runner.layer_data[l]
             hq = pinned_copy(ld["q"].cpu())
-            e = {"q": hq}
+            host.append({"q": hq})
             h2d += hq.numel() * 2
+            parts = []
             if m != "U":
                 iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
-                e["iq"] = pinned_copy(torch.from_numpy(iq))
-                e["iq_dev"] = torch.empty_like(e["iq"], device=ld["q"].device)
-                e["iq_job"] = csa2.quant_job(csa2.FMT_FP4, e["iq_dev"], csa2.DTYPE_F32, e["iq_dev"].shape[0], 64,
-                                             64, ld["iq_codes"], 32, ld["iq_scales"], 4)
-                e["iw"] = pinned_copy(ld["iw"].cpu())
-                h2d += e["iq"].numel() * 4 + e["iw"].numel() * 4
-            host.append(e)
+                parts += [("iq", torch.from_numpy(iq)), ("iw", ld["iw"].cpu())]
+            if l == 0 and writes and runner.step_rows is not None:
+                parts += [("kv", runner.step_kv.cpu()), ("ik", runner.step_ik.cpu())]
+            if parts:
+                stages[l] = Stage(parts)
+                h2d += stages[l].bytes
+        if writes and runner.step_win_rows is not None:
+            win_stage = Stage([("win", runner.step_win_lat.cpu())])
+            h2d += win_stage.bytes
         out_last = runner.layer_data[-1]["out"]
         out_host = csa2.host_empty(out_last.shape, out_last.dtype)
-    pages = host_page_report([t for e in host for k, t in e.items() if k in ("q", "iq", "iw")]
-                             + list((step_host or {}).values()) + [out_host])
+    pages = host_page_report([e["q"] for e in host] + [st.host for st in stages if st is not None]
+                             + ([win_stage.host] if win_stage else []) + [out_host])
     d2h = out_host.numel() * out_host.element_size()
+    # quantise-on-write jobs and indexer weights read the device halves of the stages
+    st0 = stages[0]
+    entry_jobs, window_jobs, query_jobs = runner.write_jobs(
+        kv=st0.views.get("kv") if st0 else None, ik=st0.views.get("ik") if st0 else None,
+        win=win_stage.views["win"] if win_stage else None,
+        iq=[st.views["iq"] if st is not None and "iq" in st.views else None for st in stages])
+    qjob = iter(query_jobs)
+    stage_jobs = []
+    for l, m in enumerate(runner.modes):
+        jobs = [next(qjob)] if m != "U" else []
+        if l == 0 and writes:
+            jobs += entry_jobs
+        stage_jobs.append(jobs)
+    saved_iw = [L.iw for L in runner.layer_descs]
+    for l, st in enumerate(stages):
+        if st is not None and "iw" in st.views:
+            runner.layer_descs[l].iw = st.views["iw"].data_ptr()
     cur = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
     ready = [torch.cuda.Event() for _ in runner.modes]
@@ -554,24 +588,17 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
             for l, m in enumerate(runner.modes):
                 ld, e = runner.layer_data[l], host[l]
                 # a layer's indexer inputs first, and before the first layer the step's new
-                # entries (the indexer scores them): the indexer starts while the main query and
-                # the window tokens, which only the attention needs, are still being copied
-                jobs = []
-                if m != "U":
-                    e["iq_dev"].copy_(e["iq"], non_blocking=True)
-                    ld["iw"].copy_(e["iw"], non_blocking=True)
-                    jobs.append(e["iq_job"])
-                if l == 0 and step_host is not None and "kv" in step_host:
-                    runner.step_kv.copy_(step_host["kv"], non_blocking=True)
-                    runner.step_ik.copy_(step_host["ik"], non_blocking=True)
-                    jobs += runner.entry_jobs
-                if jobs:
-                    csa2.csa2_quantize_kv_batch(jobs, stream=copy_stream)
+                # entries (the indexer scores them), in one copy: the indexer starts while the
+                # main query and the window tokens, which only the attention needs, are still
+                # being copied
+                if stages[l] is not None:
+                    stages[l].copy()
+                if stage_jobs[l]:
+                    csa2.csa2_quantize_kv_batch(stage_jobs[l], stream=copy_stream)
                 ready[l].record(copy_stream)
-                if l == 0 and step_host is not None and "win" in step_host:
-                    runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
-                    if runner.window_jobs:
-                        csa2.csa2_quantize_kv_batch(runner.window_jobs, stream=copy_stream)
+                if l == 0 and win_stage is not None:
+                    win_stage.copy()
+                    csa2.csa2_quantize_kv_batch(window_jobs, stream=copy_stream)
                 ld["q"].copy_(e["q"], non_blocking=True)
                 attn_ready[l].record(copy_stream)
         runner.run()
@@ -579,18 +606,12 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
 
     def copies_only():
         """The step's host->device and device->host copies alone (same buffers, same order)."""
-        if step_host is not None:
-            if "kv" in step_host:
-                runner.step_kv.copy_(step_host["kv"], non_blocking=True)
-                runner.step_ik.copy_(step_host["ik"], non_blocking=True)
-            if "win" in step_host:
-                runner.step_win_lat.copy_(step_host["win"], non_blocking=True)
-        for l, m in enumerate(runner.modes):
-            ld, e = runner.layer_data[l], host[l]
-            ld["q"].copy_(e["q"], non_blocking=True)
-            if m != "U":
-                e["iq_dev"].copy_(e["iq"], non_blocking=True)
-                ld["iw"].copy_(e["iw"], non_blocking=True)
+        for l in range(len(runner.modes)):
+            if stages[l] is not None:
+                stages[l].copy()
+            if l == 0 and win_stage is not None:
+                win_stage.copy()
+            runner.layer_data[l]["q"].copy_(host[l]["q"], non_blocking=True)
         out_host.copy_(out_last, non_blocking=True)
 
     graph = None
@@ -620,12 +641,15 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     finally:
         torch.cuda.synchronize()
         runner.set_layer_events(None, None)
+        for L, p in zip(runner.layer_descs, saved_iw):
+            L.iw = p
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": sum(ms) / steps,
             "ms_per_step_min_median_max": [min(ms), statistics.median(ms), max(ms)],
             "overlap": "input copies on a second stream, per layer: indexer inputs (and, before the first "
-                       "layer, the step's new entries), then the window tokens (first layer) and the main query",
+                       "layer, the step's new entries) in one copy, then the window tokens (first layer) and "
+                       "the main query",
             "copy_ms_per_step": copy_ms, "copy_gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
             "copy_note": "the step's copies alone, back to back on one stream (no kernels)",
             "step": "cuda graph" if graph is not None else "eager",

@@ -158,24 +158,35 @@ class GroupRunner:
                 out.extend(b * self.swa_cap + (synth.SWA_WINDOW - 1) + t for t in range(wl.T))
         return out
 
-    def _write_jobs(self):
-        """csa2_quantize_kv_batch jobs of a step's writes: (entry jobs, window jobs, query jobs)."""
+    def _write_jobs(self, kv=None, ik=None, win=None, iq=None):
+        """csa2_quantize_kv_batch jobs of a step's writes: (entry jobs, window jobs, query jobs),
+        from the runner's device inputs or from the given device tensors of the same shapes (kv,
+        ik: the new entries' latents and indexer keys; win: the window tokens; iq: a list with
+        each Full/Reindex layer's indexer query, None elsewhere)."""
         def fp4(x, codes, scales, cs, ss, dst=None):
             dt = DTYPE_F32 if x.dtype == torch.float32 else DTYPE_BF16
             return quant_job(FMT_FP4, x, dt, x.shape[0], x.shape[1], x.stride(0), codes, cs, scales, ss, dst)
+        kv = self.step_kv if kv is None else kv
+        ik = self.step_ik if ik is None else ik
+        win = self.step_win_lat if win is None else win
         entries, windows, queries = [], [], []
         if self.step_rows is not None:
-            entries.append(fp4(self.step_kv, self.kv, self.kv[:, 256:], KV_ROW, KV_ROW, self.step_rows))
-            entries.append(fp4(self.step_ik, self.k_codes, self.k_scales, 32, 4, self.step_rows))
+            entries.append(fp4(kv, self.kv, self.kv[:, 256:], KV_ROW, KV_ROW, self.step_rows))
+            entries.append(fp4(ik, self.k_codes, self.k_scales, 32, 4, self.step_rows))
         if self.step_win_rows is not None:
-            x = self.step_win_lat
-            windows.append(quant_job(FMT_FP8_TOKEN, x, DTYPE_F32, x.shape[0], x.shape[1], x.stride(0),
+            windows.append(quant_job(FMT_FP8_TOKEN, win, DTYPE_F32, win.shape[0], win.shape[1], win.stride(0),
                                      self.swa_codes_all, self.swa_codes_all.stride(0), self.swa_scale_all, 4,
                                      self.step_win_rows))
-        for ld in self.layer_data:
+        for l, ld in enumerate(self.layer_data):
             if "iq_f32" in ld:
-                queries.append(fp4(ld["iq_f32"], ld["iq_codes"], ld["iq_scales"], 32, 4))
+                x = ld["iq_f32"] if iq is None or iq[l] is None else iq[l]
+                queries.append(fp4(x, ld["iq_codes"], ld["iq_scales"], 32, 4))
         return entries, windows, queries
+
+    def write_jobs(self, kv=None, ik=None, win=None, iq=None):
+        """The step's quantise-on-write jobs (entries, windows, queries) reading the given device
+        tensors instead of the runner's own inputs (see _write_jobs)."""
+        return self._write_jobs(kv, ik, win, iq)
 
     def _group_desc(self) -> GroupDesc:
         wl = self.wl
