@@ -58,8 +58,8 @@ def _peaks():
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), together with the SHA-256 of the kernel
 # source it was taken on: when the source has changed since, the figure is stale and the line
 # reports traffic null.
-ATTN_TRAFFIC = {"bytes": 28976896 + 129536, "source_sha256": "3ca711dae2a7d0893d1e8f68af059661a851b4bf8ca3de5491a1a9a176b57cdd",
-                "capture": "ncu --set full --clock-control none -k 'regex:attn_tc_kernel|index_score_pipe|topk_cluster' "
+ATTN_TRAFFIC = {"bytes": 28974848 + 140288, "source_sha256": "3e6a7affcd4af519d0fbc9da779944ec81806f7a7b723d8fb2c6e95a1026f79b",
+                "capture": "ncu --set full --clock-control none -k 'regex:attn_tc_kernel|attn_tc_merge' "
                            "-s 8 -c 3 python bench.py --config 1 --entries 16384 --steps 2 --warmup 3 --quick "
                            "--no-cpu-baseline --eager (dram__bytes_read.sum + dram__bytes_write.sum of attn_tc_kernel; "
                            "the attention's bytes do not depend on the entry count)"}
