@@ -502,16 +502,11 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     Steps do not overlap: the copy stream starts a step after the previous step's work."""
     from compressed_sparse_attention_quantize_b200 import runtime, synth
     wl = runner.wl
-    def pinned_copy(t):
-        # the library's host buffers (csa2_host_alloc: page-locked, 2 MB pages): copies from
-        # 4 KB-page buffers ran at 32 GB/s and slowed the group beside them by 10-50 %
-        h = csa2.host_empty(t.shape, t.dtype)
-        h.copy_(t)
-        return h
-
     class Stage:
-        """Several small inputs in one host buffer and one device buffer, so that they cross in
-        one copy (every copy pays a few microseconds before its first byte lands)."""
+        """Several inputs in one host buffer from the library's allocator (csa2_host_alloc:
+        page-locked, 2 MB pages; copies from 4 KB-page buffers ran at 32 GB/s and slowed the group
+        beside them by 10-50 %) and one device buffer, so that they cross in one copy (every copy
+        pays a fixed cost before its first byte lands)."""
 
         def __init__(self, parts):
             offs, n = [], 0
@@ -520,26 +515,28 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
                 n += (t.numel() * t.element_size() + 255) // 256 * 256
             self.host = csa2.host_empty((n,), torch.uint8)
             self.dev = torch.empty((n,), dtype=torch.uint8, device="cuda")
-            self.views, self.bytes = {}, 0
+            self.views, self.bytes, self.span = {}, 0, {}
             for (name, t), o in zip(parts, offs):
                 nb = t.numel() * t.element_size()
                 self.host[o:o + nb].view(t.dtype).view(t.shape).copy_(t)
                 self.views[name] = self.dev[o:o + nb].view(t.dtype).view(t.shape)
+                self.span[name] = (o, o + nb)
                 self.bytes += nb
 
-        def copy(self):
-            self.dev.copy_(self.host, non_blocking=True)
+        def copy(self, first=None, last=None):
+            """One copy of all parts, or of the parts from `first` through `last`."""
+            if first is None:
+                self.dev.copy_(self.host, non_blocking=True)
+            else:
+                lo, hi = self.span[first][0], self.span[last][1]
+                self.dev[lo:hi].copy_(self.host[lo:hi], non_blocking=True)
 
-    host = []
     h2d = 0
-    stages = [None] * len(runner.modes)      # per layer: its indexer inputs (+ the new entries)
-    win_stage = None
+    L = len(runner.modes)
+    stages = [None] * L                      # per layer: its indexer inputs (+ the new entries)
     with gpu_local_cpus(torch) as local:
         for l, m in enumerate(runner.modes):
             ld = runner.layer_data[l]
-            hq = pinned_copy(ld["q"].cpu())
-            host.append({"q": hq})
-            h2d += hq.numel() * 2
             parts = []
             if m != "U":
                 iq = np.stack([synth.index_query(wl, l, b) for b in range(wl.B)]).reshape(-1, 64)
@@ -549,19 +546,27 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
             if parts:
                 stages[l] = Stage(parts)
                 h2d += stages[l].bytes
-        if writes and runner.step_win_rows is not None:
-            win_stage = Stage([("win", runner.step_win_lat.cpu())])
-            h2d += win_stage.bytes
+        # the window tokens and every layer's main query in one buffer, copied in groups that grow
+        # along the layers: [window, q0], [q1], [q2, q3], [q4, q5], ...: fewer copies (each has a
+        # fixed cost), while the first layers still get their query early
+        has_win = writes and runner.step_win_rows is not None
+        bulk = Stage(([("win", runner.step_win_lat.cpu())] if has_win else [])
+                     + [(f"q{l}", runner.layer_data[l]["q"].cpu()) for l in range(L)])
+        h2d += bulk.bytes
+        groups, l = [], 0
+        while l < L:
+            n = 1 if l < 2 else 2
+            groups.append(list(range(l, min(L, l + n))))
+            l += n
         out_last = runner.layer_data[-1]["out"]
         out_host = csa2.host_empty(out_last.shape, out_last.dtype)
-    pages = host_page_report([e["q"] for e in host] + [st.host for st in stages if st is not None]
-                             + ([win_stage.host] if win_stage else []) + [out_host])
+    pages = host_page_report([bulk.host] + [st.host for st in stages if st is not None] + [out_host])
     d2h = out_host.numel() * out_host.element_size()
     # quantise-on-write jobs and indexer weights read the device halves of the stages
     st0 = stages[0]
     entry_jobs, window_jobs, query_jobs = runner.write_jobs(
         kv=st0.views.get("kv") if st0 else None, ik=st0.views.get("ik") if st0 else None,
-        win=win_stage.views["win"] if win_stage else None,
+        win=bulk.views["win"] if has_win else None,
         iq=[st.views["iq"] if st is not None and "iq" in st.views else None for st in stages])
     qjob = iter(query_jobs)
     stage_jobs = []
@@ -570,10 +575,14 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
         if l == 0 and writes:
             jobs += entry_jobs
         stage_jobs.append(jobs)
-    saved_iw = [L.iw for L in runner.layer_descs]
+    saved_iw = [d.iw for d in runner.layer_descs]
+    saved_q = [d.q for d in runner.layer_descs]
     for l, st in enumerate(stages):
         if st is not None and "iw" in st.views:
             runner.layer_descs[l].iw = st.views["iw"].data_ptr()
+    for l in range(L):
+        runner.layer_descs[l].q = bulk.views[f"q{l}"].data_ptr()
+    group_of = {g[0]: g for g in groups}
     cur = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
     ready = [torch.cuda.Event() for _ in runner.modes]
@@ -586,7 +595,6 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
         copy_stream.wait_stream(main)
         with torch.cuda.stream(copy_stream):
             for l, m in enumerate(runner.modes):
-                ld, e = runner.layer_data[l], host[l]
                 # a layer's indexer inputs first, and before the first layer the step's new
                 # entries (the indexer scores them), in one copy: the indexer starts while the
                 # main query and the window tokens, which only the attention needs, are still
@@ -596,22 +604,24 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
                 if stage_jobs[l]:
                     csa2.csa2_quantize_kv_batch(stage_jobs[l], stream=copy_stream)
                 ready[l].record(copy_stream)
-                if l == 0 and win_stage is not None:
-                    win_stage.copy()
-                    csa2.csa2_quantize_kv_batch(window_jobs, stream=copy_stream)
-                ld["q"].copy_(e["q"], non_blocking=True)
+                if l in group_of:                     # this layer starts a group of main queries
+                    g = group_of[l]
+                    first = "win" if (l == 0 and has_win) else f"q{g[0]}"
+                    bulk.copy(first, f"q{g[-1]}")
+                    if first == "win":
+                        csa2.csa2_quantize_kv_batch(window_jobs, stream=copy_stream)
                 attn_ready[l].record(copy_stream)
         runner.run()
         out_host.copy_(out_last, non_blocking=True)
 
     def copies_only():
         """The step's host->device and device->host copies alone (same buffers, same order)."""
-        for l in range(len(runner.modes)):
+        for l in range(L):
             if stages[l] is not None:
                 stages[l].copy()
-            if l == 0 and win_stage is not None:
-                win_stage.copy()
-            runner.layer_data[l]["q"].copy_(host[l]["q"], non_blocking=True)
+            if l in group_of:
+                g = group_of[l]
+                bulk.copy("win" if (l == 0 and has_win) else f"q{g[0]}", f"q{g[-1]}")
         out_host.copy_(out_last, non_blocking=True)
 
     graph = None
@@ -641,15 +651,16 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     finally:
         torch.cuda.synchronize()
         runner.set_layer_events(None, None)
-        for L, p in zip(runner.layer_descs, saved_iw):
-            L.iw = p
+        for d, p, pq in zip(runner.layer_descs, saved_iw, saved_q):
+            d.iw, d.q = p, pq
     return {"value": runner.rows * steps / (sum(ms) / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": sum(ms) / steps,
             "ms_per_step_min_median_max": [min(ms), statistics.median(ms), max(ms)],
-            "overlap": "input copies on a second stream, per layer: indexer inputs (and, before the first "
-                       "layer, the step's new entries) in one copy, then the window tokens (first layer) and "
-                       "the main query",
+            "overlap": "input copies on a second stream: per layer its indexer inputs (and, before the first "
+                       "layer, the step's new entries) in one copy; the window tokens and main queries in "
+                       "growing groups [window, q0], [q1], [q2, q3], ...",
+            "copies_per_step": sum(st is not None for st in stages) + len(groups) + 1,
             "copy_ms_per_step": copy_ms, "copy_gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
             "copy_note": "the step's copies alone, back to back on one stream (no kernels)",
             "step": "cuda graph" if graph is not None else "eager",

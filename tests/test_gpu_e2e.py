@@ -30,5 +30,6 @@ def test_e2e_step_matches_device_step(config, kw):
         assert torch.equal(a, ld["out"]), l
     # the layer descriptors point at the runner's own buffers again
     for L, ld in zip(runner.layer_descs, runner.layer_data):
+        assert L.q == ld["q"].data_ptr()
         if "iw" in ld:
             assert L.iw == ld["iw"].data_ptr()
