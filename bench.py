@@ -492,6 +492,17 @@ def topk_side_reference(torch, csa2, wl, flush, reps=10):
             "note": "csa2_topk_merge_shards (one shard) vs torch.topk(sorted=False); L2 flushed before each call"}
 
 
+def query_copy_groups(n_layers):
+    """The layers whose main queries cross in one copy, in order: the first two layers alone, then
+    pairs ([0], [1], [2, 3], [4, 5], ...): fewer copies, while the first layers' queries land early."""
+    groups, l = [], 0
+    while l < n_layers:
+        n = 1 if l < 2 else 2
+        groups.append(list(range(l, min(n_layers, l + n))))
+        l += n
+    return groups
+
+
 def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
     """The metric through csa2_layer_group with host buffers.  Per step: every layer's main query
     (bf16) and indexer query/weights (fp32) are copied from pinned host memory on a copy stream,
@@ -553,11 +564,7 @@ def e2e_measure(torch, csa2, runner, steps, warmup, flush, writes=False):
         bulk = Stage(([("win", runner.step_win_lat.cpu())] if has_win else [])
                      + [(f"q{l}", runner.layer_data[l]["q"].cpu()) for l in range(L)])
         h2d += bulk.bytes
-        groups, l = [], 0
-        while l < L:
-            n = 1 if l < 2 else 2
-            groups.append(list(range(l, min(L, l + n))))
-            l += n
+        groups = query_copy_groups(L)
         out_last = runner.layer_data[-1]["out"]
         out_host = csa2.host_empty(out_last.shape, out_last.dtype)
     pages = host_page_report([bulk.host] + [st.host for st in stages if st is not None] + [out_host])
