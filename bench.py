@@ -54,30 +54,43 @@ def _peaks():
 # ------------------------------------------------------------------------------------------
 # algorithmic work per call (bytes that must move; flops of the contraction)
 # ------------------------------------------------------------------------------------------
-# DRAM bytes (read + write) of one attn_tc_kernel launch on the 128K decode workload, from one ncu
+# DRAM bytes (read + write) of one attn_tc_kernel launch per decode workload, each from one ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), together with the SHA-256 of the kernel
-# source it was taken on: when the source has changed since, the figure is stale and the line
-# reports traffic null.
-ATTN_TRAFFIC = {"bytes": 28974848 + 140288, "source_sha256": "3e6a7affcd4af519d0fbc9da779944ec81806f7a7b723d8fb2c6e95a1026f79b",
-                "capture": "ncu --set full --clock-control none -k 'regex:attn_tc_kernel|attn_tc_merge' "
-                           "-s 8 -c 3 python bench.py --config 1 --entries 16384 --steps 2 --warmup 3 --quick "
-                           "--no-cpu-baseline --eager (dram__bytes_read.sum + dram__bytes_write.sum of attn_tc_kernel; "
-                           "the attention's bytes do not depend on the entry count)"}
+# source they were taken on: when the source has changed since, the figures are stale and the
+# line reports traffic null.
+ATTN_TRAFFIC_SHA256 = "3e6a7affcd4af519d0fbc9da779944ec81806f7a7b723d8fb2c6e95a1026f79b"
+ATTN_TRAFFIC = {
+    "decode_128k_b32_F5U": {
+        "bytes": 28974848 + 140288,
+        "capture": "ncu --set full --clock-control none -k 'regex:attn_tc_kernel|attn_tc_merge' "
+                   "-s 8 -c 3 python bench.py --config 1 --entries 16384 --steps 2 --warmup 3 --quick "
+                   "--no-cpu-baseline --eager (dram__bytes_read.sum + dram__bytes_write.sum of attn_tc_kernel; "
+                   "the attention's bytes do not depend on the entry count)"},
+    "decode_1m_b4_F5U": {
+        "bytes": 3815296,                       # read 3817472 and 3813120, written 0
+        "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                   "--clock-control none -k regex:attn_tc_kernel -s 6 -c 2 python bench.py --config 3 "
+                   "--steps 3 --warmup 3 --quick --no-cpu-baseline --eager (mean of the two launches' "
+                   "dram__bytes_read.sum + dram__bytes_write.sum)"},
+}
 ATTN_SOURCE = os.path.join(ROOT, "compressed_sparse_attention_quantize_b200", "csrc", "attn_tc.cu")
 
 
-def attn_traffic():
-    """(bytes or None, note): the captured DRAM traffic of one attention launch if it was taken
-    on the current kernel source."""
+def attn_traffic(workload):
+    """(bytes or None, note): the captured DRAM traffic of one attention launch on `workload` if
+    it was taken on the current kernel source."""
     import hashlib
+    rec = ATTN_TRAFFIC.get(workload)
+    if rec is None:
+        return None, "no capture on this workload"
     try:
         with open(ATTN_SOURCE, "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
     except OSError:
         return None, "kernel source not found"
-    if ATTN_TRAFFIC["bytes"] is None or ATTN_TRAFFIC["source_sha256"] != sha:
+    if sha != ATTN_TRAFFIC_SHA256:
         return None, "no capture of the current kernel source"
-    return ATTN_TRAFFIC["bytes"], ATTN_TRAFFIC["capture"]
+    return rec["bytes"], rec["capture"]
 
 
 def visible_counts(wl, b):
@@ -722,9 +735,7 @@ def roofline(wl, kernels, peaks):
     dom = max(kernels, key=lambda k: kernels[k]["share"] or 0)
     k = kernels[dom]
     if dom == "sparse_attn":
-        traffic, note = attn_traffic()
-        if wl.name != "decode_128k_b32_F5U" and traffic is not None:
-            traffic, note = None, "captured on the 128K decode workload only"
+        traffic, note = attn_traffic(wl.name)
         roof = {"kernel": "csa2_sparse_attn", "bound": "tensor", "achieved": k["achieved_tflops"],
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": k["achieved_tflops"] / tc_peak,
                 "traffic": traffic, "traffic_source": note,

@@ -33,3 +33,19 @@ def test_host_page_report_counts_the_mapping():
     assert bench.host_page_report([torch.empty(0)]) == {"rss_kb": 0, "anon_huge_kb": 0, "nodes": {}}
     del t, a
     m.close()
+
+
+def test_attention_traffic_lookup_by_workload():
+    """The roofline's measured DRAM traffic is per workload and tied to the kernel source it was
+    captured on: a workload with no capture, or a changed source, gives None with a reason."""
+    for name in ("decode_128k_b32_F5U", "decode_1m_b4_F5U"):
+        got, note = bench.attn_traffic(name)
+        assert (got is None and "current kernel source" in note) or (got > 0 and "ncu" in note)
+    got, note = bench.attn_traffic("reindex_256k_b16_FIUIUU")
+    assert got is None and note == "no capture on this workload"
+    saved = bench.ATTN_TRAFFIC_SHA256
+    try:
+        bench.ATTN_TRAFFIC_SHA256 = "0" * 64
+        assert bench.attn_traffic("decode_1m_b4_F5U") == (None, "no capture of the current kernel source")
+    finally:
+        bench.ATTN_TRAFFIC_SHA256 = saved
