@@ -1,4 +1,5 @@
-// Top-K (and pool) selection by a cluster of 8 (or, for few rows, 16) CTAs per query row.
+// Top-K (and pool) selection by a cluster of 8 CTAs of 512 threads per query row, or, for few
+// rows, of 16 CTAs of 1024 threads (one CTA per SM) when all the rows' clusters fit on the GPU at once.
 //
 // [A] page "DeepSeek V4.1 Flash深度解析：KV缓存压缩437倍的技术路径", section
 // "压缩吸收注意力（二代）": the indexer keeps 2048 blocks per query and the first layer's
@@ -25,7 +26,8 @@ namespace cg = cooperative_groups;
 
 constexpr int kCluster = 8;                        // the portable cluster size
 constexpr int kClusterWide = 16;                   // for few rows: twice the SMs per row
-constexpr int kThreads = 512;
+constexpr int kThreads = 512;                      // two CTAs per SM (8-CTA clusters)
+constexpr int kThreadsWide = 1024;                 // one CTA per SM (16-CTA clusters, few rows)
 constexpr int kMaxChunk = 32768;                   // keys per CTA (128 KB of shared memory)
 
 struct Args {
@@ -65,10 +67,12 @@ struct alignas(16) Shared {
     int warp_sums[33];
 };
 
-static_assert(kThreads % 32 == 0 && kThreads <= 1024, "block scans need whole warps, at most 32");
-static_assert(kThreads >= 256, "one thread per histogram bin");
+static_assert(kThreads % 32 == 0 && kThreadsWide % 32 == 0 && kThreadsWide <= 1024,
+              "block scans need whole warps, at most 32");
+static_assert(kThreads >= 256 && kThreadsWide >= 256, "one thread per histogram bin");
 // Block-wide exclusive sum of per-thread counts in thread order (warp 0 scans one partial per
-// warp and zero for lanes beyond the warp count); total = the block's sum.
+// warp and zero for lanes beyond the warp count); total = the block's sum.  kT = blockDim.x.
+template <int kT>
 CSA2_D int block_excl_sum(int v, int *ws, int &total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = v;
@@ -80,7 +84,7 @@ CSA2_D int block_excl_sum(int v, int *ws, int &total) {
     if (lane == 31) ws[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int w = lane < kThreads / 32 ? ws[lane] : 0;
+        const int w = lane < kT / 32 ? ws[lane] : 0;
         int wincl = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -137,7 +141,8 @@ CSA2_D void choose_digit(const Shared &S, int shift, uint32_t &prefix, uint32_t 
 }
 
 // One selection of the k largest keys of the row (k < n): writes ids ascending to out[0..k).
-template <int kC>
+// kC CTAs per cluster, kT threads per CTA.
+template <int kC, int kT>
 CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *keys, int chunk_len,
                            int64_t chunk_base, const int32_t *ids, int k, int32_t *out) {
     const int rank = (int)cl.block_rank();
@@ -146,11 +151,11 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         unsigned int *h = S.hist[pass & 1];
-        for (int i = threadIdx.x; i < 256; i += kThreads) h[i] = 0u;
+        for (int i = threadIdx.x; i < 256; i += kT) h[i] = 0u;
         __syncthreads();
         // warp-aggregated: lanes with the same bin add once (the top digits of nearby scores
         // collide heavily, which would serialise plain shared-memory atomics)
-        for (int base = 0; base < chunk_len; base += kThreads) {
+        for (int base = 0; base < chunk_len; base += kT) {
             const int i = base + threadIdx.x;
             const uint32_t key = i < chunk_len ? keys[i] : 0u;
             const bool in = i < chunk_len && (key & mask) == prefix;
@@ -179,7 +184,7 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
     // ordered compaction of this chunk: thread t owns the consecutive keys [t*per, (t+1)*per).
     // One block scan of (above, equal) counts packed in 16-bit halves gives the thread's place
     // among this CTA's selections; the CTA's place follows from the lower-ranked CTAs' totals.
-    const int per = ((chunk_len + kThreads - 1) / kThreads) | 1;     // odd: a warp's lanes hit 32 banks
+    const int per = ((chunk_len + kT - 1) / kT) | 1;     // odd: a warp's lanes hit 32 banks
     const int i0 = min(chunk_len, threadIdx.x * per), i1 = min(chunk_len, i0 + per);
     int my_gt = 0, my_eq = 0;
     for (int i = i0; i < i1; ++i) {
@@ -188,7 +193,7 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
         my_eq += key == thr;
     }
     int tot;
-    const int pre = block_excl_sum((my_gt << 16) | my_eq, S.warp_sums, tot);   // counts < 2^16
+    const int pre = block_excl_sum<kT>((my_gt << 16) | my_eq, S.warp_sums, tot);   // counts < 2^16
     const int gt_pre = pre >> 16, eq_pre = pre & 0xFFFF;
     if (threadIdx.x == 0) { S.counts[0] = tot >> 16; S.counts[1] = tot & 0xFFFF; }
     cl.sync();
@@ -216,9 +221,9 @@ CSA2_D void select_cluster(cg::cluster_group &cl, Shared &S, const uint32_t *key
     cl.sync();                                      // counts may be reused by the next selection
 }
 
-// Launched with a cluster of kC CTAs per row (launch attribute).
-template <int kC>
-__global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(Args a) {
+// Launched with a cluster of kC CTAs of kT threads per row (launch attribute).
+template <int kC, int kT>
+__global__ void __launch_bounds__(kT, 1024 / kT) topk_cluster_kernel(Args a) {
     extern __shared__ __align__(16) uint32_t keys[];
     __shared__ Shared S;
     cg::cluster_group cl = cg::this_cluster();
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(Args a) {
     const int clen = (int)max((int64_t)0, min((int64_t)chunk, n - cbase));
     const float *s = a.scores + (int64_t)lr * a.score_stride;
     const int32_t *ids = a.cand ? a.cand + (int64_t)r * a.cand_stride : nullptr;
-    for (int i = threadIdx.x; i < clen; i += kThreads) keys[i] = float_key(s[cbase + i]);
+    for (int i = threadIdx.x; i < clen; i += kT) keys[i] = float_key(s[cbase + i]);
     __syncthreads();
     for (int which = 0; which < 2; ++which) {
         const int k = which == 0 ? a.K : a.P;
@@ -241,16 +246,16 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(Args a) {
         int32_t *cnt = which == 0 ? a.out_cnt : a.out_pool_len;
         const int c = (int)min((int64_t)k, n);
         if (n <= k) {
-            for (int i = threadIdx.x; i < clen; i += kThreads) {
+            for (int i = threadIdx.x; i < clen; i += kT) {
                 const int64_t j = cbase + i;
                 out[j] = ids ? ids[j] : (int32_t)j;
             }
         } else {
-            select_cluster<kC>(cl, S, keys, clen, cbase, ids, k, out);
+            select_cluster<kC, kT>(cl, S, keys, clen, cbase, ids, k, out);
         }
         // padding: rank 0 writes -1 to out[c..k)
         if (rank == 0) {
-            for (int i = c + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+            for (int i = c + threadIdx.x; i < k; i += kT) out[i] = -1;
             if (threadIdx.x == 0 && cnt) cnt[r] = c;
         }
     }
@@ -263,19 +268,21 @@ constexpr size_t smem_of(int chunk) { return (size_t)chunk * sizeof(uint32_t); }
 
 int64_t topk_cluster_max_n() { return (int64_t)tkc::kCluster * tkc::kMaxChunk; }
 
-static SmemLimit g_topk_smem, g_topk_smem_wide;
-static std::atomic<int> g_topk_wide_ok[kMaxDevices];      // 0 unknown, 1 yes, -1 no
+static SmemLimit g_topk_smem, g_topk_smem_wide, g_topk_smem_wide_full;
+// per device: how many 16-CTA clusters can be resident at once (0 unknown, -1 none), for CTAs of
+// 512 threads ([0]) and of 1024 threads ([1])
+static std::atomic<int> g_topk_wide_slots[2][kMaxDevices];
 
-template <int kC>
+template <int kC, int kT>
 static cudaError_t launch_topk_cluster_n(const tkc::Args &a, int nrows, int64_t max_n, SmemLimit &lim,
                                          cudaStream_t st) {
     const int chunk = (int)((max_n + kC - 1) / kC);
     const size_t smem = tkc::smem_of(chunk > 0 ? chunk : 1);
-    cudaError_t e = ensure_smem_limit(lim, tkc::topk_cluster_kernel<kC>, (int)smem);
+    cudaError_t e = ensure_smem_limit(lim, tkc::topk_cluster_kernel<kC, kT>, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(nrows * kC));
-    cfg.blockDim = dim3(tkc::kThreads);
+    cfg.blockDim = dim3(kT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -285,43 +292,48 @@ static cudaError_t launch_topk_cluster_n(const tkc::Args &a, int nrows, int64_t 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tkc::topk_cluster_kernel<kC>, a);
+    e = cudaLaunchKernelEx(&cfg, tkc::topk_cluster_kernel<kC, kT>, a);
     note_launches(1);
     return e;
 }
 
-// Whether clusters of 16 CTAs with `smem` bytes each can be resident on the current device (the
-// size is not portable: it needs the opt-in attribute and enough SMs per GPC).  Once per device.
-static bool topk_wide_clusters(size_t smem) {
+// How many clusters of 16 CTAs of kT threads with `smem` bytes each can be resident at once on
+// the current device (the size is not portable: it needs the opt-in attribute and enough SMs per
+// GPC); 0 when none.  Queried once per device and thread count.
+template <int kT>
+static int topk_wide_slots(size_t smem) {
+    constexpr int kC = tkc::kClusterWide;
     const int dev = current_device();
-    if (dev < 0) return false;
-    const int known = g_topk_wide_ok[dev].load(std::memory_order_acquire);
-    if (known != 0) return known > 0;
+    if (dev < 0) return 0;
+    std::atomic<int> &slot = g_topk_wide_slots[kT == tkc::kThreadsWide ? 1 : 0][dev];
+    const int known = slot.load(std::memory_order_acquire);
+    if (known != 0) return known > 0 ? known : 0;
     std::lock_guard<std::mutex> lock(settings_mutex());
-    bool ok = cudaFuncSetAttribute(tkc::topk_cluster_kernel<tkc::kClusterWide>,
+    bool ok = cudaFuncSetAttribute(tkc::topk_cluster_kernel<kC, kT>,
                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-              cudaFuncSetAttribute(tkc::topk_cluster_kernel<tkc::kClusterWide>,
+              cudaFuncSetAttribute(tkc::topk_cluster_kernel<kC, kT>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)tkc::smem_of(tkc::kMaxChunk)) == cudaSuccess;
+    int clusters = 0;
     if (ok) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(tkc::kClusterWide);
-        cfg.blockDim = dim3(tkc::kThreads);
+        cfg.gridDim = dim3(kC);
+        cfg.blockDim = dim3(kT);
         cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = tkc::kClusterWide;
+        attr[0].val.clusterDim.x = kC;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        int clusters = 0;
-        ok = cudaOccupancyMaxActiveClusters(&clusters, tkc::topk_cluster_kernel<tkc::kClusterWide>, &cfg) ==
-                 cudaSuccess && clusters > 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, tkc::topk_cluster_kernel<kC, kT>, &cfg) !=
+            cudaSuccess)
+            clusters = 0;
     }
     (void)cudaGetLastError();                   // a refused query leaves no error behind
-    g_topk_wide_ok[dev].store(ok ? 1 : -1, std::memory_order_release);
-    return ok;
+    slot.store(clusters > 0 ? clusters : -1, std::memory_order_release);
+    return clusters > 0 ? clusters : 0;
 }
 
 // Selection for rows [row0, row0+nrows) from scores in global memory (max_n <= topk_cluster_max_n()).
@@ -338,12 +350,20 @@ cudaError_t launch_topk_cluster(const float *scores, int64_t score_stride, const
     a.P = P; a.out_pool = out_pool; a.out_pool_len = out_pool_len;
     // few rows: clusters of 16 put twice the SMs on each row when the grid still has one CTA per
     // SM (measured: 4 rows x 256K scores 78 -> 59 us; 16 rows x 64K with a 16K pool, two CTAs per
-    // SM, was slower at 16 than at 8)
+    // SM, was slower at 16 than at 8).  Such a CTA has its SM to itself, so it runs 1024 threads
+    // when every row's cluster can be resident at once (4 rows x 147K-254K scores: index + top-K
+    // 56.4 -> 52.3 us; 16 rows x 64K with a 16K pool on 8-CTA clusters of 1024 threads: no change).
+    const int64_t nsm = device_sm_count();
     const int64_t wide_chunk = (max_n + tkc::kClusterWide - 1) / tkc::kClusterWide;
-    if ((int64_t)nrows * tkc::kClusterWide <= (int64_t)device_sm_count() && wide_chunk >= 1024 &&
-        topk_wide_clusters(tkc::smem_of((int)wide_chunk)))
-        return launch_topk_cluster_n<tkc::kClusterWide>(a, nrows, max_n, g_topk_smem_wide, st);
-    return launch_topk_cluster_n<tkc::kCluster>(a, nrows, max_n, g_topk_smem, st);
+    if ((int64_t)nrows * tkc::kClusterWide <= nsm && wide_chunk >= 1024) {
+        const size_t smem = tkc::smem_of((int)wide_chunk);
+        if (nrows <= topk_wide_slots<tkc::kThreadsWide>(smem))
+            return launch_topk_cluster_n<tkc::kClusterWide, tkc::kThreadsWide>(a, nrows, max_n,
+                                                                               g_topk_smem_wide_full, st);
+        if (topk_wide_slots<tkc::kThreads>(smem) > 0)
+            return launch_topk_cluster_n<tkc::kClusterWide, tkc::kThreads>(a, nrows, max_n, g_topk_smem_wide, st);
+    }
+    return launch_topk_cluster_n<tkc::kCluster, tkc::kThreads>(a, nrows, max_n, g_topk_smem, st);
 }
 
 }  // namespace csa2
