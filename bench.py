@@ -753,6 +753,22 @@ def roofline(wl, kernels, peaks):
             "peak_source": f"{peak_src} hbm_gbs"}
 
 
+def max_over_ranks(torch, dist, value, world, device="cuda"):
+    """The largest of the ranks' values: a multi-GPU time is the slowest rank's.  One rank: the
+    value itself, with no collective."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(rows_per_rank, world, steps, total_ms):
+    """Queries per second of the whole job: every rank's rows for every step, over the slowest
+    rank's total time."""
+    return rows_per_rank * world * steps / (total_ms / 1e3)
+
+
 def measure_workload(torch, csa2, args, wl, world, rank, local, peaks, flush, detail=True):
     """Time the workload's step (graph replays, L2 flushed before each) and, with detail, the
     per-call breakdown, roofline, e2e and the oracle's CPU baseline."""
@@ -790,14 +806,11 @@ def measure_workload(torch, csa2, args, wl, world, rank, local, peaks, flush, de
     # graph replays do not pass through the library's launch counter: count the graph's kernels
     launches = csa2.csa2_launch_count() - launches0 + graph_kernels * args.steps
     clocks = clk.summary()
-    total_ms = sum(ms)
+    total_ms = max_over_ranks(torch, dist, sum(ms), world)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
     rows = wl.B * wl.T
-    res = {"value": rows * world * args.steps / (total_ms / 1e3), "unit": UNIT,
+    res = {"value": replica_throughput(rows, world, args.steps, total_ms), "unit": UNIT,
            "ms_per_step": total_ms / args.steps, "steps": args.steps, "warmup": args.warmup,
            "gpu_launches": int(launches), "clocks": clocks,
            "config": {"workload": wl.name, "batch_per_gpu": wl.B, "queries_per_sequence": wl.T,
@@ -817,10 +830,8 @@ def measure_workload(torch, csa2, args, wl, world, rank, local, peaks, flush, de
     res["roofline"] = roofline(wl, kernels, peaks)
     e2e = e2e_measure(torch, csa2, runner, max(3, min(args.steps, 10)), 2, flush, writes)
     if world > 1:
-        t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["value"] = rows * world / (float(t.item()) / 1e3)
-        e2e["ms_per_step"] = float(t.item())
+        e2e["ms_per_step"] = max_over_ranks(torch, dist, e2e["ms_per_step"], world)
+        e2e["value"] = replica_throughput(rows, world, 1, e2e["ms_per_step"])
     res["e2e"] = e2e
     softmax_scale = runner.softmax_scale
     del runner

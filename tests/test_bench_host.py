@@ -49,3 +49,45 @@ def test_attention_traffic_lookup_by_workload():
         assert bench.attn_traffic("decode_1m_b4_F5U") == (None, "no capture of the current kernel source")
     finally:
         bench.ATTN_TRAFFIC_SHA256 = saved
+
+
+def _replica_rank(rank, world, port, out_q):
+    import os
+
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # each rank's own total time; the job's time is the slowest rank's
+        own_ms = 10.0 + 7.5 * rank
+        total = bench.max_over_ranks(torch, dist, own_ms, world, device="cpu")
+        out_q.put((rank, total, bench.replica_throughput(32, world, 20, total)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replica_timing_takes_the_slowest_rank_on_two_gloo_ranks():
+    """The multi-GPU bench reports the whole job's queries/s over the slowest rank's time: two gloo
+    ranks on the CPU with different totals both see the larger one."""
+    import socket
+
+    import torch.multiprocessing as mp
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_replica_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for rank, total, value in got:
+        assert total == 17.5
+        assert value == 32 * 2 * 20 / 17.5e-3
+    assert bench.max_over_ranks(torch, None, 3.25, 1) == 3.25       # one rank: no collective
+    assert bench.replica_throughput(32, 1, 20, 6.5) == 32 * 20 / 6.5e-3
