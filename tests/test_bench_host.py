@@ -91,3 +91,19 @@ def test_replica_timing_takes_the_slowest_rank_on_two_gloo_ranks():
         assert value == 32 * 2 * 20 / 17.5e-3
     assert bench.max_over_ranks(torch, None, 3.25, 1) == 3.25       # one rank: no collective
     assert bench.replica_throughput(32, 1, 20, 6.5) == 32 * 20 / 6.5e-3
+
+
+def test_roofline_work_matches_closed_forms_for_the_decode_workloads():
+    """The roofline's numerators (bytes and flops per launch) against the closed forms: per query
+    row, K selected rows of 288 B, 128 window rows of 516 B, Q (bf16) and O (bf16) of H x 512,
+    K ids and H log-sum-exps; 4 x 512 flop per head and key; the Full indexer reads 36 B per
+    visible entry plus H_I x 40 B of query and writes K ids."""
+    from compressed_sparse_attention_quantize_b200 import synth
+    wl1, wl3 = synth.workload(1), synth.workload(3)
+    per_row = 2048 * 288 + 128 * 516 + 64 * 512 * (2 + 2) + 2048 * 4 + 64 * 4
+    assert bench.attn_work(wl1, 2) == (32 * per_row, 32 * 64 * (2048 + 128) * 512 * 4)
+    assert bench.attn_work(wl3, 2) == (4 * per_row, 4 * 64 * (2048 + 128) * 512 * 4)
+    assert bench.attn_work(wl1, 2)[0] == 25452544
+    assert bench.index_work(wl1) == 32 * (32768 * 36 + 8 * 40 + 2048 * 4)
+    assert wl3.B == 4 and all(131072 <= n <= 262144 for n in wl3.n_entries)
+    assert bench.index_work(wl3) == sum(wl3.n_entries) * 36 + 4 * (8 * 40 + 2048 * 4)
